@@ -1,0 +1,359 @@
+#!/usr/bin/env python
+"""Throughput of the MoE expert layer on B200: prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one full layer pass (router, permute, GEMM1 + SwiGLU, GEMM2, combine) over
+one batch of T synthetic tokens already resident in HBM. Under torchrun each rank runs
+its own batch with replicated weights (weak scaling, no data-path collective); the
+step time is the maximum over ranks. L2 is flushed (a 512 MiB write) between timed
+steps, outside the timed events.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (rank 0 only),
+each step a bounded sample of the same workload's tokens.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/s"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="oai_swiglu")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the oracle sample")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ["uuid", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid.lower().replace("gpu-", "")
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS),
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS) or self.uuid not in parts[0].lower():
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle timing
+def oracle_rate(wl, inp_host, seconds: float, max_tokens: int | None = None):
+    """Tokens/s of the fp64 oracle on a sample sized to take about `seconds`."""
+    import numpy as np
+    import oracle
+    from oracle.torch_io import oracle_layer_from_inputs
+    L = oracle_layer_from_inputs(wl, inp_host)
+    t0 = time.perf_counter()
+    L.moe_rows(np.array([0], dtype=np.int32))
+    one = max(time.perf_counter() - t0, 1e-4)
+    n = int(max(1, min(max_tokens or wl.T, wl.T, math.ceil(seconds / one))))
+    toks = np.arange(n, dtype=np.int32)
+    t0 = time.perf_counter()
+    L.moe_rows(toks)
+    dt = time.perf_counter() - t0
+    return n / dt, n, dt, oracle.num_threads()
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    import oracle
+    from grouped_gemm_swiglu_b200 import workloads as W
+    from oracle.torch_io import oracle_layer_from_inputs, host_inputs
+    wl = W.WORKLOADS[args.workload]
+    inp = host_inputs(W.make_inputs(wl, "cpu"))
+    L = oracle_layer_from_inputs(wl, inp)
+    t0 = time.perf_counter()
+    L.moe_rows(np.array([0], dtype=np.int32))
+    one = max(time.perf_counter() - t0, 1e-4)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(wl.T, round(budget / one))))
+    rng = np.random.default_rng(0)
+    times = []
+    for s in range(args.warmup + args.steps):
+        toks = np.sort(rng.choice(wl.T, n, replace=False)).astype(np.int32)
+        t0 = time.perf_counter()
+        L.moe_rows(toks)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+    sec = sum(times) / len(times)
+    value = n / sec
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(wl),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"{n} random tokens of {wl.T} per step ({wl.name}), fp64 oracle"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(wl):
+    return {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "top_k": wl.k,
+            "n_sink": wl.n_sink, "n_shared": wl.n_shared,
+            "weights": "fp8_e4m3_block128" if wl.wdtype == 1 else "bf16",
+            "score": "sigmoid_logsigmoid_lse" if wl.score == 1 else "softmax_renorm",
+            "alpha": wl.alpha, "beta": wl.beta, "limit": None if math.isinf(wl.limit) else wl.limit,
+            "seed": wl.seed, "l2": "flushed between timed steps (512 MiB write, outside the timed events)"}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import grouped_gemm_swiglu_b200 as moe
+    from grouped_gemm_swiglu_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    wl = W.WORKLOADS[args.workload]
+    inp = W.make_inputs(wl, dev)
+    d = moe.MoeDims.of(wl)
+    layer = moe.MoELayer(d, inp["w1"], inp["w2"], inp["w1_scale"], inp["w2_scale"], inp["gate_scale"],
+                         inp["up_scale"])
+    out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    K, Wm = args.steps, args.warmup
+
+    def fwd():
+        layer.forward(inp["logits"], inp["x"], out=out)
+
+    for _ in range(Wm):
+        flush.zero_()
+        fwd()
+    torch.cuda.synchronize(dev)
+    assert layer.status() == 0, moe.status_string(layer.status())
+
+    # ---- timed region: K device-resident steps
+    sampler = ClockSampler(str(torch.cuda.get_device_properties(dev).uuid))
+    sampler.start()
+    time.sleep(0.4)  # let the sampler start before the timed region
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.perf_counter()
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        fwd()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / K
+    ms = max_over_ranks(ms)
+    value = world * wl.T / (ms / 1e3)
+    assert layer.status() == 0, moe.status_string(layer.status())
+
+    # ---- end to end: pinned host inputs in, result out, every step
+    x_h = inp["x"].cpu().pin_memory()
+    lg_h = inp["logits"].cpu().pin_memory()
+    out_h = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    x_d, lg_d = torch.empty_like(inp["x"]), torch.empty_like(inp["logits"])
+    Ke = max(1, min(K, 200))
+    e2e_t = []
+    for s in range(Ke + 3):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        x_d.copy_(x_h, non_blocking=True)
+        lg_d.copy_(lg_h, non_blocking=True)
+        layer.forward(lg_d, x_d, out=out)
+        out_h.copy_(out, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if s >= 3:
+            e2e_t.append(a.elapsed_time(b))
+    e2e_ms = max_over_ranks(sum(e2e_t) / len(e2e_t))
+    h2d = x_h.numel() * x_h.element_size() + lg_h.numel() * lg_h.element_size()
+    d2h = out_h.numel() * out_h.element_size()
+
+    # ---- per-stage times through the four entry points (same stream, events between)
+    fp8 = wl.wdtype == W.WDTYPE_FP8
+    A, G = d.A, d.G
+    st = {}
+    ids = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
+    tw = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
+    sw = torch.empty((wl.T, wl.n_sink), dtype=torch.float32, device=dev) if wl.n_sink else None
+    offsets = torch.empty((G + 1,), dtype=torch.int32, device=dev)
+    perm = torch.empty((A,), dtype=torch.int32, device=dev)
+    inv = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
+    xp = torch.empty((A, wl.H), dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev)
+    xs = torch.empty((wl.H // 128, A), dtype=torch.float32, device=dev) if fp8 else None
+    h = torch.empty((A, wl.I), dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev)
+    hs = torch.empty((wl.I // 128, A), dtype=torch.float32, device=dev) if fp8 else None
+    ws_p = moe.alloc_workspace(d, moe.MOE_WS_PERMUTE, dev)
+    ws_1 = moe.alloc_workspace(d, moe.MOE_WS_GEMM1, dev)
+    ws_2 = moe.alloc_workspace(d, moe.MOE_WS_GEMM2_COMBINE, dev)
+    stages = {
+        "route": lambda: moe.moe_route_topk(inp["logits"], d, ids, tw, sw),
+        "permute": lambda: moe.moe_permute(ids, inp["x"], d, offsets, perm, inv, xp, xs, ws_p),
+        "gemm1_swiglu": lambda: moe.moe_gemm1_swiglu(xp, xs, offsets, inp["w1"], inp["w1_scale"], inp["gate_scale"],
+                                                     inp["up_scale"], d, h, hs, ws_1),
+        "gemm2_combine": lambda: moe.moe_gemm2_combine(h, hs, offsets, inv, tw, sw, inp["w2"], inp["w2_scale"], d,
+                                                       out, ws_2),
+    }
+    Ks = max(1, min(K, 300))
+    acc = {k: 0.0 for k in stages}
+    for s in range(Ks + 3):
+        flush.zero_()
+        marks = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+        marks[0].record(stream)
+        for i, fn in enumerate(stages.values()):
+            fn()
+            marks[i + 1].record(stream)
+        if s >= 3:
+            torch.cuda.synchronize(dev)
+            for i, k in enumerate(stages):
+                acc[k] += marks[i].elapsed_time(marks[i + 1])
+    torch.cuda.synchronize(dev)
+    for k in acc:
+        st[k] = max_over_ranks(acc[k] / Ks)
+    off = offsets.cpu().numpy()
+    used = int(((off[1:] - off[:-1]) > 0).sum())
+
+    # ---- roofline of the dominant kernel (GEMM1 + SwiGLU)
+    hbm, bf16_tf, peak_src = peaks()
+    elt = 1 if fp8 else 2
+    g1_flops = 2.0 * A * wl.H * 2 * wl.I
+    g1_bytes = used * 2 * wl.I * wl.H * elt + A * wl.H * elt + A * wl.I * elt
+    if fp8:
+        g1_bytes += used * (2 * wl.I // 128) * (wl.H // 128) * 4 + A * (wl.H // 128 + wl.I // 128) * 4
+    t1 = st["gemm1_swiglu"] / 1e3
+    tensor_peak = bf16_tf * (2.0 if fp8 else 1.0)
+    ridge = tensor_peak * 1e12 / (hbm * 1e9)
+    if g1_flops / g1_bytes < ridge:
+        roof = {"bound": "hbm", "achieved": g1_bytes / t1 / 1e9, "peak": hbm, "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": g1_flops / t1 / 1e12, "peak": tensor_peak, "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = "grouped_gemm_kernel (GEMM1 + SwiGLU epilogue)"
+    roof["peak_source"] = peak_src + (" (fp8 = 2x measured bf16)" if fp8 else "")
+    roof["algorithmic_bytes"] = g1_bytes
+    roof["algorithmic_flops"] = g1_flops
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": Wm,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8_e4m3" if fp8 else "bf16", "data": "synthetic", "config": config_of(wl),
+            "e2e": {"value": world * wl.T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "roofline": roof, "clocks": clocks, "gpu_launches": 7 * K,
+            "stages_ms": st, "experts_touched": used,
+            "layer_tflops": wl.flops() / (ms / 1e3) / 1e12,
+            "wall_s_timed_region": wall}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle.torch_io import host_inputs
+        rate, n, dt, cores = oracle_rate(wl, host_inputs(inp), args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"first {n} of {wl.T} tokens of {wl.name} ({dt:.1f} s, fp64)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,314 @@
+// api.cu -- the C ABI declared in include/moe_b200.h: argument checks, workspace
+// layout and the launch sequence of the expert layer. Host code only.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "internal.h"
+#include "status.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr int kMaxE = 1024;
+constexpr int kMaxSlots = 32;  // k + n_sink and k + n_shared share one warp
+
+inline size_t al256(size_t b) { return (b + 255) & ~size_t(255); }
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_dims(const moe_dims* d) {
+    if (!d) return MOE_ERR_INVALID_ARG;
+    if (d->T < 0 || d->H <= 0 || d->I <= 0 || d->H % 128 || d->I % 128) return MOE_ERR_INVALID_ARG;
+    if (d->E < 1 || d->E > kMaxE) return MOE_ERR_INVALID_ARG;
+    if (d->k < 1 || d->k > d->E || d->k > kMaxSlots) return MOE_ERR_INVALID_ARG;
+    if (d->n_sink < 0 || d->k + d->n_sink > kMaxSlots) return MOE_ERR_INVALID_ARG;
+    if (d->n_shared < 0 || d->k + d->n_shared > kMaxSlots) return MOE_ERR_INVALID_ARG;
+    if (d->score != MOE_SCORE_SOFTMAX && d->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+    if (d->wdtype != MOE_WDTYPE_BF16 && d->wdtype != MOE_WDTYPE_FP8_E4M3_BLOCK128) return MOE_ERR_INVALID_ARG;
+    if (d->n_sink > 0 && d->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+    if (d->n_sink > 0 && d->n_shared > 0 && d->n_shared != d->n_sink) return MOE_ERR_INVALID_ARG;
+    if (!std::isfinite(d->alpha) || !std::isfinite(d->beta) || !std::isfinite(d->route_scale))
+        return MOE_ERR_INVALID_ARG;
+    if (!(d->limit > 0.f)) return MOE_ERR_INVALID_ARG;  // rejects NaN too; +inf = no clamp
+    const int64_t A = (int64_t)d->T * (d->k + d->n_shared);
+    if (A > INT32_MAX / 2) return MOE_ERR_INVALID_ARG;
+    const int64_t G = (int64_t)d->E + d->n_shared;
+    if (G * 2 * d->I > INT32_MAX / 2 || G * d->H > INT32_MAX / 2) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+int check_arch() {
+    static int verdict[64] = {0};  // 0 unknown, 1 ok, -1 wrong arch
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (dev >= 0 && dev < 64 && verdict[dev]) return verdict[dev] > 0 ? MOE_OK : MOE_ERR_ARCH;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MOE_ERR_CUDA;
+    const int ok = (major == 10) ? 1 : -1;
+    if (dev >= 0 && dev < 64) verdict[dev] = ok;
+    return ok > 0 ? MOE_OK : MOE_ERR_ARCH;
+}
+
+int64_t rows_A(const moe_dims* d) { return (int64_t)d->T * (d->k + d->n_shared); }
+int groups(const moe_dims* d) { return d->E + d->n_shared; }
+size_t act_elt(const moe_dims* d) { return d->wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128 ? 1 : 2; }
+bool is_fp8(const moe_dims* d) { return d->wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128; }
+
+// Sub-buffers of a workspace, as byte offsets from its start.
+struct Layout {
+    size_t ids = 0, w = 0, sw = 0, offsets = 0, perm = 0, inv = 0, xperm = 0, xscale = 0, h = 0, hscale = 0,
+           pscratch = 0, y = 0, total = 0;
+};
+
+Layout layout(const moe_dims* d, int kind) {
+    Layout L;
+    const size_t T = d->T, k = d->k, A = rows_A(d), H = d->H, I = d->I, G = groups(d);
+    size_t off = kWsHeader;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += al256(bytes);
+        return at;
+    };
+    if (kind == MOE_WS_FORWARD) {
+        L.ids = take(T * k * 4);
+        L.w = take(T * k * 4);
+        L.sw = take(T * (size_t)d->n_sink * 4);
+        L.offsets = take((G + 1) * 4);
+        L.perm = take(A * 4);
+        L.inv = take(T * k * 4);
+        L.xperm = take(A * H * act_elt(d));
+        L.xscale = take(is_fp8(d) ? (H / 128) * A * 4 : 0);
+        L.h = take(A * I * act_elt(d));
+        L.hscale = take(is_fp8(d) ? (I / 128) * A * 4 : 0);
+    }
+    if (kind == MOE_WS_FORWARD || kind == MOE_WS_PERMUTE) L.pscratch = take(permute_scratch_bytes(d->T, d->k, d->E));
+    if (kind == MOE_WS_FORWARD || kind == MOE_WS_GEMM2_COMBINE) L.y = take(A * H * 2);
+    L.total = off;
+    return L;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+int check_ws(const void* ws, size_t ws_bytes, const moe_dims* d, int kind) {
+    if (!ws || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < layout(d, kind).total) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+template <class P>
+P* at(void* ws, size_t off) {
+    return reinterpret_cast<P*>(static_cast<char*>(ws) + off);
+}
+
+// The individual steps, after every check has passed.
+int do_route(const float* logits, const moe_dims* d, int32_t* ids, float* w, float* sw, cudaStream_t s) {
+    return cuda_status(launch_router(logits, d->T, d->E, d->n_sink, d->k, d->score, d->route_scale, ids, w, sw, s));
+}
+
+int do_permute(const int32_t* ids, const void* x, const moe_dims* d, int32_t* offsets, int32_t* perm, int32_t* inv,
+               void* xperm, float* xscale, void* scratch, int* status, cudaStream_t s) {
+    return cuda_status(launch_permute(ids, x, d->T, d->H, d->k, d->E, d->n_shared, is_fp8(d), offsets, perm, inv,
+                                      xperm, xscale, scratch, status, s));
+}
+
+int do_gemm1(const void* xperm, const float* xscale, const int32_t* offsets, const void* w1, const float* w1s,
+             const float* gs, const float* us, const moe_dims* d, void* h, float* hs, int* status, cudaStream_t s) {
+    GemmArgs a;
+    a.offsets = offsets;
+    a.G = groups(d);
+    a.A = rows_A(d);
+    a.K = d->H;
+    a.wrows = 2 * d->I;
+    a.n_chunks = d->I / 128;
+    a.up_off = d->I;
+    a.act = xperm;
+    a.act_scale = xscale;
+    a.w = w1;
+    a.w_scale = w1s;
+    a.out = h;
+    a.out_scale = hs;
+    a.out_ld = d->I;
+    a.gate_scale = gs;
+    a.up_scale = us;
+    a.alpha = d->alpha;
+    a.beta = d->beta;
+    a.limit = d->limit;
+    a.status = status;
+    const int bn = gemm_pick_bn(a.A, a.G, true, is_fp8(d));
+    return cuda_status(launch_gemm(a, true, is_fp8(d), bn, s));
+}
+
+int do_gemm2_combine(const void* h, const float* hs, const int32_t* offsets, const int32_t* inv, const float* topk_w,
+                     const float* shared_w, const void* w2, const float* w2s, const moe_dims* d, void* out, void* y,
+                     int* status, cudaStream_t s) {
+    GemmArgs a;
+    a.offsets = offsets;
+    a.G = groups(d);
+    a.A = rows_A(d);
+    a.K = d->I;
+    a.wrows = d->H;
+    a.n_chunks = d->H / 128;
+    a.up_off = 0;
+    a.act = h;
+    a.act_scale = hs;
+    a.w = w2;
+    a.w_scale = w2s;
+    a.out = y;
+    a.out_scale = nullptr;
+    a.out_ld = d->H;
+    a.gate_scale = nullptr;
+    a.up_scale = nullptr;
+    a.alpha = 1.f;
+    a.beta = 0.f;
+    a.limit = INFINITY;
+    a.status = status;
+    const int bn = gemm_pick_bn(a.A, a.G, false, is_fp8(d));
+    int rc = cuda_status(launch_gemm(a, false, is_fp8(d), bn, s));
+    if (rc != MOE_OK) return rc;
+    return cuda_status(launch_combine(y, offsets, inv, topk_w, shared_w, d->T, d->H, d->k, d->E, d->n_shared,
+                                      d->n_sink, out, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_status_string(int status) {
+    switch (status) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported combination";
+        case MOE_ERR_ARCH: return "device is not compute capability 10.x (sm_100a)";
+        case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case MOE_ERR_EXPERT_ID: return "routing id outside [0, E) or repeated within a token";
+        case MOE_ERR_TIMEOUT: return "a pipeline wait exceeded its time limit";
+        case MOE_ERR_CUDA: return "CUDA runtime error";
+        default: return "unknown status";
+    }
+}
+
+int moe_workspace_size(const moe_dims* dims, int kind, size_t* bytes) {
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    int rc = check_dims(dims);
+    if (rc != MOE_OK) return rc;
+    if (kind < MOE_WS_PERMUTE || kind > MOE_WS_FORWARD) return MOE_ERR_INVALID_ARG;
+    *bytes = layout(dims, kind).total;
+    return MOE_OK;
+}
+
+int moe_read_status(const void* ws, int32_t* status, void* stream) {
+    if (!ws || !status) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t v = 0;
+    if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    *status = v;
+    return MOE_OK;
+}
+
+int moe_clear_status(void* ws, void* stream) {
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    return cuda_status(cudaMemsetAsync(ws, 0, kWsHeader, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_route_topk(const float* logits, const moe_dims* d, int32_t* topk_ids, float* topk_w, float* shared_w,
+                   void* stream) {
+    int rc = check_dims(d);
+    if (rc != MOE_OK) return rc;
+    if (d->T > 0 && (!logits || !topk_ids || !topk_w)) return MOE_ERR_INVALID_ARG;
+    if (d->T > 0 && (d->n_sink > 0) != (shared_w != nullptr)) return MOE_ERR_INVALID_ARG;
+    if ((rc = check_arch()) != MOE_OK) return rc;
+    return do_route(logits, d, topk_ids, topk_w, shared_w, static_cast<cudaStream_t>(stream));
+}
+
+int moe_permute(const int32_t* topk_ids, const void* x, const moe_dims* d, int32_t* offsets, int32_t* perm,
+                int32_t* inv_perm, void* x_perm, float* x_scale, void* ws, size_t ws_bytes, void* stream) {
+    int rc = check_dims(d);
+    if (rc != MOE_OK) return rc;
+    if (!offsets) return MOE_ERR_INVALID_ARG;
+    if (d->T > 0) {
+        if (!topk_ids || !x || !perm || !inv_perm || !x_perm) return MOE_ERR_INVALID_ARG;
+        if (is_fp8(d) && !x_scale) return MOE_ERR_INVALID_ARG;
+        if (!aligned(x, 16) || !aligned(x_perm, 16)) return MOE_ERR_INVALID_ARG;
+    }
+    if ((rc = check_ws(ws, ws_bytes, d, MOE_WS_PERMUTE)) != MOE_OK) return rc;
+    if ((rc = check_arch()) != MOE_OK) return rc;
+    const Layout L = layout(d, MOE_WS_PERMUTE);
+    return do_permute(topk_ids, x, d, offsets, perm, inv_perm, x_perm, x_scale, at<void>(ws, L.pscratch),
+                      at<int>(ws, 0), static_cast<cudaStream_t>(stream));
+}
+
+int moe_gemm1_swiglu(const void* x_perm, const float* x_scale, const int32_t* offsets, const void* w1,
+                     const float* w1_scale, const float* gate_scale, const float* up_scale, const moe_dims* d,
+                     void* h, float* h_scale, void* ws, size_t ws_bytes, void* stream) {
+    int rc = check_dims(d);
+    if (rc != MOE_OK) return rc;
+    if (d->T > 0) {
+        if (!x_perm || !offsets || !w1 || !h) return MOE_ERR_INVALID_ARG;
+        if (is_fp8(d) && (!x_scale || !w1_scale || !h_scale)) return MOE_ERR_INVALID_ARG;
+        if (!aligned(x_perm, 16) || !aligned(w1, 16) || !aligned(h, 16)) return MOE_ERR_INVALID_ARG;
+    }
+    if ((rc = check_ws(ws, ws_bytes, d, MOE_WS_GEMM1)) != MOE_OK) return rc;
+    if ((rc = check_arch()) != MOE_OK) return rc;
+    if (d->T == 0) return MOE_OK;
+    return do_gemm1(x_perm, x_scale, offsets, w1, w1_scale, gate_scale, up_scale, d, h, h_scale, at<int>(ws, 0),
+                    static_cast<cudaStream_t>(stream));
+}
+
+int moe_gemm2_combine(const void* h, const float* h_scale, const int32_t* offsets, const int32_t* inv_perm,
+                      const float* topk_w, const float* shared_w, const void* w2, const float* w2_scale,
+                      const moe_dims* d, void* out, void* ws, size_t ws_bytes, void* stream) {
+    int rc = check_dims(d);
+    if (rc != MOE_OK) return rc;
+    if (d->T > 0) {
+        if (!h || !offsets || !inv_perm || !topk_w || !w2 || !out) return MOE_ERR_INVALID_ARG;
+        if ((d->n_sink > 0) != (shared_w != nullptr)) return MOE_ERR_INVALID_ARG;
+        if (is_fp8(d) && (!h_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
+        if (!aligned(h, 16) || !aligned(w2, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+    }
+    if ((rc = check_ws(ws, ws_bytes, d, MOE_WS_GEMM2_COMBINE)) != MOE_OK) return rc;
+    if ((rc = check_arch()) != MOE_OK) return rc;
+    if (d->T == 0) return MOE_OK;
+    const Layout L = layout(d, MOE_WS_GEMM2_COMBINE);
+    return do_gemm2_combine(h, h_scale, offsets, inv_perm, topk_w, shared_w, w2, w2_scale, d, out, at<void>(ws, L.y),
+                            at<int>(ws, 0), static_cast<cudaStream_t>(stream));
+}
+
+int moe_forward(const float* logits, const void* x, const void* w1, const float* w1_scale, const float* gate_scale,
+                const float* up_scale, const void* w2, const float* w2_scale, const moe_dims* d, void* out,
+                int32_t* topk_ids, float* topk_w, float* shared_w, void* ws, size_t ws_bytes, void* stream) {
+    int rc = check_dims(d);
+    if (rc != MOE_OK) return rc;
+    if (d->T > 0) {
+        if (!logits || !x || !w1 || !w2 || !out) return MOE_ERR_INVALID_ARG;
+        if (is_fp8(d) && (!w1_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
+        if (!aligned(x, 16) || !aligned(w1, 16) || !aligned(w2, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+        if (shared_w && d->n_sink == 0) return MOE_ERR_INVALID_ARG;
+    }
+    if ((rc = check_ws(ws, ws_bytes, d, MOE_WS_FORWARD)) != MOE_OK) return rc;
+    if ((rc = check_arch()) != MOE_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const Layout L = layout(d, MOE_WS_FORWARD);
+    int* status = at<int>(ws, 0);
+    int32_t* ids = topk_ids ? topk_ids : at<int32_t>(ws, L.ids);
+    float* w = topk_w ? topk_w : at<float>(ws, L.w);
+    float* sw = d->n_sink > 0 ? (shared_w ? shared_w : at<float>(ws, L.sw)) : nullptr;
+    int32_t* offsets = at<int32_t>(ws, L.offsets);
+    if (d->T == 0) return cuda_status(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (groups(d) + 1), s));
+    float* xscale = is_fp8(d) ? at<float>(ws, L.xscale) : nullptr;
+    float* hscale = is_fp8(d) ? at<float>(ws, L.hscale) : nullptr;
+    if ((rc = do_route(logits, d, ids, w, sw, s)) != MOE_OK) return rc;
+    if ((rc = do_permute(ids, x, d, offsets, at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv), at<void>(ws, L.xperm),
+                         xscale, at<void>(ws, L.pscratch), status, s)) != MOE_OK)
+        return rc;
+    if ((rc = do_gemm1(at<void>(ws, L.xperm), xscale, offsets, w1, w1_scale, gate_scale, up_scale, d,
+                       at<void>(ws, L.h), hscale, status, s)) != MOE_OK)
+        return rc;
+    return do_gemm2_combine(at<void>(ws, L.h), hscale, offsets, at<int32_t>(ws, L.inv), w, sw, w2, w2_scale, d, out,
+                            at<void>(ws, L.y), status, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,212 @@
+/*
+ * moe_b200.h -- C ABI of the routed mixture-of-experts expert layer for NVIDIA B200
+ * (sm_100a). The layer runs, per call and entirely on the GPU:
+ *
+ *   router / gate epilogue  ->  permute by expert  ->  grouped GEMM1 (gate|up) with a
+ *   clamped, parameterised SwiGLU epilogue  ->  grouped GEMM2 (down)  ->  routing-
+ *   weighted combine.
+ *
+ * Sources of the operations (web pages, cited by title and section):
+ *   [P2] sglang PR #39920 "Fix flashinfer_trtllm silently dropping swiglu_limit",
+ *        "Modifications": gate = clamp(gate, max=L), up = clamp(up, -L, L),
+ *        out = gate * sigmoid(alpha * gate) * (up + beta); "Motivation": GLM FP8
+ *        blockwise 128x128, 288 routed experts, top-8, 1 shared expert, L = 10.
+ *   [P3] sglang PR #36385 "Enable and fuse the Inkling MoE gate epilogue on Intel XPU",
+ *        items 2-3: masked-max top-k, ties to the lower expert id, weights
+ *        exp(lp - logsumexp(lp)) with lp = logsigmoid(x), shared-sink columns that
+ *        join the normaliser but never the top-k, a scalar routing scale.
+ *   [P4] DeepGEMM PR #445 "fix(sm90): support parameterized SwiGLU in FP8 MegaMoE",
+ *        "Summary"/"Compatibility": alpha, up_bias (beta) and clamp as explicit
+ *        parameters; alpha = 1, beta = 0, no clamp is the standard SwiGLU.
+ *   [P1] xorl-wheels "FlashInfer 0.6.18 SM100a+SM103a MoE-LoRA AOT", "Changes":
+ *        activation quantisation fused into the activation kernel; gate and up halves
+ *        carry separate scales that apply before the activation; routing ids outside
+ *        the expert range are an error.
+ *   [P5] batchgen PR #239 "sm100: Fused INT4 grouped + SiLU Triton kernel": per-expert
+ *        sorted-token dispatch, fp32 accumulation, slot-specific weighted reduction.
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is a DEVICE pointer on the current CUDA device unless
+ *     stated otherwise; the caller owns (allocates and frees) every buffer. The
+ *     library never allocates, frees or synchronises on the hot path.
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *     default stream) and returns before it runs. Calls are capturable in a CUDA graph.
+ *   - Arguments are checked on the host first. A bad argument returns a negative
+ *     moe_status and enqueues nothing. A kernel launch failure returns MOE_ERR_CUDA.
+ *   - Errors found while the kernels run (an expert id outside [0, E); a pipeline wait
+ *     that exceeded its time limit) are written to a status word at the start of the
+ *     workspace `ws`; read it with moe_read_status(). It is sticky until
+ *     moe_clear_status(). No kernel traps.
+ *   - Row-major layouts throughout. bf16 is stored as 16-bit words, E4M3 as bytes.
+ *   - Calls that share a workspace or outputs must not overlap on the GPU.
+ */
+#ifndef MOE_B200_H_
+#define MOE_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,  /* a size, pointer or parameter outside the documented range */
+    MOE_ERR_UNSUPPORTED = -2,  /* a valid combination this build does not implement */
+    MOE_ERR_ARCH = -3,         /* the current device is not compute capability 10.x */
+    MOE_ERR_WORKSPACE = -4,    /* ws is NULL, misaligned (256 B) or smaller than required */
+    MOE_ERR_EXPERT_ID = -5,    /* (device) a routing id lies outside [0, E) */
+    MOE_ERR_TIMEOUT = -6,      /* (device) a pipeline wait exceeded its limit; outputs invalid */
+    MOE_ERR_CUDA = -7          /* a CUDA runtime/driver call failed */
+} moe_status;
+
+typedef enum moe_score_fn {
+    MOE_SCORE_SOFTMAX = 0,     /* weights = softmax over the k selected logits          */
+    MOE_SCORE_SIGMOID = 1      /* weights = exp(lp - logsumexp(lp)), lp = logsigmoid(x),
+                                  over the k selected columns plus the sink columns      */
+} moe_score_fn;
+
+typedef enum moe_wdtype {
+    MOE_WDTYPE_BF16 = 0,             /* bf16 weights and activations                       */
+    MOE_WDTYPE_FP8_E4M3_BLOCK128 = 1 /* E4M3 weights with one fp32 scale per 128x128 block;
+                                        E4M3 activations with one fp32 scale per 1x128 block */
+} moe_wdtype;
+
+/* Problem statement. All fields are read on every call.
+ *   T        tokens (>= 0; T = 0 is a no-op that still writes empty offsets)
+ *   H        hidden size (multiple of 128)
+ *   I        intermediate size per expert (multiple of 128)
+ *   E        routed experts (1 .. 1024)
+ *   k        experts per token (1 .. min(E, 32))
+ *   n_sink   shared-sink columns after the E routed logits (0 .. 32-k; sigmoid only)
+ *   n_shared always-on shared experts, stored after the routed ones in the weights;
+ *            shared expert s is weighted by sink s when n_sink > 0 (then
+ *            n_shared == n_sink), else by 1
+ *   wdtype   moe_wdtype;  score  moe_score_fn
+ *   alpha, beta  SwiGLU sigmoid slope and up bias ([P4] "Summary")
+ *   limit    clamp L > 0; +INFINITY disables the clamp
+ *   route_scale  scalar multiplying every routing weight (routed and sink), usually 1
+ * Derived: G = E + n_shared weight groups; A = T*k + T*n_shared permuted rows. */
+typedef struct moe_dims {
+    int32_t T, H, I, E, k, n_sink, n_shared;
+    int32_t wdtype;
+    int32_t score;
+    float alpha, beta, limit, route_scale;
+} moe_dims;
+
+/* Which call a workspace is sized for (moe_workspace_size). */
+typedef enum moe_ws_kind {
+    MOE_WS_PERMUTE = 0,
+    MOE_WS_GEMM1 = 1,
+    MOE_WS_GEMM2_COMBINE = 2,
+    MOE_WS_FORWARD = 3
+} moe_ws_kind;
+
+/* ABI version compiled into the library (MOE_ABI_VERSION). */
+int moe_abi_version(void);
+
+/* Static string for a moe_status value. Never NULL. */
+const char* moe_status_string(int status);
+
+/* Bytes of device workspace the given call needs for these dims (written to *bytes).
+ * The workspace must be 256-byte aligned. Its first 256 bytes hold the status word;
+ * zero them once (moe_clear_status) before first use. */
+int moe_workspace_size(const moe_dims* dims, int kind, size_t* bytes);
+
+/* Copies the workspace's device status word to *status (host). Synchronises `stream`.
+ * Not for the hot path. */
+int moe_read_status(const void* ws, int32_t* status, void* stream);
+
+/* Zeroes the workspace's status word (asynchronous, on `stream`). */
+int moe_clear_status(void* ws, void* stream);
+
+/* Router / gate epilogue ([P3] items 2 and 3).
+ *   logits   [T][E + n_sink] fp32, read only. Finite values required.
+ *   topk_ids [T][k] int32 out: per token, the k routed columns with the largest logit,
+ *            in descending order; equal logits go to the lower id. Ranking is on the raw
+ *            logit (no correction bias), which orders like sigmoid(logit).
+ *   topk_w   [T][k] fp32 out: routing weights in the same order, times route_scale.
+ *            softmax: exp(l_j - logsumexp(l_sel)); sigmoid: exp(lp_j - logsumexp(lp over
+ *            the selected and the sink columns)), lp = logsigmoid(l) -- finite even when
+ *            every logit is below -104.
+ *   shared_w [T][n_sink] fp32 out (NULL iff n_sink == 0): the sink columns' weights.
+ * Errors: INVALID_ARG (sizes, NULL pointers, n_sink > 0 with softmax), ARCH, CUDA. */
+int moe_route_topk(const float* logits, const moe_dims* dims, int32_t* topk_ids,
+                   float* topk_w, float* shared_w, void* stream);
+
+/* Permute by expert ([P5]: per-expert sorted-token dispatch; [P1]: fused act-quant).
+ *   topk_ids [T][k] int32 in: expert ids in [0, E), distinct within a token.
+ *            Ids outside the range set MOE_ERR_EXPERT_ID in the status word; those
+ *            entries are dropped (never read out of bounds).
+ *   x        [T][H] bf16 in.
+ *   offsets  [G+1] int32 out: group g occupies rows [offsets[g], offsets[g+1]); groups
+ *            0..E-1 are the routed experts, E..G-1 the shared experts (T rows each).
+ *   perm     [A] int32 out: source token of each permuted row. Within a group rows are
+ *            ordered by token, then slot (deterministic).
+ *   inv_perm [T][k] int32 out: the row that holds slot j of token t.
+ *   x_perm   [A][H] out: x[perm[r]] as bf16 (wdtype BF16) or as E4M3 codes (FP8), where
+ *            each 1x128 block is quantised with s = amax/448 (1 if amax = 0), code =
+ *            E4M3 round-to-nearest-even, saturating, of x/s (fp32 arithmetic).
+ *   x_scale  [H/128][A] fp32 out (FP8 only, else may be NULL): s per block, block-major.
+ *   ws       workspace of moe_workspace_size(MOE_WS_PERMUTE) bytes.
+ * Errors: INVALID_ARG, WORKSPACE, ARCH, CUDA. */
+int moe_permute(const int32_t* topk_ids, const void* x, const moe_dims* dims,
+                int32_t* offsets, int32_t* perm, int32_t* inv_perm,
+                void* x_perm, float* x_scale, void* ws, size_t ws_bytes, void* stream);
+
+/* Grouped GEMM1 with the SwiGLU epilogue ([P2] "Modifications", [P4] "Summary",
+ * [P1] "Changes"). For every row r of group g:
+ *   gate = s_g[g] * sum_c x_perm[r][c] * W1[g][i][c]       (i < I)
+ *   up   = s_u[g] * sum_c x_perm[r][c] * W1[g][I + i][c]
+ *   h[r][i] = min(gate, L) * sigmoid(alpha * min(gate, L)) * (clamp(up, -L, L) + beta)
+ * accumulated in fp32 (FP8: per 128-deep K block, times x_scale * w1_scale).
+ *   x_perm, x_scale, offsets   as written by moe_permute (A = offsets[G]).
+ *   w1        [G][2I][H]: rows [0, I) gate, [I, 2I) up; bf16 or E4M3.
+ *   w1_scale  [G][2I/128][H/128] fp32 (FP8 only, else NULL).
+ *   gate_scale, up_scale  [G] fp32 per-group scales, or NULL for 1.0.
+ *   h         [A][I] out: bf16, or E4M3 codes quantised per 1x128 block like x_perm.
+ *   h_scale   [I/128][A] fp32 out (FP8 only, else NULL).
+ * Errors: INVALID_ARG, WORKSPACE, ARCH, CUDA; TIMEOUT in the status word. */
+int moe_gemm1_swiglu(const void* x_perm, const float* x_scale, const int32_t* offsets,
+                     const void* w1, const float* w1_scale, const float* gate_scale,
+                     const float* up_scale, const moe_dims* dims, void* h, float* h_scale,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* Grouped GEMM2 and the routing-weighted combine ([P5]: slot-specific weighted
+ * reduction in fp32). y[r] = h[r] . W2[g]^T for each row r of group g (fp32
+ * accumulation, stored as bf16 in the workspace), then for every token t
+ *   out[t] = sum_{j<k} topk_w[t][j] * y[inv_perm[t][j]]
+ *          + sum_{s<n_shared} gamma[t][s] * y[offsets[E+s] + t],
+ *   gamma = shared_w[t][s] when n_sink > 0, else 1,
+ * summed in fp32 in that fixed order and rounded once to bf16.
+ *   h, h_scale, offsets  as written by moe_gemm1_swiglu / moe_permute.
+ *   inv_perm [T][k], topk_w [T][k], shared_w [T][n_sink] (NULL iff n_sink == 0).
+ *   w2       [G][H][I] bf16 or E4M3; w2_scale [G][H/128][I/128] fp32 (FP8 only).
+ *   out      [T][H] bf16 out.
+ * Errors: INVALID_ARG, WORKSPACE, ARCH, CUDA; TIMEOUT in the status word. */
+int moe_gemm2_combine(const void* h, const float* h_scale, const int32_t* offsets,
+                      const int32_t* inv_perm, const float* topk_w, const float* shared_w,
+                      const void* w2, const float* w2_scale, const moe_dims* dims,
+                      void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* The whole layer: moe_route_topk, moe_permute, moe_gemm1_swiglu, moe_gemm2_combine in
+ * sequence on `stream`, with every intermediate in the workspace
+ * (moe_workspace_size(MOE_WS_FORWARD)).
+ *   logits [T][E+n_sink] fp32, x [T][H] bf16, weights and scales as above.
+ *   out [T][H] bf16 out.
+ *   topk_ids / topk_w / shared_w: optional outputs ([T][k], [T][k], [T][n_sink]); pass
+ *   NULL to keep them in the workspace.
+ * Errors: as the four calls. */
+int moe_forward(const float* logits, const void* x, const void* w1, const float* w1_scale,
+                const float* gate_scale, const float* up_scale, const void* w2,
+                const float* w2_scale, const moe_dims* dims, void* out, int32_t* topk_ids,
+                float* topk_w, float* shared_w, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H_ */

@@ -1,0 +1,93 @@
+"""The C ABI library on the host (CPU only): it builds, loads, exports every function the
+header declares, and rejects bad arguments before touching a GPU."""
+import ctypes
+import math
+
+import pytest
+
+import grouped_gemm_swiglu_b200 as moe
+from grouped_gemm_swiglu_b200 import build as B
+from grouped_gemm_swiglu_b200 import workloads as W
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return moe.lib()
+
+
+def test_every_header_function_is_exported(L):
+    names = moe.header_functions()
+    assert set(names) >= {"moe_route_topk", "moe_permute", "moe_gemm1_swiglu", "moe_gemm2_combine", "moe_forward",
+                          "moe_workspace_size", "moe_status_string", "moe_abi_version", "moe_read_status",
+                          "moe_clear_status"}
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/moe_b200.h but not exported"
+
+
+def test_version_and_status_strings(L):
+    assert moe.moe_abi_version() == 1
+    for code in range(-7, 1):
+        assert moe.status_string(code)
+    assert "unknown" in moe.status_string(-99)
+
+
+def _dims(**kw):
+    d = moe.MoeDims.of(W.WORKLOADS["tiny"])
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+@pytest.mark.parametrize("bad", [dict(H=200), dict(I=64), dict(E=0), dict(E=2000), dict(k=0), dict(k=9),
+                                 dict(k=33, E=64), dict(n_sink=1, score=moe.MOE_SCORE_SOFTMAX),
+                                 dict(n_sink=2, n_shared=1, score=moe.MOE_SCORE_SIGMOID), dict(T=-1),
+                                 dict(limit=0.0), dict(limit=float("nan")), dict(alpha=float("inf")),
+                                 dict(wdtype=5), dict(score=3), dict(k=8, n_sink=25, score=moe.MOE_SCORE_SIGMOID)])
+def test_invalid_dims_rejected(L, bad):
+    d = _dims(**bad)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_workspace_size(d, moe.MOE_WS_FORWARD)
+    assert ei.value.status == -1
+    # the entry points reject the same dims before any CUDA call
+    assert L.moe_route_topk(None, ctypes.byref(d), None, None, None, None) == -1
+
+
+def test_null_pointers_and_small_workspace_rejected(L):
+    d = _dims()
+    assert L.moe_route_topk(None, ctypes.byref(d), None, None, None, None) == -1
+    assert L.moe_forward(*([None] * 8), ctypes.byref(d), None, None, None, None, None, 0, None) == -1
+    fake = 1 << 20  # never dereferenced: the checks fail first
+    n = moe.moe_workspace_size(d, moe.MOE_WS_PERMUTE)
+    rc = L.moe_permute(fake, fake, ctypes.byref(d), fake, fake, fake, fake, None, fake, n - 1, None)
+    assert rc == -4
+    rc = L.moe_permute(fake, fake, ctypes.byref(d), fake, fake, fake, fake, None, fake + 8, n, None)
+    assert rc == -4  # misaligned workspace
+    rc = L.moe_permute(fake, fake + 2, ctypes.byref(d), fake, fake, fake, fake, None, fake, n, None)
+    assert rc == -1  # x not 16-byte aligned
+    # sink weights pointer must match n_sink
+    rc = L.moe_route_topk(fake, ctypes.byref(d), fake, fake, fake, None)
+    assert rc == -1
+
+
+@pytest.mark.parametrize("name", list(W.WORKLOADS))
+def test_workspace_sizes_cover_the_intermediates(L, name):
+    wl = W.WORKLOADS[name]
+    d = moe.MoeDims.of(wl)
+    A, H, I = d.A, d.H, d.I
+    elt = 1 if wl.wdtype == W.WDTYPE_FP8 else 2
+    fwd = moe.moe_workspace_size(d, moe.MOE_WS_FORWARD)
+    need = A * H * elt + A * I * elt + A * H * 2  # x_perm, h, y
+    if elt == 1:
+        need += (H // 128 + I // 128) * A * 4
+    assert fwd >= need + 256
+    assert fwd % 256 == 0
+    assert moe.moe_workspace_size(d, moe.MOE_WS_GEMM1) == 256
+    assert moe.moe_workspace_size(d, moe.MOE_WS_GEMM2_COMBINE) >= A * H * 2
+    assert moe.moe_workspace_size(d, moe.MOE_WS_PERMUTE) >= d.T * d.k * 4
+
+
+def test_no_clamp_is_infinite_limit():
+    d = moe.MoeDims.of(W.WORKLOADS["tiny"])
+    assert math.isinf(d.limit) and d.limit > 0
+    assert moe.MoeDims.of(W.WORKLOADS["oai_swiglu"]).limit == pytest.approx(7.0)

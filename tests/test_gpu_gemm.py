@@ -1,0 +1,145 @@
+"""Grouped GEMM1 (+ SwiGLU epilogue) and GEMM2 (+ weighted combine) on the GPU against
+the oracle, on synthetic permuted inputs that span several tiles, every token-tile width
+(16/32/64/128 rows), ragged group tails, empty groups and shared groups."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import grouped_gemm_swiglu_b200 as moe
+from grouped_gemm_swiglu_b200 import workloads as W
+from helpers import assert_bf16_close, assert_fp8_close, bits16, e4m3_to_np, f32, u8
+
+pytestmark = pytest.mark.gpu
+
+
+def make_case(T, E, k, S, H, I, fp8, seed, gate_up_mult=1.0, scales=False, sinks=False, skew=0.0):
+    ids = W.random_topk_ids(T, E, k, seed=seed, skew=skew)
+    offsets, perm, inv = oracle.permute(ids.numpy(), E, S)
+    A = T * (k + S)
+    G = E + S
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    w1f = torch.randn((G, 2 * I, H), generator=g, device="cuda") * 0.02 * gate_up_mult
+    w2f = torch.randn((G, H, I), generator=g, device="cuda") * 0.02
+    xf = torch.randn((A, H), generator=g, device="cuda")
+    hf = torch.randn((A, I), generator=g, device="cuda")
+    c = dict(T=T, E=E, k=k, S=S, H=H, I=I, A=A, G=G, fp8=fp8, ids=ids, offsets=offsets, perm=perm, inv=inv)
+    if fp8:
+        c["w1"], c["w1_scale"] = W.fp8_block_quantize_weights(w1f)
+        c["w2"], c["w2_scale"] = W.fp8_block_quantize_weights(w2f)
+        q, s = oracle.quant_1x128(xf.cpu().numpy())
+        c["xp"], c["xs"] = torch.from_numpy(q).cuda(), torch.from_numpy(np.ascontiguousarray(s.T)).cuda()
+        q, s = oracle.quant_1x128(hf.cpu().numpy())
+        c["hp"], c["hs"] = torch.from_numpy(q).cuda(), torch.from_numpy(np.ascontiguousarray(s.T)).cuda()
+    else:
+        c["w1"], c["w2"] = w1f.to(torch.bfloat16), w2f.to(torch.bfloat16)
+        c["w1_scale"] = c["w2_scale"] = c["xs"] = c["hs"] = None
+        c["xp"], c["hp"] = xf.to(torch.bfloat16), hf.to(torch.bfloat16)
+    c["gate_scale"] = (0.52 + 0.7 * torch.rand((G,), generator=g, device="cuda")) if scales else None
+    c["up_scale"] = (0.52 + 0.7 * torch.rand((G,), generator=g, device="cuda")) if scales else None
+    c["topk_w"] = torch.rand((T, k), generator=g, device="cuda")
+    c["shared_w"] = torch.rand((T, S), generator=g, device="cuda") if (sinks and S) else None
+    return c
+
+
+def dims_of(c, alpha=1.0, beta=0.0, limit=math.inf):
+    return moe.MoeDims(T=c["T"], H=c["H"], I=c["I"], E=c["E"], k=c["k"], n_sink=c["S"] if c["shared_w"] is not None else 0,
+                       n_shared=c["S"], wdtype=1 if c["fp8"] else 0, score=1, alpha=alpha, beta=beta,
+                       limit=limit, route_scale=1.0)
+
+
+def oracle_of(c, d):
+    fp8 = c["fp8"]
+    return oracle.Layer(T=c["T"], H=c["H"], I=c["I"], E=c["E"], k=c["k"], n_sink=d.n_sink, n_shared=c["S"],
+                        wdtype=1 if fp8 else 0, score=1, alpha=d.alpha, beta=d.beta, limit=d.limit,
+                        route_scale=1.0, logits=np.zeros((c["T"], c["E"] + d.n_sink), np.float32),
+                        x=np.zeros((c["T"], c["H"]), np.uint16),
+                        w1=u8(c["w1"]) if fp8 else bits16(c["w1"]), w2=u8(c["w2"]) if fp8 else bits16(c["w2"]),
+                        w1_scale=f32(c["w1_scale"]), w2_scale=f32(c["w2_scale"]),
+                        gate_scale=f32(c["gate_scale"]), up_scale=f32(c["up_scale"]))
+
+
+GEMM1_CASES = [
+    # T, E, k, S, H, I, fp8, extra
+    (8, 64, 4, 0, 256, 256, False, {}),                         # token tile 16, most groups empty
+    (64, 16, 4, 0, 512, 256, False, {}),                        # tile 32
+    (128, 8, 2, 0, 512, 384, False, {"scales": True}),          # tile 64, per-group gate/up scales
+    (512, 8, 2, 0, 512, 256, False, {"skew": 3.0}),             # tile 128, several blocks, ragged tails
+    (300, 16, 4, 1, 512, 256, False, {}),                       # a shared group of T rows
+    (96, 32, 4, 0, 2048, 768, False, {"oai": True}),            # OAI-SwiGLU shape and parameters
+    (512, 8, 2, 0, 512, 256, True, {}),                         # FP8, tile 64
+    (40, 32, 4, 1, 512, 256, True, {"glm": True}),              # FP8, tile 16, shared group, L = 10
+    (200, 8, 2, 0, 1024, 512, True, {"oai": True, "scales": True}),
+]
+
+
+@pytest.mark.parametrize("T,E,k,S,H,I,fp8,extra", GEMM1_CASES)
+def test_gemm1_swiglu(T, E, k, S, H, I, fp8, extra):
+    oai, glm = extra.get("oai", False), extra.get("glm", False)
+    c = make_case(T, E, k, S, H, I, fp8, seed=T + E + H, gate_up_mult=4.0 if oai else 1.0,
+                  scales=extra.get("scales", False), skew=extra.get("skew", 0.0))
+    d = dims_of(c, alpha=1.702 if oai else 1.0, beta=1.0 if oai else 0.0,
+                limit=7.0 if oai else (10.0 if glm else math.inf))
+    A = c["A"]
+    h = torch.zeros((A, I), dtype=torch.uint8 if fp8 else torch.bfloat16, device="cuda")
+    hs = torch.zeros((I // 128, A), dtype=torch.float32, device="cuda") if fp8 else None
+    ws = moe.alloc_workspace(d, moe.MOE_WS_GEMM1)
+    offsets = torch.from_numpy(c["offsets"]).cuda()
+    moe.moe_gemm1_swiglu(c["xp"], c["xs"], offsets, c["w1"], c["w1_scale"], c["gate_scale"], c["up_scale"], d,
+                         h, hs, ws)
+    assert moe.moe_read_status(ws) == 0
+    n = int(c["offsets"][-1])
+    rows = np.arange(n, dtype=np.int32)
+    grp = (np.searchsorted(c["offsets"], rows, side="right") - 1).astype(np.int32)
+    L = oracle_of(c, d)
+    xp_host = u8(c["xp"]) if fp8 else bits16(c["xp"])
+    ref = L.gemm1_rows(A, xp_host, f32(c["xs"]), rows, grp)
+    if not fp8:
+        assert_bf16_close(h[:n].float().cpu().numpy(), ref, "h")
+    else:
+        got = e4m3_to_np(h[:n]) * np.repeat(f32(hs)[:, :n].T, 128, axis=1)
+        q, s = oracle.quant_1x128(ref.astype(np.float32))
+        mirrored = oracle.e4m3_decode(q) * np.repeat(s, 128, axis=1)
+        assert_fp8_close(got, mirrored, "h (E4M3)")
+
+
+GEMM2_CASES = [
+    (8, 64, 4, 0, 256, 256, False, False),
+    (64, 16, 4, 0, 512, 256, False, False),
+    (128, 8, 2, 0, 384, 512, False, False),
+    (512, 8, 2, 0, 512, 256, False, False),
+    (300, 16, 4, 2, 512, 256, False, True),     # two sink-gated shared groups
+    (300, 16, 4, 1, 512, 256, False, False),    # one shared group with weight 1
+    (512, 8, 2, 0, 512, 256, True, False),
+    (40, 32, 4, 1, 512, 256, True, False),
+]
+
+
+@pytest.mark.parametrize("T,E,k,S,H,I,fp8,sinks", GEMM2_CASES)
+def test_gemm2_combine(T, E, k, S, H, I, fp8, sinks):
+    c = make_case(T, E, k, S, H, I, fp8, seed=3 * T + E, sinks=sinks)
+    d = dims_of(c)
+    out = torch.zeros((T, H), dtype=torch.bfloat16, device="cuda")
+    ws = moe.alloc_workspace(d, moe.MOE_WS_GEMM2_COMBINE)
+    offsets = torch.from_numpy(c["offsets"]).cuda()
+    inv = torch.from_numpy(c["inv"]).cuda()
+    moe.moe_gemm2_combine(c["hp"], c["hs"], offsets, inv, c["topk_w"], c["shared_w"], c["w2"], c["w2_scale"], d,
+                          out, ws)
+    assert moe.moe_read_status(ws) == 0
+    A = c["A"]
+    row_w = np.zeros(A, np.float32)
+    tw = f32(c["topk_w"])
+    for t in range(T):
+        for j in range(k):
+            row_w[c["inv"][t, j]] = tw[t, j]
+        for s in range(S):
+            row_w[c["offsets"][E + s] + t] = f32(c["shared_w"])[t, s] if c["shared_w"] is not None else 1.0
+    L = oracle_of(c, d)
+    hp_host = u8(c["hp"]) if fp8 else bits16(c["hp"])
+    ref = L.gemm2_rows(A, hp_host, f32(c["hs"]), c["offsets"], c["inv"], row_w, np.arange(T, dtype=np.int32))
+    got = out.float().cpu().numpy()
+    if fp8:
+        assert_fp8_close(got, ref, "out")
+    assert_bf16_close(got, ref, "out")
