@@ -86,6 +86,7 @@ def test_router_dominating_sink_and_invariant():
     assert np.all(total >= inv["observed_min"] - 1e-6) and np.all(total <= inv["observed_max"] + 1e-6)
     logits[:, :N] -= 40.0
     logits[:, N] = 50.0
+    logits[:, N + 1] = -40.0
     _, w, sw = check(logits.cuda(), N, k, 1)
     assert np.all(sw[:, 0] > 1 - 1e-6) and np.all(w.sum(1) < 1e-6)
 
