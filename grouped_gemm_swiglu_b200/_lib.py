@@ -188,3 +188,15 @@ def alloc_workspace(dims: MoeDims, kind: int, device="cuda") -> torch.Tensor:
     ws = torch.zeros(n + 256, dtype=torch.uint8, device=device)
     off = (-ws.data_ptr()) % 256
     return ws[off:off + n]
+
+
+def moe_permute_noalloc(topk_ids, x, dims: MoeDims, offsets, perm, inv_perm, x_perm, x_scale, status=None,
+                        stream=None) -> None:
+    """moe_permute without a workspace: the scratch is a fixed array inside the library
+    (for callers that cannot allocate device memory; see include/moe_b200.h)."""
+    fn = lib().moe_permute_noalloc
+    if fn.restype is not ctypes.c_int:
+        fn.argtypes = [_VP, _VP, ctypes.POINTER(MoeDims), _VP, _VP, _VP, _VP, _VP, _VP, _VP]
+        fn.restype = ctypes.c_int
+    _check("moe_permute_noalloc", fn(_p(topk_ids), _p(x), ctypes.byref(dims), _p(offsets), _p(perm),
+                                     _p(inv_perm), _p(x_perm), _p(x_scale), _p(status), _s(stream)))

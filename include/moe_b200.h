@@ -157,6 +157,30 @@ int moe_permute(const int32_t* topk_ids, const void* x, const moe_dims* dims,
                 int32_t* offsets, int32_t* perm, int32_t* inv_perm,
                 void* x_perm, float* x_scale, void* ws, size_t ws_bytes, void* stream);
 
+/* moe_permute_noalloc -- the same permutation as moe_permute for callers that cannot
+ * allocate device memory: no workspace argument, and the library allocates nothing.
+ * (The pages have no counterpart; this is a deployment convenience.)
+ * Which callers: those whose device memory is laid out in advance by a host framework
+ * (a serving engine that reserves the whole GPU, a static memory planner, a plugin
+ * interface that passes only inputs and outputs), and latency-critical code where
+ * cudaMalloc and the synchronisation it may cause are not allowed.
+ *   Arguments as moe_permute, except: no ws/ws_bytes; `status` is an optional device
+ *   int32 (NULL = not reported) where a routing id outside [0, E) or repeated within a
+ *   token is recorded (first error wins, the caller zeroes it).
+ *   Scratch: a 1 MiB array compiled into the library, one per GPU that loads it, held
+ *   until the process exits. Calls needing more -- 256-byte-rounded
+ *   ceil(T/256)*E*4 + T*k*4 bytes above 1 MiB (about T > 16000 at k = 8, E = 288) --
+ *   return MOE_ERR_WORKSPACE and enqueue nothing.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   Every call shares the array: calls that overlap on the GPU (two streams, or two
+ *   host threads) race and corrupt each other's results. Nothing in it has to be
+ *   zeroed: each call writes what it reads.
+ * Errors: INVALID_ARG, WORKSPACE (too large), ARCH, CUDA. */
+int moe_permute_noalloc(const int32_t* topk_ids, const void* x, const moe_dims* dims,
+                        int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* x_perm,
+                        float* x_scale, int32_t* status, void* stream);
+
 /* Grouped GEMM1 with the SwiGLU epilogue ([P2] "Modifications", [P4] "Summary",
  * [P1] "Changes"). For every row r of group g:
  *   gate = s_g[g] * sum_c x_perm[r][c] * W1[g][i][c]       (i < I)
