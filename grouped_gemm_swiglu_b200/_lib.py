@@ -20,7 +20,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "moe_b200.h")
 MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_ARCH",
                 -4: "MOE_ERR_WORKSPACE", -5: "MOE_ERR_EXPERT_ID", -6: "MOE_ERR_TIMEOUT", -7: "MOE_ERR_CUDA"}
-MOE_WS_PERMUTE, MOE_WS_GEMM1, MOE_WS_GEMM2_COMBINE, MOE_WS_FORWARD = 0, 1, 2, 3
+MOE_WS_PERMUTE, MOE_WS_GEMM1, MOE_WS_GEMM2_COMBINE, MOE_WS_FORWARD, MOE_WS_EXPERTS, MOE_WS_COMBINE = 0, 1, 2, 3, 4, 5
 MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
 MOE_WDTYPE_BF16, MOE_WDTYPE_FP8_E4M3_BLOCK128 = 0, 1
 
@@ -80,6 +80,9 @@ def lib() -> ctypes.CDLL:
                                   ctypes.c_int),
             "moe_forward": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, P, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t,
                              _VP], ctypes.c_int),
+            "moe_experts": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, P, _VP, _VP, _VP, _VP, ctypes.c_size_t,
+                             _VP], ctypes.c_int),
+            "moe_combine": ([_VP, _VP, _VP, _VP, _VP, P, _VP, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -174,6 +177,18 @@ def moe_forward(logits, x, w1, w1_scale, gate_scale, up_scale, w2, w2_scale, dim
     _check("moe_forward", lib().moe_forward(_p(logits), _p(x), _p(w1), _p(w1_scale), _p(gate_scale), _p(up_scale),
                                             _p(w2), _p(w2_scale), ctypes.byref(dims), _p(out), _p(topk_ids),
                                             _p(topk_w), _p(shared_w), _p(ws), _nbytes(ws), _s(stream)))
+
+
+def moe_experts(x_perm, x_scale, offsets, w1, w1_scale, gate_scale, up_scale, w2, w2_scale, dims: MoeDims, h,
+                h_scale, y, ws, stream=None) -> None:
+    _check("moe_experts", lib().moe_experts(_p(x_perm), _p(x_scale), _p(offsets), _p(w1), _p(w1_scale),
+                                            _p(gate_scale), _p(up_scale), _p(w2), _p(w2_scale), ctypes.byref(dims),
+                                            _p(h), _p(h_scale), _p(y), _p(ws), _nbytes(ws), _s(stream)))
+
+
+def moe_combine(y, offsets, inv_perm, topk_w, shared_w, dims: MoeDims, out, ws, stream=None) -> None:
+    _check("moe_combine", lib().moe_combine(_p(y), _p(offsets), _p(inv_perm), _p(topk_w), _p(shared_w),
+                                            ctypes.byref(dims), _p(out), _p(ws), _nbytes(ws), _s(stream)))
 
 
 def _nbytes(t) -> int:

@@ -58,7 +58,7 @@ bool is_fp8(const moe_dims* d) { return d->wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK12
 // Sub-buffers of a workspace, as byte offsets from its start.
 struct Layout {
     size_t ids = 0, w = 0, sw = 0, offsets = 0, perm = 0, inv = 0, xperm = 0, xscale = 0, h = 0, hscale = 0,
-           pscratch = 0, y = 0, total = 0;
+           flags = 0, splitcnt = 0, part = 0, pscratch = 0, y = 0, total = 0;
 };
 
 Layout layout(const moe_dims* d, int kind) {
@@ -81,6 +81,12 @@ Layout layout(const moe_dims* d, int kind) {
         L.xscale = take(is_fp8(d) ? (H / 128) * A * 4 : 0);
         L.h = take(A * I * act_elt(d));
         L.hscale = take(is_fp8(d) ? (I / 128) * A * 4 : 0);
+    }
+    // block flags and split-K counters are adjacent so one clear covers both
+    if (kind == MOE_WS_FORWARD || kind == MOE_WS_EXPERTS) L.flags = take(gemm_block_flags_bytes(A, G));
+    if (kind == MOE_WS_FORWARD || kind == MOE_WS_EXPERTS || kind == MOE_WS_GEMM1) {
+        L.splitcnt = take(gemm_split_counter_bytes(A, G, H, I, is_fp8(d)));
+        L.part = take(gemm_split_scratch_bytes(A, G, H, I, is_fp8(d)));
     }
     if (kind == MOE_WS_FORWARD || kind == MOE_WS_PERMUTE) L.pscratch = take(permute_scratch_bytes(d->T, d->k, d->E));
     if (kind == MOE_WS_FORWARD || kind == MOE_WS_GEMM2_COMBINE) L.y = take(A * H * 2);
@@ -107,67 +113,67 @@ int do_route(const float* logits, const moe_dims* d, int32_t* ids, float* w, flo
 }
 
 int do_permute(const int32_t* ids, const void* x, const moe_dims* d, int32_t* offsets, int32_t* perm, int32_t* inv,
-               void* xperm, float* xscale, void* scratch, int* status, cudaStream_t s) {
+               void* xperm, float* xscale, void* scratch, int* status, cudaStream_t s, int* zero = nullptr,
+               size_t zero_words = 0) {
+    unsigned int* counter = reinterpret_cast<unsigned int*>(reinterpret_cast<char*>(status) + kWsCounterOffset);
     return cuda_status(launch_permute(ids, x, d->T, d->H, d->k, d->E, d->n_shared, is_fp8(d), offsets, perm, inv,
-                                      xperm, xscale, scratch, status, s));
+                                      xperm, xscale, scratch, counter, status, s, zero, zero_words));
 }
 
-int do_gemm1(const void* xperm, const float* xscale, const int32_t* offsets, const void* w1, const float* w1s,
-             const float* gs, const float* us, const moe_dims* d, void* h, float* hs, int* status, cudaStream_t s) {
-    GemmArgs a;
+MoeGemmArgs gemm_args(const moe_dims* d, const int32_t* offsets, int* status) {
+    MoeGemmArgs a{};
     a.offsets = offsets;
     a.G = groups(d);
     a.A = rows_A(d);
-    a.K = d->H;
-    a.wrows = 2 * d->I;
-    a.n_chunks = d->I / 128;
-    a.up_off = d->I;
-    a.act = xperm;
-    a.act_scale = xscale;
-    a.w = w1;
-    a.w_scale = w1s;
-    a.out = h;
-    a.out_scale = hs;
-    a.out_ld = d->I;
-    a.gate_scale = gs;
-    a.up_scale = us;
+    a.H = d->H;
+    a.I = d->I;
+    a.fp8 = is_fp8(d);
     a.alpha = d->alpha;
     a.beta = d->beta;
     a.limit = d->limit;
     a.status = status;
-    const int bn = gemm_pick_bn(a.A, a.G, true, is_fp8(d));
-    return cuda_status(launch_gemm(a, true, is_fp8(d), bn, s));
+    a.tile_ctr = reinterpret_cast<unsigned int*>(reinterpret_cast<char*>(status) + kWsTileCtrOffset);
+    a.exit_ctr = a.tile_ctr + 1;
+    return a;
+}
+
+int do_gemm1(const void* xperm, const float* xscale, const int32_t* offsets, const void* w1, const float* w1s,
+             const float* gs, const float* us, const moe_dims* d, void* h, float* hs, void* ws, cudaStream_t s) {
+    const Layout L = layout(d, MOE_WS_GEMM1);
+    MoeGemmArgs a = gemm_args(d, offsets, at<int>(ws, 0));
+    a.split_cnt = L.part ? at<int>(ws, L.splitcnt) : nullptr;
+    a.part = L.part ? at<float>(ws, L.part) : nullptr;
+    a.run_gemm1 = true;
+    a.x_perm = xperm;
+    a.x_scale = xscale;
+    a.w1 = w1;
+    a.w1_scale = w1s;
+    a.gate_scale = gs;
+    a.up_scale = us;
+    a.h = h;
+    a.h_scale = hs;
+    return cuda_status(launch_moe_gemm(a, s));
+}
+
+int do_combine(const void* y, const int32_t* offsets, const int32_t* inv, const float* topk_w,
+               const float* shared_w, const moe_dims* d, void* out, int* status, cudaStream_t s) {
+    return cuda_status(launch_combine(y, offsets, inv, topk_w, shared_w, d->T, d->H, d->k, d->E, d->n_shared,
+                                      d->n_sink, rows_A(d), out, status, s));
 }
 
 int do_gemm2_combine(const void* h, const float* hs, const int32_t* offsets, const int32_t* inv, const float* topk_w,
                      const float* shared_w, const void* w2, const float* w2s, const moe_dims* d, void* out, void* y,
                      int* status, cudaStream_t s) {
-    GemmArgs a;
-    a.offsets = offsets;
-    a.G = groups(d);
-    a.A = rows_A(d);
-    a.K = d->I;
-    a.wrows = d->H;
-    a.n_chunks = d->H / 128;
-    a.up_off = 0;
-    a.act = h;
-    a.act_scale = hs;
-    a.w = w2;
-    a.w_scale = w2s;
-    a.out = y;
-    a.out_scale = nullptr;
-    a.out_ld = d->H;
-    a.gate_scale = nullptr;
-    a.up_scale = nullptr;
-    a.alpha = 1.f;
-    a.beta = 0.f;
-    a.limit = INFINITY;
-    a.status = status;
-    const int bn = gemm_pick_bn(a.A, a.G, false, is_fp8(d));
-    int rc = cuda_status(launch_gemm(a, false, is_fp8(d), bn, s));
+    MoeGemmArgs a = gemm_args(d, offsets, status);
+    a.run_gemm2 = true;
+    a.h = const_cast<void*>(h);
+    a.h_scale = const_cast<float*>(hs);
+    a.w2 = w2;
+    a.w2_scale = w2s;
+    a.y = y;
+    int rc = cuda_status(launch_moe_gemm(a, s));
     if (rc != MOE_OK) return rc;
-    return cuda_status(launch_combine(y, offsets, inv, topk_w, shared_w, d->T, d->H, d->k, d->E, d->n_shared,
-                                      d->n_sink, out, s));
+    return do_combine(y, offsets, inv, topk_w, shared_w, d, out, status, s);
 }
 
 }  // namespace
@@ -194,7 +200,7 @@ int moe_workspace_size(const moe_dims* dims, int kind, size_t* bytes) {
     if (!bytes) return MOE_ERR_INVALID_ARG;
     int rc = check_dims(dims);
     if (rc != MOE_OK) return rc;
-    if (kind < MOE_WS_PERMUTE || kind > MOE_WS_FORWARD) return MOE_ERR_INVALID_ARG;
+    if (kind < MOE_WS_PERMUTE || kind > MOE_WS_COMBINE) return MOE_ERR_INVALID_ARG;
     *bytes = layout(dims, kind).total;
     return MOE_OK;
 }
@@ -254,7 +260,7 @@ int moe_gemm1_swiglu(const void* x_perm, const float* x_scale, const int32_t* of
     if ((rc = check_ws(ws, ws_bytes, d, MOE_WS_GEMM1)) != MOE_OK) return rc;
     if ((rc = check_arch()) != MOE_OK) return rc;
     if (d->T == 0) return MOE_OK;
-    return do_gemm1(x_perm, x_scale, offsets, w1, w1_scale, gate_scale, up_scale, d, h, h_scale, at<int>(ws, 0),
+    return do_gemm1(x_perm, x_scale, offsets, w1, w1_scale, gate_scale, up_scale, d, h, h_scale, ws,
                     static_cast<cudaStream_t>(stream));
 }
 
@@ -275,6 +281,57 @@ int moe_gemm2_combine(const void* h, const float* h_scale, const int32_t* offset
     const Layout L = layout(d, MOE_WS_GEMM2_COMBINE);
     return do_gemm2_combine(h, h_scale, offsets, inv_perm, topk_w, shared_w, w2, w2_scale, d, out, at<void>(ws, L.y),
                             at<int>(ws, 0), static_cast<cudaStream_t>(stream));
+}
+
+int moe_experts(const void* x_perm, const float* x_scale, const int32_t* offsets, const void* w1,
+                const float* w1_scale, const float* gate_scale, const float* up_scale, const void* w2,
+                const float* w2_scale, const moe_dims* d, void* h, float* h_scale, void* y, void* ws,
+                size_t ws_bytes, void* stream) {
+    int rc = check_dims(d);
+    if (rc != MOE_OK) return rc;
+    if (d->T > 0) {
+        if (!x_perm || !offsets || !w1 || !w2 || !h || !y) return MOE_ERR_INVALID_ARG;
+        if (is_fp8(d) && (!x_scale || !w1_scale || !w2_scale || !h_scale)) return MOE_ERR_INVALID_ARG;
+        if (!aligned(x_perm, 16) || !aligned(w1, 16) || !aligned(w2, 16) || !aligned(h, 16) || !aligned(y, 16))
+            return MOE_ERR_INVALID_ARG;
+    }
+    if ((rc = check_ws(ws, ws_bytes, d, MOE_WS_EXPERTS)) != MOE_OK) return rc;
+    if ((rc = check_arch()) != MOE_OK) return rc;
+    if (d->T == 0) return MOE_OK;
+    const Layout L = layout(d, MOE_WS_EXPERTS);
+    MoeGemmArgs a = gemm_args(d, offsets, at<int>(ws, 0));
+    a.run_gemm1 = a.run_gemm2 = true;
+    a.x_perm = x_perm;
+    a.x_scale = x_scale;
+    a.w1 = w1;
+    a.w1_scale = w1_scale;
+    a.gate_scale = gate_scale;
+    a.up_scale = up_scale;
+    a.h = h;
+    a.h_scale = h_scale;
+    a.w2 = w2;
+    a.w2_scale = w2_scale;
+    a.y = y;
+    a.done1 = at<int>(ws, L.flags);
+    a.split_cnt = L.part ? at<int>(ws, L.splitcnt) : nullptr;
+    a.part = L.part ? at<float>(ws, L.part) : nullptr;
+    return cuda_status(launch_moe_gemm(a, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_combine(const void* y, const int32_t* offsets, const int32_t* inv_perm, const float* topk_w,
+                const float* shared_w, const moe_dims* d, void* out, void* ws, size_t ws_bytes, void* stream) {
+    int rc = check_dims(d);
+    if (rc != MOE_OK) return rc;
+    if (d->T > 0) {
+        if (!y || !offsets || !inv_perm || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+        if ((d->n_sink > 0) != (shared_w != nullptr)) return MOE_ERR_INVALID_ARG;
+        if (!aligned(y, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+    }
+    if ((rc = check_ws(ws, ws_bytes, d, MOE_WS_COMBINE)) != MOE_OK) return rc;
+    if ((rc = check_arch()) != MOE_OK) return rc;
+    if (d->T == 0) return MOE_OK;
+    return do_combine(y, offsets, inv_perm, topk_w, shared_w, d, out, at<int>(ws, 0),
+                      static_cast<cudaStream_t>(stream));
 }
 
 int moe_forward(const float* logits, const void* x, const void* w1, const float* w1_scale, const float* gate_scale,
@@ -301,14 +358,32 @@ int moe_forward(const float* logits, const void* x, const void* w1, const float*
     float* xscale = is_fp8(d) ? at<float>(ws, L.xscale) : nullptr;
     float* hscale = is_fp8(d) ? at<float>(ws, L.hscale) : nullptr;
     if ((rc = do_route(logits, d, ids, w, sw, s)) != MOE_OK) return rc;
+    // The counting kernel also clears the GEMM's per-block completion flags.
+    int* flags = at<int>(ws, L.flags);
+    const size_t clear_words =
+        (L.splitcnt + gemm_split_counter_bytes(rows_A(d), groups(d), d->H, d->I, is_fp8(d)) - L.flags) / sizeof(int);
     if ((rc = do_permute(ids, x, d, offsets, at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv), at<void>(ws, L.xperm),
-                         xscale, at<void>(ws, L.pscratch), status, s)) != MOE_OK)
+                         xscale, at<void>(ws, L.pscratch), status, s, flags, clear_words)) != MOE_OK)
         return rc;
-    if ((rc = do_gemm1(at<void>(ws, L.xperm), xscale, offsets, w1, w1_scale, gate_scale, up_scale, d,
-                       at<void>(ws, L.h), hscale, status, s)) != MOE_OK)
-        return rc;
-    return do_gemm2_combine(at<void>(ws, L.h), hscale, offsets, at<int32_t>(ws, L.inv), w, sw, w2, w2_scale, d, out,
-                            at<void>(ws, L.y), status, s);
+    // GEMM1 + SwiGLU and GEMM2 in one persistent launch, then the combine.
+    MoeGemmArgs a = gemm_args(d, offsets, status);
+    a.run_gemm1 = a.run_gemm2 = true;
+    a.x_perm = at<void>(ws, L.xperm);
+    a.x_scale = xscale;
+    a.w1 = w1;
+    a.w1_scale = w1_scale;
+    a.gate_scale = gate_scale;
+    a.up_scale = up_scale;
+    a.h = at<void>(ws, L.h);
+    a.h_scale = hscale;
+    a.w2 = w2;
+    a.w2_scale = w2_scale;
+    a.y = at<void>(ws, L.y);
+    a.done1 = flags;
+    a.split_cnt = L.part ? at<int>(ws, L.splitcnt) : nullptr;
+    a.part = L.part ? at<float>(ws, L.part) : nullptr;
+    if ((rc = cuda_status(launch_moe_gemm(a, s))) != MOE_OK) return rc;
+    return do_combine(at<void>(ws, L.y), offsets, at<int32_t>(ws, L.inv), w, sw, d, out, status, s);
 }
 
 }  // extern "C"

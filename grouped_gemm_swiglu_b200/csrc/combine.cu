@@ -2,65 +2,81 @@
 // sum_s gamma[t,s] * y[shared row of t], in fp32 in that fixed slot order, rounded once
 // to bf16 (slot-specific routing-weight reduction with fp32 accumulation, batchgen
 // PR #239 commit notes; shared-sink weights gamma from sglang PR #36385 item 3).
+//
+// One thread per 8 output columns (16 bytes) of one token; blockIdx.x is the token, so
+// every thread issues its k + n_shared row loads back to back and the kernel runs at
+// the memory system's rate instead of one dependent load chain per warp.
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "status.cuh"
 
 namespace moe {
 
-__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y, const int32_t* __restrict__ offsets,
-                                                      const int32_t* __restrict__ inv, const float* __restrict__ topk_w,
-                                                      const float* __restrict__ shared_w, int T, int H, int k, int E,
-                                                      int n_shared, int n_sink, uint16_t* __restrict__ out) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * 8 + warp;
-    if (t >= T) return;
-    int r = -1;
-    float wt = 0.f;
-    if (lane < k) {
-        r = inv[(size_t)t * k + lane];
-        wt = topk_w[(size_t)t * k + lane];
-    } else if (lane < k + n_shared) {
-        r = offsets[E + (lane - k)] + t;
-        wt = n_sink > 0 ? shared_w[(size_t)t * n_sink + (lane - k)] : 1.f;
-    }
+constexpr int kCombineThreads = 128;
+
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(
+    const uint16_t* __restrict__ y, const int32_t* __restrict__ offsets, const int32_t* __restrict__ inv,
+    const float* __restrict__ topk_w, const float* __restrict__ shared_w, int T, int H, int k, int E, int n_shared,
+    int n_sink, int64_t A, uint16_t* __restrict__ out, int* status) {
+    __shared__ int s_row[32];
+    __shared__ float s_w[32];
+    const int t = blockIdx.x;
     const int nd = k + n_shared;
-    const int nvec = H / 8;
-    // Warp-uniform trip count: every lane takes part in the shuffles below.
-    for (int v0 = 0; v0 < nvec; v0 += 32) {
-        const int v = v0 + lane;
-        const bool act = v < nvec;
-        float acc[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-        for (int d = 0; d < nd; ++d) {
-            const int R = __shfl_sync(0xffffffffu, r, d);
-            const float W = __shfl_sync(0xffffffffu, wt, d);
-            if (R < 0 || !act) continue;
-            const uint4 yv = __ldg(reinterpret_cast<const uint4*>(y + (size_t)R * H) + v);
-            const uint32_t wv[4] = {yv.x, yv.y, yv.z, yv.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                acc[2 * i] = fmaf(W, __uint_as_float(wv[i] << 16), acc[2 * i]);
-                acc[2 * i + 1] = fmaf(W, __uint_as_float(wv[i] & 0xFFFF0000u), acc[2 * i + 1]);
-            }
+    if (threadIdx.x < nd) {
+        const int d = threadIdx.x;
+        int64_t r;
+        float wt;
+        if (d < k) {
+            r = inv[(size_t)t * k + d];
+            wt = topk_w[(size_t)t * k + d];
+        } else {
+            r = (int64_t)offsets[E + (d - k)] + t;
+            wt = n_sink > 0 ? shared_w[(size_t)t * n_sink + (d - k)] : 1.f;
         }
-        uint32_t o[4];
+        if (r >= A) {  // never read past the intermediate, whatever the routing data says
+            set_status(status, MOE_ERR_EXPERT_ID);
+            r = -1;
+        }
+        s_row[d] = (int)r;
+        s_w[d] = wt;
+    }
+    __syncthreads();
+    const int v = blockIdx.y * blockDim.x + threadIdx.x;
+    if (v >= H / 8) return;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 4
+    for (int d = 0; d < nd; ++d) {
+        const int R = s_row[d];
+        if (R < 0) continue;
+        const float W = s_w[d];
+        const uint4 yv = __ldg(reinterpret_cast<const uint4*>(y + (size_t)R * H) + v);
+        const uint32_t wv[4] = {yv.x, yv.y, yv.z, yv.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const __nv_bfloat162 p = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-            o[i] = *reinterpret_cast<const uint32_t*>(&p);
+            acc[2 * i] = fmaf(W, __uint_as_float(wv[i] << 16), acc[2 * i]);
+            acc[2 * i + 1] = fmaf(W, __uint_as_float(wv[i] & 0xFFFF0000u), acc[2 * i + 1]);
         }
-        if (act) reinterpret_cast<uint4*>(out + (size_t)t * H)[v] = make_uint4(o[0], o[1], o[2], o[3]);
     }
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 p = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        o[i] = *reinterpret_cast<const uint32_t*>(&p);
+    }
+    reinterpret_cast<uint4*>(out + (size_t)t * H)[v] = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 cudaError_t launch_combine(const void* y, const int32_t* offsets, const int32_t* inv, const float* topk_w,
-                           const float* shared_w, int T, int H, int k, int E, int n_shared, int n_sink, void* out,
-                           cudaStream_t stream) {
+                           const float* shared_w, int T, int H, int k, int E, int n_shared, int n_sink, int64_t A,
+                           void* out, int* status, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    combine_kernel<<<(T + 7) / 8, 256, 0, stream>>>(static_cast<const uint16_t*>(y), offsets, inv, topk_w, shared_w,
-                                                    T, H, k, E, n_shared, n_sink, static_cast<uint16_t*>(out));
+    dim3 grid(T, (H / 8 + kCombineThreads - 1) / kCombineThreads);
+    combine_kernel<<<grid, kCombineThreads, 0, stream>>>(static_cast<const uint16_t*>(y), offsets, inv, topk_w,
+                                                         shared_w, T, H, k, E, n_shared, n_sink, A,
+                                                         static_cast<uint16_t*>(out), status);
     return cudaGetLastError();
 }
 

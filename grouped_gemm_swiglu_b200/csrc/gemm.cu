@@ -1,17 +1,18 @@
-// gemm.cu -- grouped GEMMs of the expert layer on the 5th-generation tensor cores.
+// gemm.cu -- grouped GEMMs of the expert layer on the 5th-generation tensor cores, as
+// one persistent kernel that can run GEMM1 (+ SwiGLU), GEMM2, or both in one launch.
 //
 // Orientation: the expert's weight rows are the MMA's M side (128 rows per tile, TMEM
 // lanes) and the permuted token rows of the group are the N side (up to BN per tile,
 // TMEM columns), so a group with n rows costs ceil(n/16)*16 MMA columns, not a 128-row
 // tile, and decode-sized groups stream weights with N = 16.
 //
-// GEMM1 (gated): each tile covers 128 gate rows and the matching 128 up rows of W1[g]
-// (two MMAs per K step into two TMEM column ranges), so one thread holds gate and up
-// of the same intermediate index and the clamped, parameterised SwiGLU (sglang PR
+// Phase 1, GEMM1 (gated): a tile covers 128 gate rows and the matching 128 up rows of
+// W1[g] (two MMAs per K step into two TMEM column ranges), so one thread holds gate and
+// up of the same intermediate index and the clamped, parameterised SwiGLU (sglang PR
 // #39920 "Modifications"; DeepGEMM PR #445 "Summary") runs in the epilogue, with the
 // per-group gate/up scales applied to the accumulators first (xorl-wheels FlashInfer
 // 0.6.18 release notes, "Changes"). The intermediate never leaves the SM unactivated.
-// GEMM2: one MMA per K step; the epilogue stores y in bf16.
+// Phase 2, GEMM2: one MMA per K step; the epilogue stores y in bf16.
 //
 // FP8 (E4M3, 128x128 weight blocks, 1x128 activation blocks; GLM FP8 blockwise, sglang
 // PR #39920 "Motivation"): every 128-deep K block is one pipeline stage; its product
@@ -19,12 +20,19 @@
 // registers with the product of the two block scales, while the tensor core fills the
 // other buffer. GEMM1's epilogue then quantises h per 1x128 block (fused act-quant).
 //
+// Scheduling: tiles are numbered GEMM1 first -- (token block, 128-row chunk of I) --
+// then GEMM2 -- (token block, 128-row chunk of H). The producer warp claims the next
+// tile from a global counter and hands its number to the MMA and epilogue warps through
+// a two-slot ring in shared memory. When both phases run, a GEMM2 tile of token block b
+// first loads its weights, then waits until all GEMM1 tiles of b have published their h
+// rows (a per-block release counter); a tile only ever waits for tiles claimed before
+// it, which never wait themselves, so the schedule cannot deadlock.
+//
 // Roles (320 threads): warp 0 lane 0 issues TMA loads into a STAGES-deep ring; warp 1
 // owns TMEM and lane 0 issues tcgen05.mma; warps 2..9 are the epilogue (warp w reads
-// TMEM lanes 32*(w%4).., and columns of half (w-2)/4 of the tile). Tiles are scheduled
-// persistently: tile L = (token block, chunk), CTA b takes L = b, b + grid, ...
-// Every wait is bounded (ptx.cuh): on timeout the CTA sets MOE_ERR_TIMEOUT, drains its
-// outstanding copies and MMAs, frees TMEM and returns.
+// TMEM lanes 32*(w%4).., and columns of half (w-2)/4 of the tile). Every wait is bounded
+// (ptx.cuh): on timeout the CTA sets MOE_ERR_TIMEOUT, drains its outstanding copies and
+// MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
@@ -36,9 +44,9 @@
 
 namespace moe {
 
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in per block
+constexpr int kRing = 2;            // tile-number ring depth
+constexpr int kMaxGroupsGemm = 1024 + 32;
 
 constexpr int pow2_at_least(int v) {
     int p = 32;
@@ -46,72 +54,128 @@ constexpr int pow2_at_least(int v) {
     return p;
 }
 
-template <int BN_, bool GATED_, bool FP8_>
+template <int BN_, bool FP8_>
 struct Cfg {
     static constexpr int BN = BN_;
-    static constexpr bool GATED = GATED_;
     static constexpr bool FP8 = FP8_;
     static constexpr int BK = FP8 ? 128 : 64;  // K elements per stage: one 128-byte row
-    static constexpr int NUM_A = GATED ? 2 : 1;
     static constexpr int A_BYTES = 128 * 128;
     static constexpr int B_BYTES = BN * 128;
-    static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
-    static constexpr int STAGES_RAW = (196 * 1024) / STAGE_BYTES;
+    static constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES;  // sized for GEMM1 (gate + up)
+    // as many stages as fit next to the control block and the largest group table
+    static constexpr int STAGE_BUDGET = kSmemLimit - 1024 - 8 * (kMaxGroupsGemm + 1) - 1024 - 4 * 16 * 16 * 3;
+    static constexpr int STAGES_RAW = STAGE_BUDGET / STAGE_BYTES;
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
-    static constexpr int ACC_COLS = NUM_A * BN;  // one TMEM buffer
-    static constexpr int TMEM_COLS = pow2_at_least(2 * ACC_COLS);
-    static constexpr int HALF = BN / 2;           // columns per epilogue warp
-    static constexpr int CW = HALF < 16 ? HALF : 16;
-    static constexpr int RED_FLOATS = (FP8 && GATED) ? 2 * 4 * HALF : 4;
+    static constexpr int ACC_COLS = 2 * BN;  // one TMEM buffer: gate | up (GEMM2 uses the first BN)
+    // bf16 hands one buffer per tile to the epilogue, FP8 one per 128-deep K block, so
+    // FP8 keeps up to four partial buffers in flight.
+    static constexpr int NBUF = (FP8 && 4 * ACC_COLS <= 512) ? 4 : 2;
+    static constexpr int TMEM_COLS = pow2_at_least(NBUF * ACC_COLS);
+    // Epilogue warps: two groups of four (one warp per TMEM lane quarter), each group
+    // owning half of the tile's columns.
+    static constexpr int EPI = 8;
+    static constexpr int THREADS = 64 + 32 * EPI;
+    static constexpr int GROUPS = EPI / 4;
+    static constexpr int COLS = BN / GROUPS;  // columns per epilogue warp
+    static constexpr int CW = COLS < 16 ? COLS : 16;  // TMEM load width (columns)
+    static constexpr int RED_FLOATS = FP8 ? EPI * COLS : 4;
+    // FP8: per epilogue warp, the two rows of scale products (A0, A1) of its columns
+    static constexpr int SCT_FLOATS = FP8 ? EPI * 2 * COLS : 4;
     static_assert(STAGE_BYTES % 1024 == 0, "stage tiles must stay 1024-byte aligned");
     static_assert(TMEM_COLS <= 512, "TMEM holds 512 columns");
-    static_assert(HALF % CW == 0, "column share must be a multiple of the load width");
+    static_assert(COLS % CW == 0 && CW >= 4, "column share must be a multiple of the load width");
+    static_assert(!FP8 || COLS <= 32, "FP8 loads a warp's whole column share at once");
+    static_assert(STAGES >= 2, "at least two pipeline stages");
+    // Split-K of GEMM1 is compiled in where it can be chosen (see gemm_split_factor):
+    // every tile width except FP8 at 64 columns, whose promotion registers are full.
+    static constexpr bool SPLIT_OK = !(FP8 && BN >= 64);
 
-    static constexpr size_t ctrl_bytes() { return 8 * (2 * STAGES + 6) + 16 + 4 * RED_FLOATS; }
-    static size_t smem_bytes(int G) {
-        return 1024 + (size_t)STAGES * STAGE_BYTES + ctrl_bytes() + 4 * (size_t)(G + 1) + 16;
+    // full/empty per stage, tfull/tempty per TMEM buffer, ring_full/ring_empty x kRing, drain, epibar
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 2 * kRing + 2;
+    static constexpr size_t ctrl_bytes() {
+        return 8 * NUM_BARS + 16 + 4 * kRing + 16 + 4 * RED_FLOATS + 16 + 4 * SCT_FLOATS;
+    }
+    static size_t smem_bytes(int G) {  // + block table and clamped offsets, G+1 ints each
+        return 1024 + (size_t)STAGES * STAGE_BYTES + ctrl_bytes() + 8 * (size_t)(G + 1) + 16;
     }
 };
 
 struct DevArgs {
     const int32_t* offsets;
-    int G;
-    int num_kb;       // K / BK
-    int wrows;        // weight rows per group
-    int n_chunks;     // 128-row chunks per group
-    int up_off;       // gate->up row offset (GEMM1)
-    int kblocks;      // K / 128 (FP8 scale columns)
-    int64_t A;
-    const float* act_scale;
-    const float* w_scale;
-    void* out;
-    float* out_scale;
-    int out_ld;
+    int G, A, H, I;
+    int c1;      // GEMM1 tiles per token block: I/128 (0 = phase absent)
+    int c2;      // GEMM2 tiles per token block: ceil(H/256), each two 128-row chunks of H (0 = absent)
+    const float* x_scale;   // FP8: [H/128][A]
+    const float* w1_scale;  // FP8: [G][2I/128][H/128]
+    const float* w2_scale;  // FP8: [G][H/128][I/128]
     const float* gate_scale;
     const float* up_scale;
     float alpha, beta, limit;
+    void* h;                // GEMM1 out / GEMM2 in: [A][I]
+    float* h_scale;         // FP8: [I/128][A]
+    void* y;                // GEMM2 out: [A][H] bf16
+    unsigned int* tile_ctr;  // next tile to claim (zero when idle)
+    unsigned int* exit_ctr;  // CTAs finished (zero when idle)
+    int* done1;              // per token block: GEMM1 chunks published (zero at launch; both phases only)
+    int s1;                  // GEMM1 split-K factor
+    float* part;             // split-K partials [tile1][s1][2][BN][128]
+    int* split_cnt;          // per GEMM1 tile: splits finished
     int* status;
 };
 
+// A tile is one or two 128-row weight blocks (A0, A1) against BN token rows: GEMM1 =
+// gate rows and the matching up rows; GEMM2 = two consecutive 128-row chunks of H (the
+// second absent when H/128 is odd and this is the last pair).
 struct Tile {
-    int g, c, row0, nrows;
+    int phase;  // 1 = GEMM1 + SwiGLU, 2 = GEMM2
+    int blk, g, c, row0, nrows;
+    int ks;           // GEMM1 split index (0 .. s1-1)
+    bool dual;        // A1 present
+    int a0row, a1row; // first weight row of A0 / A1 in the [G*rows][K] weight matrix
+    int col0, col1;   // first output column of A0 / A1 (intermediate or hidden index)
 };
 
+// blk_start: first token block of each group; s_off: group bounds clamped into [0, A].
 template <int BN>
-__device__ __forceinline__ Tile decode_tile(int L, const int32_t* blk_start, const DevArgs& p) {
-    const int blk = L / p.n_chunks;
+__device__ __forceinline__ Tile decode_tile(int L, int T1, const int32_t* blk_start, const int32_t* s_off,
+                                            const DevArgs& p) {
     Tile t;
-    t.c = L - blk * p.n_chunks;
+    if (L < T1) {
+        t.phase = 1;
+        const int tile1 = L / p.s1;  // the splits of one GEMM1 tile are consecutive
+        t.ks = L - tile1 * p.s1;
+        t.blk = tile1 / p.c1;
+        t.c = tile1 - t.blk * p.c1;
+    } else {
+        t.ks = 0;
+        t.phase = 2;
+        const int L2 = L - T1;
+        t.blk = L2 / p.c2;
+        t.c = L2 - t.blk * p.c2;
+    }
     int lo = 0, hi = p.G - 1;  // largest g with blk_start[g] <= blk
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (blk_start[mid] <= blk) lo = mid;
+        if (blk_start[mid] <= t.blk) lo = mid;
         else hi = mid - 1;
     }
     t.g = lo;
-    const int end = __ldg(p.offsets + lo + 1);
-    t.row0 = __ldg(p.offsets + lo) + (blk - blk_start[lo]) * BN;
-    t.nrows = min(BN, end - t.row0);
+    const int g0 = s_off[lo];
+    const int g1 = max(s_off[lo + 1], g0);
+    t.row0 = g0 + (t.blk - blk_start[lo]) * BN;
+    t.nrows = min(BN, g1 - t.row0);
+    if (t.phase == 1) {
+        t.dual = true;
+        t.a0row = t.g * 2 * p.I + t.c * 128;
+        t.a1row = t.a0row + p.I;
+        t.col0 = t.col1 = t.c * 128;
+    } else {
+        t.dual = 2 * t.c + 1 < p.H / 128;
+        t.a0row = t.g * p.H + 2 * t.c * 128;
+        t.a1row = t.a0row + 128;
+        t.col0 = 2 * t.c * 128;
+        t.col1 = t.col0 + 128;
+    }
     return t;
 }
 
@@ -120,6 +184,15 @@ __device__ __forceinline__ float swiglu_dev(float gate, float up, float alpha, f
     const float u = fminf(fmaxf(up, -limit), limit);
     const float sig = 1.f / (1.f + __expf(-alpha * g));
     return g * sig * (u + beta);
+}
+
+// a0 += p0 * s0, a1 += p1 * s1 as one packed fp32x2 fused multiply-add.
+__device__ __forceinline__ void ffma2(float& a0, float& a1, float p0, float p1, float s0, float s1) {
+    asm("{\n\t.reg .b64 d, x, y, z;\n\t"
+        "mov.b64 x, {%2, %3};\n\tmov.b64 y, {%4, %5};\n\tmov.b64 z, {%0, %1};\n\t"
+        "fma.rn.f32x2 d, x, y, z;\n\tmov.b64 {%0, %1}, d;\n\t}\n"
+        : "+f"(a0), "+f"(a1)
+        : "f"(p0), "f"(p1), "f"(s0), "f"(s1));
 }
 
 // Warp-collective bounded wait: lane 0 waits, the verdict is broadcast.
@@ -132,21 +205,27 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, PipeAb
 }
 
 template <class C>
-__global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const DevArgs p) {
+__global__ void __launch_bounds__(C::THREADS, 1)
+    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmX,
+                    const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmH,
+                    const DevArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)C::STAGES * C::STAGE_BYTES);
     uint64_t* empty = full + C::STAGES;
     uint64_t* tfull = empty + C::STAGES;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* drain = tempty + 2;
+    uint64_t* tempty = tfull + C::NBUF;
+    uint64_t* ring_full = tempty + C::NBUF;
+    uint64_t* ring_empty = ring_full + kRing;
+    uint64_t* drain = ring_empty + kRing;
     uint64_t* epibar = drain + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epibar + 1);
     PipeAbort* ab = reinterpret_cast<PipeAbort*>(tmem_slot + 1);
-    float* red = reinterpret_cast<float*>(tmem_slot + 4);
-    int32_t* blk_start = reinterpret_cast<int32_t*>(red + C::RED_FLOATS);
+    int* ring = reinterpret_cast<int*>(tmem_slot + 4);
+    float* red = reinterpret_cast<float*>(ring + kRing + 4);
+    float* sct = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(red + C::RED_FLOATS) + 15) & ~uintptr_t(15));
+    int32_t* blk_start = reinterpret_cast<int32_t*>(sct + C::SCT_FLOATS);
+    int32_t* s_off = blk_start + (p.G + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.G;
@@ -156,12 +235,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < C::NBUF; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], kEpiWarps);
+            mbar_init(&tempty[b], C::EPI);
+        }
+        for (int r = 0; r < kRing; ++r) {
+            mbar_init(&ring_full[r], 1);
+            mbar_init(&ring_empty[r], 1 + C::EPI);
         }
         mbar_init(drain, 1);
-        mbar_init(epibar, kEpiWarps);
+        mbar_init(epibar, C::EPI);
         ab->flag = 0;
         fence_barrier_init();
     }
@@ -170,9 +253,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_relinquish();
     }
     // Token blocks per group and their running start: blk_start[g] = sum_{g'<g} ceil(n_g'/BN).
+    // The offsets may come from the caller: group bounds are clamped into [0, A] (and a
+    // bad array is flagged), so no tile ever reads or writes a row outside the matrices.
     for (int g = threadIdx.x; g < G; g += blockDim.x) {
-        const int n = __ldg(p.offsets + g + 1) - __ldg(p.offsets + g);
-        blk_start[g + 1] = n > 0 ? (n + C::BN - 1) / C::BN : 0;
+        const int o0 = __ldg(p.offsets + g), o1 = __ldg(p.offsets + g + 1);
+        const int lo = min(max(o0, 0), p.A), hi = min(max(o1, lo), p.A);
+        if (o0 != lo || o1 != hi) set_status(p.status, MOE_ERR_EXPERT_ID);
+        blk_start[g + 1] = (hi - lo + C::BN - 1) / C::BN;
+        s_off[g] = lo;
+        if (g == G - 1) s_off[G] = min(max(o1, 0), p.A);
     }
     __syncthreads();
     if (warp == 0) {
@@ -195,29 +284,75 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int total = blk_start[G] * p.n_chunks;
+    const int nblk = blk_start[G];
+    const int T1 = nblk * p.c1 * p.s1;
+    const int total = T1 + nblk * p.c2;
+    const bool chained = p.done1 != nullptr && p.c1 > 0 && p.c2 > 0;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            tma_prefetch_desc(&tmA);
-            tma_prefetch_desc(&tmB);
+            tma_prefetch_desc(&tmW1);
+            tma_prefetch_desc(&tmX);
+            tma_prefetch_desc(&tmW2);
+            tma_prefetch_desc(&tmH);
             uint32_t stage = 0, phase = 0, pend_mask = 0, pend_phase = 0;
             bool ok = true;
-            for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-                const Tile tl = decode_tile<C::BN>(L, blk_start, p);
-                const int arow = tl.g * p.wrows + tl.c * 128;
-                for (int kb = 0; kb < p.num_kb; ++kb) {
+            // Tiles are claimed one ahead, so the atomic's latency overlaps the current tile.
+            auto claim = [&](int i) -> int {
+                return p.tile_ctr ? (int)atomicAdd(p.tile_ctr, 1u) : (int)blockIdx.x + i * (int)gridDim.x;
+            };
+            int next_L = claim(0);
+            for (int i = 0; ok; ++i) {
+                const int slot = i % kRing;
+                int L = next_L;
+                if (L >= total) L = -1;
+                else next_L = claim(i + 1);
+                if (!mbar_wait(&ring_empty[slot], ((i / kRing) & 1) ^ 1, ab, p.status)) break;
+                ring[slot] = L;
+                mbar_arrive(&ring_full[slot]);
+                if (L < 0) break;
+                const Tile tl = decode_tile<C::BN>(L, T1, blk_start, s_off, p);
+                const bool g1 = tl.phase == 1;
+                const CUtensorMap* tw = g1 ? &tmW1 : &tmW2;
+                const CUtensorMap* ta = g1 ? &tmX : &tmH;
+                const int all_kb = (g1 ? p.H : p.I) / C::BK;
+                const int kbase = g1 ? tl.ks * all_kb / p.s1 : 0;  // this tile's K blocks
+                const int num_kb = g1 ? (tl.ks + 1) * all_kb / p.s1 - kbase : all_kb;
+                const uint32_t tx = (tl.dual ? 2 : 1) * C::A_BYTES + C::B_BYTES;
+                // GEMM2 after GEMM1 in the same launch: weights of the first stages go out
+                // before waiting for the block's h rows.
+                const bool dep = chained && !g1;
+                const int pre = dep ? min(num_kb, C::STAGES) : 0;
+                const uint32_t st0 = stage;
+                // Wait for the block's h rows, then load the activation rows of the
+                // prefetched stages. They are loaded even when the wait gave up (the rows
+                // are in bounds; the results are discarded), so every armed stage completes.
+                auto release_prefetched = [&]() -> bool {
+                    const bool dep_ok = wait_counter_geq(p.done1 + tl.blk, p.c1, ab, p.status);
+                    uint32_t s2 = st0;
+                    for (int k2 = 0; k2 < pre; ++k2) {
+                        tma_load_2d(smem + (size_t)s2 * C::STAGE_BYTES + 2 * C::A_BYTES, ta, &full[s2],
+                                    (kbase + k2) * C::BK, tl.row0);
+                        if (++s2 == (uint32_t)C::STAGES) s2 = 0;
+                    }
+                    return dep_ok;
+                };
+                for (int kb = 0; kb < num_kb && ok; ++kb) {
+                    if (kb == pre && dep && !release_prefetched()) {
+                        ok = false;
+                        break;
+                    }
                     if (!mbar_wait(&empty[stage], phase ^ 1, ab, p.status)) {
                         ok = false;
                         break;
                     }
                     uint8_t* st = smem + (size_t)stage * C::STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-                    tma_load_2d(st, &tmA, &full[stage], kb * C::BK, arow);
-                    if constexpr (C::GATED)
-                        tma_load_2d(st + C::A_BYTES, &tmA, &full[stage], kb * C::BK, arow + p.up_off);
-                    tma_load_2d(st + C::NUM_A * C::A_BYTES, &tmB, &full[stage], kb * C::BK, tl.row0);
+                    mbar_arrive_expect_tx(&full[stage], tx);
+                    const int kx = (kbase + kb) * C::BK;
+                    tma_load_2d(st, tw, &full[stage], kx, tl.a0row);
+                    if (tl.dual) tma_load_2d(st + C::A_BYTES, tw, &full[stage], kx, tl.a1row);
+                    if (kb >= pre) tma_load_2d(st + 2 * C::A_BYTES, ta, &full[stage], kx, tl.row0);
                     pend_mask |= 1u << stage;
                     pend_phase = (pend_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == (uint32_t)C::STAGES) {
@@ -225,6 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         phase ^= 1;
                     }
                 }
+                if (ok && dep && pre == num_kb && !release_prefetched()) ok = false;  // whole K prefetched
             }
             // Never leave with a copy in flight: wait for the last fill of every stage.
             for (int s = 0; s < C::STAGES; ++s)
@@ -236,33 +372,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             uint32_t stage = 0, phase = 0, it = 0;
             bool ok = true;
-            for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-                const Tile tl = decode_tile<C::BN>(L, blk_start, p);
+            for (int i = 0; ok; ++i) {
+                const int slot = i % kRing;
+                if (!mbar_wait(&ring_full[slot], (i / kRing) & 1, ab, p.status)) break;
+                const int L = ring[slot];
+                mbar_arrive(&ring_empty[slot]);
+                if (L < 0) break;
+                const Tile tl = decode_tile<C::BN>(L, T1, blk_start, s_off, p);
+                const bool g1 = tl.phase == 1;
+                const int all_kb = (g1 ? p.H : p.I) / C::BK;
+                const int kbase = g1 ? tl.ks * all_kb / p.s1 : 0;
+                const int num_kb = g1 ? (tl.ks + 1) * all_kb / p.s1 - kbase : all_kb;
                 const int n_mma = max(16, (tl.nrows + 15) & ~15);
                 const uint32_t idesc = idesc_m128(n_mma, C::FP8);
-                if constexpr (!C::FP8) {
-                    const uint32_t buf = it & 1, bph = (it >> 1) & 1;
+                // bf16: one TMEM buffer per tile; FP8: one per 128-deep K block
+                const int units = C::FP8 ? num_kb : 1;
+                const int kb_per_unit = C::FP8 ? 1 : num_kb;
+                int kb = 0;
+                for (int u = 0; u < units && ok; ++u) {
+                    const uint32_t buf = it % C::NBUF, bph = (it / C::NBUF) & 1;
                     if (!mbar_wait(&tempty[buf], bph ^ 1, ab, p.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t d0 = tmem_base + buf * C::ACC_COLS;
-                    for (int kb = 0; kb < p.num_kb; ++kb) {
+                    for (int j = 0; j < kb_per_unit; ++j, ++kb) {
                         if (!mbar_wait(&full[stage], phase, ab, p.status)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                         const uint32_t a0 = smem_u32(smem + (size_t)stage * C::STAGE_BYTES);
-                        const uint32_t b0 = a0 + C::NUM_A * C::A_BYTES;
+                        const uint32_t b0 = a0 + 2 * C::A_BYTES;
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             const uint64_t bd = smem_desc_sw128(b0 + kk * 32);
-                            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-                            mma_bf16(d0, smem_desc_sw128(a0 + kk * 32), bd, idesc, acc);
-                            if constexpr (C::GATED)
-                                mma_bf16(d0 + C::BN, smem_desc_sw128(a0 + C::A_BYTES + kk * 32), bd, idesc, acc);
+                            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+                            if constexpr (C::FP8) {
+                                mma_fp8(d0, smem_desc_sw128(a0 + kk * 32), bd, idesc, acc);
+                                if (tl.dual)
+                                    mma_fp8(d0 + C::BN, smem_desc_sw128(a0 + C::A_BYTES + kk * 32), bd, idesc, acc);
+                            } else {
+                                mma_bf16(d0, smem_desc_sw128(a0 + kk * 32), bd, idesc, acc);
+                                if (tl.dual)
+                                    mma_bf16(d0 + C::BN, smem_desc_sw128(a0 + C::A_BYTES + kk * 32), bd, idesc, acc);
+                            }
                         }
                         tc_commit(&empty[stage]);
                         if (++stage == (uint32_t)C::STAGES) {
@@ -273,38 +428,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     tc_commit(&tfull[buf]);
                     ++it;
-                } else {
-                    for (int kb = 0; kb < p.num_kb; ++kb) {
-                        const uint32_t buf = it & 1, bph = (it >> 1) & 1;
-                        if (!mbar_wait(&tempty[buf], bph ^ 1, ab, p.status)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        if (!mbar_wait(&full[stage], phase, ab, p.status)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t d0 = tmem_base + buf * C::ACC_COLS;
-                        const uint32_t a0 = smem_u32(smem + (size_t)stage * C::STAGE_BYTES);
-                        const uint32_t b0 = a0 + C::NUM_A * C::A_BYTES;
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t bd = smem_desc_sw128(b0 + kk * 32);
-                            const uint32_t acc = kk > 0 ? 1u : 0u;
-                            mma_fp8(d0, smem_desc_sw128(a0 + kk * 32), bd, idesc, acc);
-                            if constexpr (C::GATED)
-                                mma_fp8(d0 + C::BN, smem_desc_sw128(a0 + C::A_BYTES + kk * 32), bd, idesc, acc);
-                        }
-                        tc_commit(&empty[stage]);
-                        tc_commit(&tfull[buf]);
-                        ++it;
-                        if (++stage == (uint32_t)C::STAGES) {
-                            stage = 0;
-                            phase ^= 1;
-                        }
-                    }
                 }
             }
             // All MMAs issued by this thread complete before TMEM is released.
@@ -315,53 +438,117 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int ew = warp - 2;
-        const int q = warp & 3;        // TMEM lane quarter this warp may access
-        const int hc = ew >> 2;        // which half of the tile's columns
-        const int c0 = hc * C::HALF;
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int cg = ew >> 2;  // which group of the tile's columns
+        const int c0 = cg * C::COLS;
         const int row_local = q * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         uint32_t it = 0, ephase = 0;
         bool ok = true;
-        for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-            const Tile tl = decode_tile<C::BN>(L, blk_start, p);
+        int* merge_flag = ring + kRing + 1;
+        // Split-K of GEMM1: this split's partials are in memory. Returns 1 when this CTA
+        // holds the last split of the tile (and merges), 0 when another split merges, -1
+        // when the CTA aborted. The counter goes back to zero in the merging CTA.
+        auto split_arrive = [&](int tile1) -> int {
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(epibar);
+            if (!warp_wait(epibar, ephase, ab, p.status)) return -1;
+            ephase ^= 1;
+            if (ew == 0 && lane == 0) {
+                const int old = atomicAdd(p.split_cnt + tile1, 1);
+                const int last = old == p.s1 - 1;
+                if (last) {
+                    __threadfence();
+                    p.split_cnt[tile1] = 0;
+                }
+                *merge_flag = last;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(epibar);
+            if (!warp_wait(epibar, ephase, ab, p.status)) return -1;
+            ephase ^= 1;
+            return *reinterpret_cast<volatile int*>(merge_flag);
+        };
+        // partial of split ks, half (0 gate, 1 up), column n, this thread's row
+        auto part_at = [&](int tile1, int ks, int half, int n) -> float* {
+            return p.part + (((size_t)(tile1 * p.s1 + ks) * 2 + half) * C::BN + n) * 128 + row_local;
+        };
+        for (int i = 0; ok; ++i) {
+            const int slot = i % kRing;
+            if (!warp_wait(&ring_full[slot], (i / kRing) & 1, ab, p.status)) break;
+            const int L = ring[slot];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ring_empty[slot]);
+            if (L < 0) break;
+            const Tile tl = decode_tile<C::BN>(L, T1, blk_start, s_off, p);
+            const bool g1 = tl.phase == 1;
             const int n_mma = max(16, (tl.nrows + 15) & ~15);
-            const int col = tl.c * 128 + row_local;  // output column (intermediate or hidden index)
+            // output columns of this thread: A0's and A1's row (intermediate or hidden index)
+            const int col = tl.col0 + row_local, col_b = tl.col1 + row_local;
+            const int out_ld = g1 ? p.I : p.H;
+            const float sg = (g1 && p.gate_scale) ? __ldg(p.gate_scale + tl.g) : 1.f;
+            const float su = (g1 && p.up_scale) ? __ldg(p.up_scale + tl.g) : 1.f;
             if constexpr (!C::FP8) {
-                const uint32_t buf = it & 1, bph = (it >> 1) & 1;
+                const uint32_t buf = it % C::NBUF, bph = (it / C::NBUF) & 1;
                 if (!warp_wait(&tfull[buf], bph, ab, p.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t tb = tmem_base + lane_off + buf * C::ACC_COLS;
-                __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-                if constexpr (C::GATED) {
-                    const float sg = p.gate_scale ? __ldg(p.gate_scale + tl.g) : 1.f;
-                    const float su = p.up_scale ? __ldg(p.up_scale + tl.g) : 1.f;
+                __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g1 ? p.h : p.y);
+                const int tile1 = tl.blk * p.c1 + tl.c;
+                if (g1 && p.s1 > 1) {
+                    // split-K: store this split's fp32 gate/up sums; the last split merges
 #pragma unroll 1
-                    for (int cc = c0; cc < c0 + C::HALF && cc < n_mma; cc += C::CW) {
+                    for (int cc = c0; cc < c0 + C::COLS && cc < n_mma; cc += C::CW) {
                         float gv[C::CW], uv[C::CW];
-                        if constexpr (C::CW == 16) tmem_ld16x2(tb + cc, tb + C::BN + cc, gv, uv);
-                        else tmem_ld8x2(tb + cc, tb + C::BN + cc, gv, uv);
+                        tmem_ld_x2<C::CW>(tb + cc, tb + C::BN + cc, gv, uv);
+#pragma unroll
+                        for (int j = 0; j < C::CW; ++j) {
+                            *part_at(tile1, tl.ks, 0, cc + j) = gv[j];
+                            *part_at(tile1, tl.ks, 1, cc + j) = uv[j];
+                        }
+                    }
+                } else if (g1) {
+#pragma unroll 1
+                    for (int cc = c0; cc < c0 + C::COLS && cc < n_mma; cc += C::CW) {
+                        float gv[C::CW], uv[C::CW];
+                        tmem_ld_x2<C::CW>(tb + cc, tb + C::BN + cc, gv, uv);
 #pragma unroll
                         for (int j = 0; j < C::CW; ++j) {
                             const int n = cc + j;
                             if (n < tl.nrows) {
                                 const float h = swiglu_dev(sg * gv[j], su * uv[j], p.alpha, p.beta, p.limit);
-                                out[(size_t)(tl.row0 + n) * p.out_ld + col] = __float2bfloat16_rn(h);
+                                out[(size_t)(tl.row0 + n) * out_ld + col] = __float2bfloat16_rn(h);
+                            }
+                        }
+                    }
+                } else if (tl.dual) {
+#pragma unroll 1
+                    for (int cc = c0; cc < c0 + C::COLS && cc < n_mma; cc += C::CW) {
+                        float v[C::CW], v2[C::CW];
+                        tmem_ld_x2<C::CW>(tb + cc, tb + C::BN + cc, v, v2);
+#pragma unroll
+                        for (int j = 0; j < C::CW; ++j) {
+                            const int n = cc + j;
+                            if (n < tl.nrows) {
+                                __nv_bfloat16* row = out + (size_t)(tl.row0 + n) * out_ld;
+                                row[col] = __float2bfloat16_rn(v[j]);
+                                row[col_b] = __float2bfloat16_rn(v2[j]);
                             }
                         }
                     }
                 } else {
 #pragma unroll 1
-                    for (int cc = c0; cc < c0 + C::HALF && cc < n_mma; cc += C::CW) {
+                    for (int cc = c0; cc < c0 + C::COLS && cc < n_mma; cc += C::CW) {
                         float v[C::CW];
-                        if constexpr (C::CW == 16) tmem_ld16(tb + cc, v);
-                        else tmem_ld8(tb + cc, v);
+                        tmem_ld_x1<C::CW>(tb + cc, v);
 #pragma unroll
                         for (int j = 0; j < C::CW; ++j) {
                             const int n = cc + j;
-                            if (n < tl.nrows) out[(size_t)(tl.row0 + n) * p.out_ld + col] = __float2bfloat16_rn(v[j]);
+                            if (n < tl.nrows) out[(size_t)(tl.row0 + n) * out_ld + col] = __float2bfloat16_rn(v[j]);
                         }
                     }
                 }
@@ -369,74 +556,157 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[buf]);
                 ++it;
-            } else {
-                float acc_g[C::HALF];
-                float acc_u[C::GATED ? C::HALF : 1];
-#pragma unroll
-                for (int j = 0; j < C::HALF; ++j) acc_g[j] = 0.f;
-#pragma unroll
-                for (int j = 0; j < (C::GATED ? C::HALF : 1); ++j) acc_u[j] = 0.f;
-                const float* wsg = p.w_scale + ((size_t)tl.g * (p.wrows / 128) + tl.c) * p.kblocks;
-                const float* wsu = p.w_scale + ((size_t)tl.g * (p.wrows / 128) + p.up_off / 128 + tl.c) * p.kblocks;
-                for (int kb = 0; kb < p.num_kb; ++kb) {
-                    const uint32_t buf = it & 1, bph = (it >> 1) & 1;
-                    // Per-column activation scales of this K block (one lane per column).
-                    float sb0 = 0.f, sb1 = 0.f;
-                    {
-                        const int n = c0 + lane;
-                        if (n < tl.nrows) sb0 = __ldg(p.act_scale + (size_t)kb * p.A + tl.row0 + n);
-                        if constexpr (C::HALF > 32) {
-                            const int n2 = c0 + 32 + lane;
-                            if (n2 < tl.nrows) sb1 = __ldg(p.act_scale + (size_t)kb * p.A + tl.row0 + n2);
-                        }
+                if (g1 && p.s1 > 1) {
+                    const int r = split_arrive(tile1);
+                    if (r < 0) {
+                        ok = false;
+                        break;
                     }
-                    const float sa_g = __ldg(wsg + kb);
-                    const float sa_u = C::GATED ? __ldg(wsu + kb) : 0.f;
+                    if (r == 0) continue;  // another split of this tile writes h
+                    for (int j = 0; j < C::COLS; ++j) {
+                        const int n = c0 + j;
+                        if (n >= tl.nrows) break;
+                        float gsum = 0.f, usum = 0.f;
+                        for (int ks = 0; ks < p.s1; ++ks) {
+                            gsum += __ldcg(part_at(tile1, ks, 0, n));
+                            usum += __ldcg(part_at(tile1, ks, 1, n));
+                        }
+                        const float hv = swiglu_dev(sg * gsum, su * usum, p.alpha, p.beta, p.limit);
+                        out[(size_t)(tl.row0 + n) * out_ld + col] = __float2bfloat16_rn(hv);
+                    }
+                }
+            } else {
+                const int kblocks = (g1 ? p.H : p.I) / C::BK;  // BK = 128 for FP8: one scale per K block
+                const int kbase = g1 ? tl.ks * kblocks / p.s1 : 0;
+                const int num_kb = g1 ? (tl.ks + 1) * kblocks / p.s1 - kbase : kblocks;
+                const float* act_scale = g1 ? p.x_scale : p.h_scale;
+                // block scales of A0 and A1: weight row block a_row / 128 of the [G*rows/128][K/128] grid
+                const float* wscale = g1 ? p.w1_scale : p.w2_scale;
+                const float* wsg = wscale + (size_t)(tl.a0row / 128) * kblocks + kbase;
+                const float* wsu = wscale + (size_t)(tl.a1row / 128) * kblocks + kbase;
+                float acc_g[C::COLS], acc_u[C::COLS];
+#pragma unroll
+                for (int j = 0; j < C::COLS; ++j) acc_g[j] = acc_u[j] = 0.f;
+                // h_scale of a GEMM2 tile may have been written by other CTAs of this launch:
+                // acquire the block's counter in this warp and read the scales through L2.
+                if (!g1 && chained) {
+                    if (lane == 0) (void)ld_acquire_gpu(p.done1 + tl.blk);
+                    __syncwarp();
+                }
+                // This warp's scale products: tab[j] = sa0 * sb[c0+j], tab[COLS+j] = sa1 * sb[c0+j].
+                // The scales of block kb are loaded kPF blocks ahead (a register ring), so the
+                // L2 latency of those loads stays off the tensor core's critical path.
+                float* tab = sct + ew * 2 * C::COLS;
+                constexpr int kPF = C::BN >= 64 ? 2 : 4;
+                const bool has_col = lane < C::COLS && c0 + lane < tl.nrows;
+                const float* sb_ptr = act_scale + (size_t)kbase * p.A + tl.row0 + c0 + lane;
+                float q_sb[kPF], q_s0[kPF], q_s1[kPF];
+#pragma unroll
+                for (int i = 0; i < kPF; ++i) {
+                    const bool in = i < num_kb;
+                    q_sb[i] = (in && has_col) ? __ldcg(sb_ptr + (size_t)i * p.A) : 0.f;
+                    q_s0[i] = in ? __ldg(wsg + i) : 0.f;
+                    q_s1[i] = (in && tl.dual) ? __ldg(wsu + i) : 0.f;
+                }
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    const uint32_t buf = it % C::NBUF, bph = (it / C::NBUF) & 1;
+                    {
+                        const float sb = q_sb[0], sa0 = q_s0[0], sa1 = q_s1[0];
+#pragma unroll
+                        for (int i = 0; i + 1 < kPF; ++i) {
+                            q_sb[i] = q_sb[i + 1];
+                            q_s0[i] = q_s0[i + 1];
+                            q_s1[i] = q_s1[i + 1];
+                        }
+                        const int kn = kb + kPF;
+                        const bool in = kn < num_kb;
+                        q_sb[kPF - 1] = (in && has_col) ? __ldcg(sb_ptr + (size_t)kn * p.A) : 0.f;
+                        q_s0[kPF - 1] = in ? __ldg(wsg + kn) : 0.f;
+                        q_s1[kPF - 1] = (in && tl.dual) ? __ldg(wsu + kn) : 0.f;
+                        __syncwarp();  // the previous block's reads of tab are done
+                        if (lane < C::COLS) {
+                            tab[lane] = sa0 * sb;
+                            tab[C::COLS + lane] = sa1 * sb;
+                        }
+                        __syncwarp();
+                    }
                     if (!warp_wait(&tfull[buf], bph, ab, p.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t tb = tmem_base + lane_off + buf * C::ACC_COLS;
+                    // Partials in chunks of 16 columns; the TMEM buffer goes back to the MMA as
+                    // soon as the last chunk is in registers, before its arithmetic runs.
+                    const bool live = c0 < n_mma;  // warp-uniform
+                    if (!live) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tempty[buf]);
+                    }
 #pragma unroll
-                    for (int ch = 0; ch < C::HALF / C::CW; ++ch) {
+                    for (int ch = 0; ch < C::COLS / C::CW; ++ch) {
+                        if (!live) break;
                         const int cc = c0 + ch * C::CW;
-                        if (cc < n_mma) {
-                            float pg[C::CW], pu[C::CW];
-                            if constexpr (C::GATED) {
-                                if constexpr (C::CW == 16) tmem_ld16x2(tb + cc, tb + C::BN + cc, pg, pu);
-                                else tmem_ld8x2(tb + cc, tb + C::BN + cc, pg, pu);
-                            } else {
-                                if constexpr (C::CW == 16) tmem_ld16(tb + cc, pg);
-                                else tmem_ld8(tb + cc, pg);
-                            }
+                        float pg[C::CW], pu[C::CW];
+                        if (tl.dual) tmem_ld_x2<C::CW>(tb + cc, tb + C::BN + cc, pg, pu);
+                        else tmem_ld_x1<C::CW>(tb + cc, pg);
+                        if (ch == C::COLS / C::CW - 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&tempty[buf]);
+                        }
 #pragma unroll
-                            for (int j = 0; j < C::CW; ++j) {
-                                const int jj = ch * C::CW + j;
-                                const float sb = __shfl_sync(0xffffffffu, jj < 32 ? sb0 : sb1, jj & 31);
-                                acc_g[jj] = fmaf(pg[j], sa_g * sb, acc_g[jj]);
-                                if constexpr (C::GATED) acc_u[jj] = fmaf(pu[j], sa_u * sb, acc_u[jj]);
+                        for (int j = 0; j < C::CW; j += 4) {
+                            const int jj = ch * C::CW + j;
+                            const float4 s0 = *reinterpret_cast<const float4*>(tab + jj);
+                            ffma2(acc_g[jj], acc_g[jj + 1], pg[j], pg[j + 1], s0.x, s0.y);
+                            ffma2(acc_g[jj + 2], acc_g[jj + 3], pg[j + 2], pg[j + 3], s0.z, s0.w);
+                            if (tl.dual) {
+                                const float4 s1 = *reinterpret_cast<const float4*>(tab + C::COLS + jj);
+                                ffma2(acc_u[jj], acc_u[jj + 1], pu[j], pu[j + 1], s1.x, s1.y);
+                                ffma2(acc_u[jj + 2], acc_u[jj + 3], pu[j + 2], pu[j + 3], s1.z, s1.w);
                             }
                         }
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&tempty[buf]);
                     ++it;
                 }
                 if (!ok) break;
-                if constexpr (C::GATED) {
-                    // SwiGLU, then 1x128 E4M3 quantisation of h: the block of row r is
-                    // the 128 intermediate indices of this chunk = the 4 lane quarters.
-                    const float sg = p.gate_scale ? __ldg(p.gate_scale + tl.g) : 1.f;
-                    const float su = p.up_scale ? __ldg(p.up_scale + tl.g) : 1.f;
+                if (C::SPLIT_OK && g1 && p.s1 > 1) {
+                    // split-K: store this split's promoted sums; the last split merges
+                    const int tile1 = tl.blk * p.c1 + tl.c;
 #pragma unroll
-                    for (int j = 0; j < C::HALF; ++j) {
+                    for (int j = 0; j < C::COLS; ++j) {
+                        *part_at(tile1, tl.ks, 0, c0 + j) = acc_g[j];
+                        *part_at(tile1, tl.ks, 1, c0 + j) = acc_u[j];
+                    }
+                    const int r = split_arrive(tile1);
+                    if (r < 0) {
+                        ok = false;
+                        break;
+                    }
+                    if (r == 0) continue;  // another split of this tile writes h
+#pragma unroll
+                    for (int j = 0; j < C::COLS; ++j) {
+                        float gsum = 0.f, usum = 0.f;
+                        for (int ks = 0; ks < p.s1; ++ks) {
+                            gsum += __ldcg(part_at(tile1, ks, 0, c0 + j));
+                            usum += __ldcg(part_at(tile1, ks, 1, c0 + j));
+                        }
+                        acc_g[j] = gsum;
+                        acc_u[j] = usum;
+                    }
+                }
+                if (g1) {
+                    // SwiGLU, then 1x128 E4M3 quantisation of h: the block of row r is the
+                    // 128 intermediate indices of this chunk = the 4 lane quarters.
+#pragma unroll
+                    for (int j = 0; j < C::COLS; ++j) {
                         acc_g[j] = swiglu_dev(sg * acc_g[j], su * acc_u[j], p.alpha, p.beta, p.limit);
                         float m = fabsf(acc_g[j]);
 #pragma unroll
                         for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-                        if (lane == 0) red[(hc * 4 + q) * C::HALF + j] = m;
+                        if (lane == 0) red[(cg * 4 + q) * C::COLS + j] = m;
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(epibar);
@@ -445,37 +715,52 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     ephase ^= 1;
-                    uint8_t* out = static_cast<uint8_t*>(p.out);
+                    uint8_t* out = static_cast<uint8_t*>(p.h);
 #pragma unroll
-                    for (int j = 0; j < C::HALF; ++j) {
+                    for (int j = 0; j < C::COLS; ++j) {
                         const int n = c0 + j;
-                        float amax = red[(hc * 4 + 0) * C::HALF + j];
-                        amax = fmaxf(amax, red[(hc * 4 + 1) * C::HALF + j]);
-                        amax = fmaxf(amax, red[(hc * 4 + 2) * C::HALF + j]);
-                        amax = fmaxf(amax, red[(hc * 4 + 3) * C::HALF + j]);
+                        float amax = red[(cg * 4 + 0) * C::COLS + j];
+                        amax = fmaxf(amax, red[(cg * 4 + 1) * C::COLS + j]);
+                        amax = fmaxf(amax, red[(cg * 4 + 2) * C::COLS + j]);
+                        amax = fmaxf(amax, red[(cg * 4 + 3) * C::COLS + j]);
                         const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+                        const float inv_s = amax == 0.f ? 1.f : __fdividef(448.f, amax);
                         if (n < tl.nrows) {
-                            out[(size_t)(tl.row0 + n) * p.out_ld + col] = (uint8_t)__nv_cvt_float_to_fp8(
-                                __fdiv_rn(acc_g[j], s), __NV_SATFINITE, __NV_E4M3);
-                            if (q == 0 && lane == 0) p.out_scale[(size_t)tl.c * p.A + tl.row0 + n] = s;
+                            out[(size_t)(tl.row0 + n) * p.I + col] =
+                                (uint8_t)__nv_cvt_float_to_fp8(acc_g[j] * inv_s, __NV_SATFINITE, __NV_E4M3);
+                            if (q == 0 && lane == 0) p.h_scale[(size_t)tl.c * p.A + tl.row0 + n] = s;
                         }
                     }
-                    // red is rewritten by the next tile: everyone must have read it.
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(epibar);
-                    if (!warp_wait(epibar, ephase, ab, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    ephase ^= 1;
                 } else {
-                    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+                    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.y);
 #pragma unroll
-                    for (int j = 0; j < C::HALF; ++j) {
+                    for (int j = 0; j < C::COLS; ++j) {
                         const int n = c0 + j;
-                        if (n < tl.nrows) out[(size_t)(tl.row0 + n) * p.out_ld + col] = __float2bfloat16_rn(acc_g[j]);
+                        if (n < tl.nrows) {
+                            __nv_bfloat16* row = out + (size_t)(tl.row0 + n) * p.H;
+                            row[col] = __float2bfloat16_rn(acc_g[j]);
+                            if (tl.dual) row[col_b] = __float2bfloat16_rn(acc_u[j]);
+                        }
                     }
                 }
+            }
+            // GEMM1 tile done: publish its h rows (and scales) to GEMM2 tiles of this block.
+            // Every epilogue thread makes its stores visible at GPU scope and to the async
+            // proxy, the eight warps meet, and one thread releases the block counter. In
+            // FP8 mode this meeting also keeps `red` from being rewritten while read.
+            if (g1 && (chained || C::FP8)) {
+                if (chained) {
+                    __threadfence();
+                    fence_proxy_async_global();
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(epibar);
+                if (!warp_wait(epibar, ephase, ab, p.status)) {
+                    ok = false;
+                    break;
+                }
+                ephase ^= 1;
+                if (chained && ew == 0 && lane == 0) red_release_add_gpu(p.done1 + tl.blk, 1);
             }
         }
     }
@@ -484,6 +769,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+    // The CTA that finishes last leaves the tile counter, the exit counter and the block
+    // flags at zero for the next launch.
+    // (the flag lives in dynamic shared memory: the kernel has no static shared memory,
+    // so the whole 227 KB can be requested dynamically)
+    int* s_last = ring + kRing;
+    if (threadIdx.x == 0) {
+        *s_last = 0;
+        if (p.tile_ctr) {
+            __threadfence();
+            *s_last = atomicAdd(p.exit_ctr, 1u) == gridDim.x - 1;
+        }
+    }
+    __syncthreads();
+    if (*s_last) {
+        if (chained)
+            for (int b = threadIdx.x; b < nblk; b += blockDim.x) p.done1[b] = 0;
+        if (p.s1 > 1)
+            for (int t = threadIdx.x; t < nblk * p.c1; t += blockDim.x) p.split_cnt[t] = 0;
+        if (threadIdx.x == 0) {
+            atomicExch(p.tile_ctr, 0u);
+            atomicExch(p.exit_ctr, 0u);
+        }
     }
 }
 
@@ -529,71 +837,130 @@ int num_sms() {
 }
 
 template <class C>
-static cudaError_t launch_cfg(const GemmArgs& a, cudaStream_t stream) {
-    CUtensorMap tmA, tmB;
-    if (!make_map(&tmA, a.w, (uint64_t)a.G * a.wrows, a.K, C::FP8, 128)) return cudaErrorInvalidValue;
-    if (!make_map(&tmB, a.act, (uint64_t)a.A, a.K, C::FP8, C::BN)) return cudaErrorInvalidValue;
+static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
+    // Unused maps of an absent phase point at the present phase's buffers (never read).
+    CUtensorMap tmW1, tmX, tmW2, tmH;
+    const bool p1 = a.run_gemm1, p2 = a.run_gemm2;
+    const void* w1 = p1 ? a.w1 : a.w2;
+    const void* x = p1 ? a.x_perm : a.h;
+    const void* w2 = p2 ? a.w2 : a.w1;
+    const void* hh = p2 ? a.h : a.x_perm;
+    const uint64_t k1 = p1 ? a.H : a.I, k2 = p2 ? a.I : a.H;
+    const uint64_t r1 = p1 ? (uint64_t)a.G * 2 * a.I : (uint64_t)a.G * a.H;
+    const uint64_t r2 = p2 ? (uint64_t)a.G * a.H : (uint64_t)a.G * 2 * a.I;
+    if (!make_map(&tmW1, w1, r1, k1, C::FP8, 128) || !make_map(&tmX, x, (uint64_t)a.A, k1, C::FP8, C::BN) ||
+        !make_map(&tmW2, w2, r2, k2, C::FP8, 128) || !make_map(&tmH, hh, (uint64_t)a.A, k2, C::FP8, C::BN))
+        return cudaErrorInvalidValue;
     DevArgs p;
     p.offsets = a.offsets;
     p.G = a.G;
-    p.num_kb = a.K / C::BK;
-    p.wrows = a.wrows;
-    p.n_chunks = a.n_chunks;
-    p.up_off = a.up_off;
-    p.kblocks = a.K / 128;
-    p.A = a.A;
-    p.act_scale = a.act_scale;
-    p.w_scale = a.w_scale;
-    p.out = a.out;
-    p.out_scale = a.out_scale;
-    p.out_ld = a.out_ld;
+    p.A = (int)a.A;
+    p.H = a.H;
+    p.I = a.I;
+    p.c1 = p1 ? a.I / 128 : 0;
+    p.c2 = p2 ? (a.H / 128 + 1) / 2 : 0;
+    p.x_scale = a.x_scale;
+    p.w1_scale = a.w1_scale;
+    p.w2_scale = a.w2_scale;
     p.gate_scale = a.gate_scale;
     p.up_scale = a.up_scale;
     p.alpha = a.alpha;
     p.beta = a.beta;
     p.limit = a.limit;
+    p.h = a.h;
+    p.h_scale = a.h_scale;
+    p.y = a.y;
+    p.tile_ctr = a.tile_ctr;
+    p.exit_ctr = a.exit_ctr;
+    p.done1 = (p1 && p2) ? a.done1 : nullptr;
+    p.s1 = p1 ? gemm_split_factor(a.A, a.G, a.H, a.I, C::FP8) : 1;
+    p.part = a.part;
+    p.split_cnt = a.split_cnt;
+    if (p.s1 > 1 && (!p.part || !p.split_cnt)) return cudaErrorInvalidValue;
     p.status = a.status;
     const size_t smem = C::smem_bytes(a.G);
-    if (smem > (size_t)kSmemLimit) return cudaErrorInvalidValue;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(grouped_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kSmemLimit);
-    });
-    if (attr_err != cudaSuccess) return attr_err;
-    grouped_gemm_kernel<C><<<num_sms(), kThreads, smem, stream>>>(tmA, tmB, p);
+    static std::mutex mu;
+    static int max_dyn[64] = {0};  // per device: dynamic shared memory the kernel may request
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    int limit = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (dev >= 64 || !max_dyn[dev]) {
+            cudaFuncAttributes fa;
+            cudaError_t e = cudaFuncGetAttributes(&fa, moe_gemm_kernel<C>);
+            if (e != cudaSuccess) return e;
+            limit = kSmemLimit - (int)fa.sharedSizeBytes;
+            e = cudaFuncSetAttribute(moe_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, limit);
+            if (e != cudaSuccess) return e;
+            if (dev < 64) max_dyn[dev] = limit;
+        } else {
+            limit = max_dyn[dev];
+        }
+    }
+    if (smem > (size_t)limit) return cudaErrorInvalidValue;
+    moe_gemm_kernel<C><<<num_sms(), C::THREADS, smem, stream>>>(tmW1, tmX, tmW2, tmH, p);
     return cudaGetLastError();
 }
 
-int gemm_pick_bn(int64_t A, int G, bool gated, bool fp8) {
+int gemm_pick_bn(int64_t A, int G, bool fp8) {
     const double avg = G > 0 ? (double)A / (double)G : 0.0;
     int bn = 16;
-    while (bn < 128 && bn < 1.5 * avg) bn <<= 1;
-    if (gated && fp8 && bn > 64) bn = 64;
+    while (bn < 128 && bn < avg) bn <<= 1;  // smallest tile holding an average group
+    if (fp8 && bn > 64) bn = 64;  // FP8 keeps fp32 promotion registers for gate and up
     return bn;
 }
 
-template <int BN>
-static cudaError_t launch_bn(const GemmArgs& a, bool gated, bool fp8, cudaStream_t s) {
-    if (gated) {
-        if (fp8) {
-            if constexpr (BN <= 64) return launch_cfg<Cfg<BN, true, true>>(a, s);
-            else return cudaErrorInvalidValue;
-        }
-        return launch_cfg<Cfg<BN, true, false>>(a, s);
-    }
-    if (fp8) return launch_cfg<Cfg<BN, false, true>>(a, s);
-    return launch_cfg<Cfg<BN, false, false>>(a, s);
+int64_t gemm_max_blocks(int64_t A, int G, int bn) {
+    return (A < G ? A : (int64_t)G) + A / bn;
 }
 
-cudaError_t launch_gemm(const GemmArgs& a, bool gated, bool fp8, int bn, cudaStream_t stream) {
-    if (a.A == 0 || a.G == 0) return cudaSuccess;
+size_t gemm_block_flags_bytes(int64_t A, int G) {
+    return sizeof(int) * (size_t)(gemm_max_blocks(A, G, 16) + 1);
+}
+
+// Split GEMM1's K range when its tiles cannot fill two waves of the 148 SMs (decode-sized
+// batches), keeping at least two K blocks per split.
+int gemm_split_factor(int64_t A, int G, int H, int I, bool fp8) {
+    constexpr int64_t kTarget = 2 * 148;
+    const int bn = gemm_pick_bn(A, G, fp8);
+    const int64_t tiles = gemm_max_blocks(A, G, bn) * (I / 128);
+    const int kb = H / (fp8 ? 128 : 64);
+    if (fp8 && bn >= 64) return 1;  // the kernel variant has no split-K path
+    int s = 1;
+    while (s < 4 && tiles * s < kTarget && kb >= 4 * s) s *= 2;
+    return s;
+}
+
+size_t gemm_split_scratch_bytes(int64_t A, int G, int H, int I, bool fp8) {
+    const int s = gemm_split_factor(A, G, H, I, fp8);
+    if (s == 1) return 0;
+    const int bn = gemm_pick_bn(A, G, fp8);
+    return (size_t)gemm_max_blocks(A, G, bn) * (I / 128) * s * 2 * bn * 128 * sizeof(float);
+}
+
+size_t gemm_split_counter_bytes(int64_t A, int G, int H, int I, bool fp8) {
+    if (gemm_split_factor(A, G, H, I, fp8) == 1) return 0;
+    const int bn = gemm_pick_bn(A, G, fp8);
+    return (size_t)gemm_max_blocks(A, G, bn) * (I / 128) * sizeof(int);
+}
+
+cudaError_t launch_moe_gemm(const MoeGemmArgs& a, cudaStream_t stream) {
+    if (a.A == 0 || a.G == 0 || (!a.run_gemm1 && !a.run_gemm2)) return cudaSuccess;
+    const int bn = gemm_pick_bn(a.A, a.G, a.fp8);
+    if (a.fp8) {
+        switch (bn) {
+            case 16: return launch_cfg<Cfg<16, true>>(a, stream);
+            case 32: return launch_cfg<Cfg<32, true>>(a, stream);
+            case 64: return launch_cfg<Cfg<64, true>>(a, stream);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     switch (bn) {
-        case 16: return launch_bn<16>(a, gated, fp8, stream);
-        case 32: return launch_bn<32>(a, gated, fp8, stream);
-        case 64: return launch_bn<64>(a, gated, fp8, stream);
-        case 128: return launch_bn<128>(a, gated, fp8, stream);
+        case 16: return launch_cfg<Cfg<16, false>>(a, stream);
+        case 32: return launch_cfg<Cfg<32, false>>(a, stream);
+        case 64: return launch_cfg<Cfg<64, false>>(a, stream);
+        case 128: return launch_cfg<Cfg<128, false>>(a, stream);
         default: return cudaErrorInvalidValue;
     }
 }

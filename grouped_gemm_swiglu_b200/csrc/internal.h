@@ -14,42 +14,61 @@ cudaError_t launch_router(const float* logits, int T, int N, int S, int k, int s
                           int32_t* ids, float* w, float* sw, cudaStream_t stream);
 
 // Scratch of the permutation: per 256-token chunk counts/bases [nchunk][E] and the
-// in-chunk rank of every (token, slot) [T][k].
+// in-chunk rank of every (token, slot) [T][k]. `counter` is one word that must be zero
+// before the first call; every call leaves it at zero.
 size_t permute_scratch_bytes(int T, int k, int E);
+// `zero`/`zero_words`: an optional buffer the counting kernel clears on the way (the
+// GEMM's per-block flags of the same layer pass).
 cudaError_t launch_permute(const int32_t* ids, const void* x, int T, int H, int k, int E, int n_shared, bool fp8,
                            int32_t* offsets, int32_t* perm, int32_t* inv, void* x_perm, float* x_scale,
-                           void* scratch, int* status, cudaStream_t stream);
+                           void* scratch, unsigned int* counter, int* status, cudaStream_t stream,
+                           int* zero = nullptr, size_t zero_words = 0);
 
 cudaError_t launch_combine(const void* y, const int32_t* offsets, const int32_t* inv, const float* topk_w,
-                           const float* shared_w, int T, int H, int k, int E, int n_shared, int n_sink, void* out,
-                           cudaStream_t stream);
+                           const float* shared_w, int T, int H, int k, int E, int n_shared, int n_sink, int64_t A,
+                           void* out, int* status, cudaStream_t stream);
 
-// Grouped GEMM over the groups described by offsets. Weights are the MMA's M side
-// (128 rows per tile), permuted activation rows the N side (BN rows per tile).
-struct GemmArgs {
+// Grouped GEMM1 (+ SwiGLU) and/or GEMM2 over the groups described by offsets, in one
+// persistent launch. Weights are the MMA's M side (128 rows per tile), permuted token
+// rows the N side. With both phases, GEMM2 tiles of a token block start once the
+// block's GEMM1 tiles have published h (done1 counters, zero at launch).
+struct MoeGemmArgs {
     const int32_t* offsets;  // [G+1]
     int G;
-    int64_t A;               // rows of the activation matrix (tensor-map extent)
-    int K;                   // reduction depth (H for GEMM1, I for GEMM2)
-    int wrows;               // weight rows per group (2I for GEMM1, H for GEMM2)
-    int n_chunks;            // 128-row output chunks per group (I/128 or H/128)
-    int up_off;              // GEMM1: row offset of the up half inside a group (I)
-    const void* act;         // activation matrix [A][K]
-    const float* act_scale;  // FP8: [K/128][A]
-    const void* w;           // weights [G][wrows][K]
-    const float* w_scale;    // FP8: [G][wrows/128][K/128]
-    void* out;               // GEMM1: h [A][I]; GEMM2: y [A][H] bf16
-    float* out_scale;        // GEMM1 FP8: [I/128][A]
-    int out_ld;              // I or H
+    int64_t A;               // rows of x_perm / h / y
+    int H, I;
+    bool fp8;
+    bool run_gemm1, run_gemm2;
+    const void* x_perm;      // [A][H]
+    const float* x_scale;    // FP8: [H/128][A]
+    const void* w1;          // [G][2I][H]
+    const float* w1_scale;   // FP8: [G][2I/128][H/128]
     const float* gate_scale; // [G] or NULL
     const float* up_scale;   // [G] or NULL
     float alpha, beta, limit;
+    void* h;                 // [A][I]
+    float* h_scale;          // FP8: [I/128][A]
+    const void* w2;          // [G][H][I]
+    const float* w2_scale;   // FP8: [G][H/128][I/128]
+    void* y;                 // [A][H] bf16
+    unsigned int* tile_ctr;  // zero when idle; left at zero
+    unsigned int* exit_ctr;  // zero when idle; left at zero
+    int* done1;              // gemm_block_flags_bytes(A, G), zeroed before a two-phase launch
+    float* part;             // split-K partials of GEMM1 (gemm_split_scratch_bytes), or NULL
+    int* split_cnt;          // per GEMM1 tile: splits finished (zero when idle), or NULL
     int* status;
 };
 
-// Picks the token-tile width from the expected rows per group.
-int gemm_pick_bn(int64_t A, int G, bool gated, bool fp8);
-cudaError_t launch_gemm(const GemmArgs& a, bool gated, bool fp8, int bn, cudaStream_t stream);
+int gemm_pick_bn(int64_t A, int G, bool fp8);
+// Upper bound on token blocks: every non-empty group adds at most one partial block.
+int64_t gemm_max_blocks(int64_t A, int G, int bn);
+size_t gemm_block_flags_bytes(int64_t A, int G);
+// GEMM1 split-K factor (1, 2 or 4) for these sizes, and the scratch it needs: fp32
+// partials [tiles][splits][2][BN][128] plus one counter per GEMM1 tile.
+int gemm_split_factor(int64_t A, int G, int H, int I, bool fp8);
+size_t gemm_split_scratch_bytes(int64_t A, int G, int H, int I, bool fp8);
+size_t gemm_split_counter_bytes(int64_t A, int G, int H, int I, bool fp8);
+cudaError_t launch_moe_gemm(const MoeGemmArgs& a, cudaStream_t stream);
 
 int num_sms();
 

@@ -6,7 +6,8 @@
 // Order inside a group is (token, slot), fixed by construction, so the result does not
 // depend on scheduling: every 256-token chunk builds one membership bitmap per warp
 // and expert (atomicOr is order-free), ranks come from popcounts, and chunk bases from
-// a prefix over chunks.
+// a prefix over chunks. Two launches: count (+ scan in the CTA that finishes last), and
+// the scatter/copy.
 #include <cuda_fp8.h>
 
 #include "internal.h"
@@ -14,7 +15,9 @@
 
 namespace moe {
 
-constexpr int kChunk = 256;  // tokens per counting chunk (8 warps x 32 lanes)
+constexpr int kChunk = 256;          // tokens per counting chunk (8 warps x 32 lanes)
+constexpr int kMaxGroups = 1024 + 32;
+constexpr int kScatterThreads = 128;
 
 size_t permute_scratch_bytes(int T, int k, int E) {
     const size_t nchunk = (size_t)(T + kChunk - 1) / kChunk;
@@ -22,16 +25,50 @@ size_t permute_scratch_bytes(int T, int k, int E) {
     return al(nchunk * E * sizeof(int32_t)) + al((size_t)T * k * sizeof(int32_t));
 }
 
+// Exclusive scan of v[0..n) (n <= kMaxGroups) into out[0..n], out[n] = total; 256 threads.
+__device__ void block_exclusive_scan_256(const int32_t* v, int n, int32_t* out) {
+    __shared__ int32_t warp_tot[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int per = (n + 255) / 256;
+    const int b = min(tid * per, n), e = min(b + per, n);
+    int local = 0;
+    for (int i = b; i < e; ++i) local += v[i];
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += warp_tot[w];
+    int run = before + incl - local;
+    for (int i = b; i < e; ++i) {
+        out[i] = run;
+        run += v[i];
+    }
+    if (tid == 255) out[n] = before + incl;
+}
+
 // One CTA per 256-token chunk. Writes cnt[chunk][e] (tokens of the chunk routed to e)
-// and rank[t][j] (position of (t, j) among the chunk's rows of its expert).
+// and rank[t][j] (position of (t, j) among the chunk's rows of its expert). The CTA
+// that finishes last turns cnt into exclusive chunk bases (in place) and writes
+// offsets[0..G] (shared groups hold T rows each), then resets the counter to zero.
 __global__ void __launch_bounds__(256) permute_count_kernel(const int32_t* __restrict__ ids, int T, int k, int E,
-                                                            int32_t* __restrict__ cnt, int32_t* __restrict__ rank,
-                                                            int* status) {
+                                                            int n_shared, int32_t* __restrict__ cnt,
+                                                            int32_t* __restrict__ rank, int32_t* __restrict__ offsets,
+                                                            unsigned int* counter, int* status, int* zero,
+                                                            size_t zero_words) {
     extern __shared__ uint32_t sm[];
+    __shared__ int32_t tot[kMaxGroups];
+    __shared__ bool s_last;
     uint32_t* flags = sm;                                      // [8][E] membership bitmaps
     uint16_t* pre = reinterpret_cast<uint16_t*>(sm + 8 * E);  // [8][E] rows of earlier warps
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < 8 * E; i += blockDim.x) flags[i] = 0;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < zero_words; i += (size_t)gridDim.x * blockDim.x)
+        zero[i] = 0;
     __syncthreads();
     const int t = blockIdx.x * kChunk + threadIdx.x;
     uint32_t* f = flags + warp * E;
@@ -64,118 +101,109 @@ __global__ void __launch_bounds__(256) permute_count_kernel(const int32_t* __res
             rank[(size_t)t * k + j] = (e >= 0 && e < E) ? (int32_t)pre[warp * E + e] + __popc(f[e] & lt) : -1;
         }
     }
-}
 
-// Single CTA. Turns cnt[chunk][e] into exclusive chunk bases (in place), and writes
-// offsets[0..G] = exclusive scan of the group sizes (shared groups hold T rows).
-__global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict__ cnt, int nchunk, int E,
-                                                            int n_shared, int T, int32_t* __restrict__ offsets) {
-    extern __shared__ int32_t tot[];  // [G]
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-    const int G = E + n_shared;
-    const int cpl = (nchunk + 31) / 32;  // chunks per lane
-    for (int e = warp; e < E; e += nwarps) {
-        const int c0 = min(lane * cpl, nchunk), c1 = min(c0 + cpl, nchunk);
-        int s = 0;
-        for (int c = c0; c < c1; ++c) s += cnt[(size_t)c * E + e];
-        int incl = s;
+    // ---- the last CTA to get here scans
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(counter, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const int nchunk = gridDim.x;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = 0;
+        for (int c0 = 0; c0 < nchunk; c0 += 8) {
+            int v[8];
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += n;
+            for (int i = 0; i < 8; ++i) v[i] = (c0 + i < nchunk) ? __ldcg(cnt + (size_t)(c0 + i) * E + e) : 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (c0 + i < nchunk) {
+                    cnt[(size_t)(c0 + i) * E + e] = run;
+                    run += v[i];
+                }
         }
-        int run = incl - s;
-        for (int c = c0; c < c1; ++c) {
-            const int v = cnt[(size_t)c * E + e];
-            cnt[(size_t)c * E + e] = run;
-            run += v;
-        }
-        if (lane == 31) tot[e] = incl;
+        tot[e] = run;
     }
     for (int s = threadIdx.x; s < n_shared; s += blockDim.x) tot[E + s] = T;
     __syncthreads();
-    if (warp == 0) {
-        int carry = 0;
-        for (int base = 0; base < G; base += 32) {
-            const int g = base + lane;
-            const int v = g < G ? tot[g] : 0;
-            int incl = v;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += n;
-            }
-            if (g < G) offsets[g] = carry + incl - v;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0) offsets[G] = carry;
-    }
+    block_exclusive_scan_256(tot, E + n_shared, offsets);
+    if (threadIdx.x == 0) *counter = 0u;
 }
 
-// One warp per token: destinations of its k routed slots and n_shared shared rows,
-// perm / inv_perm, and the copy (bf16) or quantised copy (E4M3 + scales) of x[t].
+// blockIdx.x = token, blockIdx.y = 128 16-byte vectors of its row. Destinations of the
+// token's k routed slots and n_shared shared rows, perm / inv_perm (first column block),
+// and the copy (bf16) or quantised copy (E4M3 + scales) of x[t].
 template <bool FP8>
-__global__ void __launch_bounds__(256) permute_scatter_kernel(
+__global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
     const int32_t* __restrict__ ids, const int32_t* __restrict__ rank, const int32_t* __restrict__ base,
     const int32_t* __restrict__ offsets, const uint16_t* __restrict__ x, int T, int H, int k, int E, int n_shared,
     int64_t A, int32_t* __restrict__ perm, int32_t* __restrict__ inv, void* __restrict__ x_perm,
-    float* __restrict__ x_scale) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * 8 + warp;
-    if (t >= T) return;
-    int dst = -1;
-    if (lane < k) {
-        const int e = ids[(size_t)t * k + lane];
-        const int r = rank[(size_t)t * k + lane];
-        if (e >= 0 && e < E && r >= 0) dst = offsets[e] + base[(size_t)(t / kChunk) * E + e] + r;
-        inv[(size_t)t * k + lane] = dst;
-    } else if (lane < k + n_shared) {
-        dst = offsets[E + (lane - k)] + t;
-    }
-    if (dst >= 0) perm[dst] = t;
+    float* __restrict__ x_scale, int* status) {
+    __shared__ int s_dst[32];
+    const int t = blockIdx.x;
     const int nd = k + n_shared;
-    const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * H);
-    const int nvec = H / 8;
-    // Warp-uniform trip count: every lane takes part in the shuffles below.
-    for (int v0 = 0; v0 < nvec; v0 += 32) {
-        const int v = v0 + lane;
-        const bool act = v < nvec;
-        const uint4 xv = act ? __ldg(xr + v) : make_uint4(0, 0, 0, 0);
-        if constexpr (!FP8) {
-            for (int d = 0; d < nd; ++d) {
-                const int D = __shfl_sync(0xffffffffu, dst, d);
-                if (D >= 0 && act) reinterpret_cast<uint4*>(static_cast<uint16_t*>(x_perm) + (size_t)D * H)[v] = xv;
-            }
+    if (threadIdx.x < nd) {
+        const int d = threadIdx.x;
+        int64_t dst = -1;
+        if (d < k) {
+            const int e = ids[(size_t)t * k + d];
+            const int r = rank[(size_t)t * k + d];
+            if (e >= 0 && e < E && r >= 0) dst = (int64_t)offsets[e] + base[(size_t)(t / kChunk) * E + e] + r;
         } else {
-            // 16 lanes x 8 values = one 128-wide block; amax, s = amax/448 (1 if 0),
-            // code = E4M3(x/s) with round-to-nearest-even and saturation, in fp32.
-            float f[8];
-            const uint32_t wv[4] = {xv.x, xv.y, xv.z, xv.w};
+            dst = (int64_t)offsets[E + (d - k)] + t;
+        }
+        if (dst >= A) {
+            set_status(status, MOE_ERR_EXPERT_ID);
+            dst = -1;
+        }
+        s_dst[d] = (int)dst;
+        if (blockIdx.y == 0) {
+            if (d < k) inv[(size_t)t * k + d] = (int)dst;
+            if (dst >= 0) perm[dst] = t;
+        }
+    }
+    __syncthreads();
+    const int nvec = H / 8;
+    const int v = blockIdx.y * blockDim.x + threadIdx.x;
+    const bool act = v < nvec;  // nvec is a multiple of 16: a 128-wide block is all in or all out
+    const uint4 xv = act ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H) + v) : make_uint4(0, 0, 0, 0);
+    if constexpr (!FP8) {
+        if (!act) return;
+        for (int d = 0; d < nd; ++d) {
+            const int D = s_dst[d];
+            if (D >= 0) reinterpret_cast<uint4*>(static_cast<uint16_t*>(x_perm) + (size_t)D * H)[v] = xv;
+        }
+    } else {
+        // 16 threads x 8 values = one 128-wide block: amax, s = amax/448 (1 if 0),
+        // code = E4M3(x/s) with round-to-nearest-even and saturation, all in fp32.
+        float f[8];
+        const uint32_t wv[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                f[2 * i] = __uint_as_float(wv[i] << 16);
-                f[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
-            }
-            float amax = 0.f;
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(wv[i] << 16);
+            f[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+        }
+        float amax = 0.f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
 #pragma unroll
-            for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-            const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
-            uint32_t lo = 0, hi = 0;
+        for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if (!act) return;
+        const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+        uint32_t lo = 0, hi = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t q = (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(f[i], s), __NV_SATFINITE, __NV_E4M3);
-                if (i < 4) lo |= q << (8 * i);
-                else hi |= q << (8 * (i - 4));
-            }
-            const int blk = v / 16;
-            for (int d = 0; d < nd; ++d) {
-                const int D = __shfl_sync(0xffffffffu, dst, d);
-                if (D >= 0 && act) {
-                    reinterpret_cast<uint2*>(static_cast<uint8_t*>(x_perm) + (size_t)D * H)[v] = make_uint2(lo, hi);
-                    if ((lane & 15) == 0) x_scale[(size_t)blk * A + D] = s;
-                }
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t q = (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(f[i], s), __NV_SATFINITE, __NV_E4M3);
+            if (i < 4) lo |= q << (8 * i);
+            else hi |= q << (8 * (i - 4));
+        }
+        const int blk = v / 16;
+        for (int d = 0; d < nd; ++d) {
+            const int D = s_dst[d];
+            if (D >= 0) {
+                reinterpret_cast<uint2*>(static_cast<uint8_t*>(x_perm) + (size_t)D * H)[v] = make_uint2(lo, hi);
+                if ((threadIdx.x & 15) == 0) x_scale[(size_t)blk * A + D] = s;
             }
         }
     }
@@ -183,31 +211,33 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(
 
 cudaError_t launch_permute(const int32_t* ids, const void* x, int T, int H, int k, int E, int n_shared, bool fp8,
                            int32_t* offsets, int32_t* perm, int32_t* inv, void* x_perm, float* x_scale,
-                           void* scratch, int* status, cudaStream_t stream) {
+                           void* scratch, unsigned int* counter, int* status, cudaStream_t stream, int* zero,
+                           size_t zero_words) {
     const int G = E + n_shared;
     if (T == 0) return cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (G + 1), stream);
+    if (G > kMaxGroups) return cudaErrorInvalidValue;
     const int nchunk = (T + kChunk - 1) / kChunk;
     int32_t* cnt = static_cast<int32_t*>(scratch);
     int32_t* rank = reinterpret_cast<int32_t*>(static_cast<char*>(scratch) +
                                                (((size_t)nchunk * E * sizeof(int32_t) + 255) & ~size_t(255)));
     const size_t sm1 = (size_t)8 * E * sizeof(uint32_t) + (size_t)8 * E * sizeof(uint16_t);
     cudaError_t err;
-    if (sm1 > 48 * 1024) {
+    if (sm1 > 40 * 1024) {
         err = cudaFuncSetAttribute(permute_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
         if (err != cudaSuccess) return err;
     }
-    permute_count_kernel<<<nchunk, 256, sm1, stream>>>(ids, T, k, E, cnt, rank, status);
-    permute_scan_kernel<<<1, 1024, (size_t)G * sizeof(int32_t), stream>>>(cnt, nchunk, E, n_shared, T, offsets);
+    permute_count_kernel<<<nchunk, 256, sm1, stream>>>(ids, T, k, E, n_shared, cnt, rank, offsets, counter, status,
+                                                       zero, zero ? zero_words : 0);
     const int64_t A = (int64_t)T * (k + n_shared);
-    dim3 grid((T + 7) / 8);
+    dim3 grid(T, (H / 8 + kScatterThreads - 1) / kScatterThreads);
     if (fp8)
-        permute_scatter_kernel<true><<<grid, 256, 0, stream>>>(ids, rank, cnt, offsets,
-                                                               static_cast<const uint16_t*>(x), T, H, k, E,
-                                                               n_shared, A, perm, inv, x_perm, x_scale);
+        permute_scatter_kernel<true><<<grid, kScatterThreads, 0, stream>>>(
+            ids, rank, cnt, offsets, static_cast<const uint16_t*>(x), T, H, k, E, n_shared, A, perm, inv, x_perm,
+            x_scale, status);
     else
-        permute_scatter_kernel<false><<<grid, 256, 0, stream>>>(ids, rank, cnt, offsets,
-                                                                static_cast<const uint16_t*>(x), T, H, k, E,
-                                                                n_shared, A, perm, inv, x_perm, x_scale);
+        permute_scatter_kernel<false><<<grid, kScatterThreads, 0, stream>>>(
+            ids, rank, cnt, offsets, static_cast<const uint16_t*>(x), T, H, k, E, n_shared, A, perm, inv, x_perm,
+            x_scale, status);
     return cudaGetLastError();
 }
 

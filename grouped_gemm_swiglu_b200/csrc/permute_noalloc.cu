@@ -65,8 +65,8 @@ extern "C" int moe_permute_noalloc(const int32_t* topk_ids, const void* x, const
         if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(x_perm) % 16)
             return MOE_ERR_INVALID_ARG;
     }
-    // Sizes beyond the static scratch are refused up front.
-    if (moe::permute_scratch_bytes(d->T, d->k, d->E) > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
+    // Sizes beyond the static scratch (after its 256-byte counter header) are refused up front.
+    if (moe::permute_scratch_bytes(d->T, d->k, d->E) > kNoAllocScratchBytes - 256) return MOE_ERR_WORKSPACE;
     int major = 0, dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
@@ -75,9 +75,12 @@ extern "C" int moe_permute_noalloc(const int32_t* topk_ids, const void* x, const
     void* scratch = nullptr;
     int rc = scratch_address(&scratch);
     if (rc != MOE_OK) return rc;
-    // Nothing in the scratch has to start at zero: every call writes the counts and
-    // ranks it later reads. The status word, when given, is the caller's.
+    // The first word of the array counts finished CTAs of the counting kernel; it must be
+    // zero when a call starts. It is zero at module load and every call leaves it at zero;
+    // the rest of the array is written before it is read. The status word is the caller's.
+    unsigned int* counter = static_cast<unsigned int*>(scratch);
     cudaError_t e = moe::launch_permute(topk_ids, x, d->T, d->H, d->k, d->E, d->n_shared, fp8, offsets, perm,
-                                        inv_perm, x_perm, x_scale, scratch, status, static_cast<cudaStream_t>(stream));
+                                        inv_perm, x_perm, x_scale, static_cast<char*>(scratch) + 256, counter, status,
+                                        static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

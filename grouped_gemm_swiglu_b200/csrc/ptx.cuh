@@ -10,17 +10,13 @@
 namespace moe {
 
 // Longest time any single pipeline wait may take before the kernel gives up, sets
-// MOE_ERR_TIMEOUT in the status word and drains. Whole launches take milliseconds.
-constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
+// MOE_ERR_TIMEOUT in the status word and drains: 2^31 SM cycles (about 1.1 s at the
+// 1965 MHz maximum clock, longer at lower clocks). Whole launches take milliseconds.
+// The SM cycle counter is used because it is cheap to read on every slow poll.
+constexpr long long kWaitLimitCycles = 1ll << 31;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ unsigned long long globaltimer_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
 }
 
 // ------------------------------------------------------------------ mbarrier
@@ -45,14 +41,17 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Test for completion of the phase with the given parity. The thread may be suspended
+// for up to the hint (in ns) while the phase is pending; it resumes when the phase
+// completes, so the hint only reduces polling.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(20000u)
         : "memory");
     return ok != 0;
 }
@@ -64,20 +63,20 @@ struct PipeAbort {
 
 // Wait until the phase with the given parity of `bar` has completed. Returns false
 // (and leaves the wait) when this CTA has aborted or when the wait exceeds
-// kWaitLimitNs, in which case it records MOE_ERR_TIMEOUT and raises the abort flag.
+// kWaitLimitCycles, in which case it records MOE_ERR_TIMEOUT and raises the abort flag.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, PipeAbort* ab, int* status) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
-    const unsigned long long t0 = globaltimer_ns();
-    while (true) {
-        #pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(a, parity)) return true;
-        if (ab->flag) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            ab->flag = 1;
-            if (status) atomicCAS(status, 0, MOE_ERR_TIMEOUT);
-            return false;
+    const long long t0 = clock64();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(a, parity)) return true;
+        if ((n & 15) == 0) {
+            if (ab->flag) return false;
+            if (clock64() - t0 > kWaitLimitCycles) {
+                ab->flag = 1;
+                if (status) atomicCAS(status, 0, MOE_ERR_TIMEOUT);
+                return false;
+            }
         }
     }
 }
@@ -85,10 +84,46 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, PipeAb
 // Drain wait used on the abort path only: no abort check, same time limit.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
     const uint32_t a = smem_u32(bar);
-    const unsigned long long t0 = globaltimer_ns();
+    const long long t0 = clock64();
     while (!mbar_try_wait(a, parity)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+        if (clock64() - t0 > kWaitLimitCycles) return false;
     }
+    return true;
+}
+
+// ------------------------------------------------------------------ global flags
+// Makes this thread's earlier generic-proxy global accesses ordered with its later
+// async-proxy (TMA) accesses, and the other way round.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_add_gpu(int* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Wait until *p >= target (another CTA's release-add), bounded like mbar_wait. On
+// success the data published before the add is visible to this thread's later TMA loads.
+__device__ __forceinline__ bool wait_counter_geq(const int* p, int target, PipeAbort* ab, int* status) {
+    if (ld_acquire_gpu(p) < target) {
+        const long long t0 = clock64();
+        while (ld_acquire_gpu(p) < target) {
+            if (ab->flag) return false;
+            if (clock64() - t0 > kWaitLimitCycles) {
+                ab->flag = 1;
+                if (status) atomicCAS(status, 0, MOE_ERR_TIMEOUT);
+                return false;
+            }
+            __nanosleep(64);
+        }
+    }
+    fence_proxy_async_global();
     return true;
 }
 
@@ -252,6 +287,79 @@ __device__ __forceinline__ void tmem_ld8(uint32_t ta, float* a) {
         : "memory");
 #pragma unroll
     for (int i = 0; i < 8; ++i) a[i] = __uint_as_float(r[i]);
+}
+
+// 4-column variants (used when a warp's column share is 4).
+__device__ __forceinline__ void tmem_ld4x2(uint32_t ta, uint32_t tb, float* a, float* b) {
+    uint32_t r[8];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%8];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%4, %5, %6, %7}, [%9];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+        : "r"(ta), "r"(tb)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        a[i] = __uint_as_float(r[i]);
+        b[i] = __uint_as_float(r[4 + i]);
+    }
+}
+
+__device__ __forceinline__ void tmem_ld4(uint32_t ta, float* a) {
+    uint32_t r[4];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+        : "r"(ta)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = __uint_as_float(r[i]);
+}
+
+// 32 consecutive columns from each of two addresses (four x16 loads, one wait).
+__device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, float* a, float* b) {
+    uint32_t r[64];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%65];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47}, [%66];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%67];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(ta), "r"(ta + 16), "r"(tb), "r"(tb + 16)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        a[i] = __uint_as_float(r[i]);
+        b[i] = __uint_as_float(r[32 + i]);
+    }
+}
+
+// 32 consecutive columns from one address (two x16 loads, one wait).
+__device__ __forceinline__ void tmem_ld32(uint32_t ta, float* a) {
+    float b[16];
+    tmem_ld16x2(ta, ta + 16, a, b);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a[16 + i] = b[i];
+}
+
+// CW consecutive columns from each of two addresses (CW in {4, 8, 16, 32}), one wait.
+template <int CW>
+__device__ __forceinline__ void tmem_ld_x2(uint32_t ta, uint32_t tb, float* a, float* b) {
+    if constexpr (CW == 32) tmem_ld32x2(ta, tb, a, b);
+    else if constexpr (CW == 16) tmem_ld16x2(ta, tb, a, b);
+    else if constexpr (CW == 8) tmem_ld8x2(ta, tb, a, b);
+    else tmem_ld4x2(ta, tb, a, b);
+}
+
+template <int CW>
+__device__ __forceinline__ void tmem_ld_x1(uint32_t ta, float* a) {
+    if constexpr (CW == 32) tmem_ld32(ta, a);
+    else if constexpr (CW == 16) tmem_ld16(ta, a);
+    else if constexpr (CW == 8) tmem_ld8(ta, a);
+    else tmem_ld4(ta, a);
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {

@@ -33,10 +33,12 @@
  *     default stream) and returns before it runs. Calls are capturable in a CUDA graph.
  *   - Arguments are checked on the host first. A bad argument returns a negative
  *     moe_status and enqueues nothing. A kernel launch failure returns MOE_ERR_CUDA.
- *   - Errors found while the kernels run (an expert id outside [0, E); a pipeline wait
- *     that exceeded its time limit) are written to a status word at the start of the
- *     workspace `ws`; read it with moe_read_status(). It is sticky until
- *     moe_clear_status(). No kernel traps.
+ *   - Errors found while the kernels run (an expert id outside [0, E) or repeated
+ *     within a token, offsets or inverse-permutation entries outside [0, A], a pipeline
+ *     wait that exceeded its time limit) are written to a status word at the start of
+ *     the workspace `ws`; read it with moe_read_status(). It is sticky until
+ *     moe_clear_status(). Offending entries are dropped or clamped, never used to read
+ *     or write out of bounds. No kernel traps.
  *   - Row-major layouts throughout. bf16 is stored as 16-bit words, E4M3 as bytes.
  *   - Calls that share a workspace or outputs must not overlap on the GPU.
  */
@@ -58,7 +60,8 @@ typedef enum moe_status {
     MOE_ERR_UNSUPPORTED = -2,  /* a valid combination this build does not implement */
     MOE_ERR_ARCH = -3,         /* the current device is not compute capability 10.x */
     MOE_ERR_WORKSPACE = -4,    /* ws is NULL, misaligned (256 B) or smaller than required */
-    MOE_ERR_EXPERT_ID = -5,    /* (device) a routing id lies outside [0, E) */
+    MOE_ERR_EXPERT_ID = -5,    /* (device) routing data out of range: an id outside [0, E) or
+                                  repeated in a token, offsets / inv_perm outside [0, A] */
     MOE_ERR_TIMEOUT = -6,      /* (device) a pipeline wait exceeded its limit; outputs invalid */
     MOE_ERR_CUDA = -7          /* a CUDA runtime/driver call failed */
 } moe_status;
@@ -102,7 +105,9 @@ typedef enum moe_ws_kind {
     MOE_WS_PERMUTE = 0,
     MOE_WS_GEMM1 = 1,
     MOE_WS_GEMM2_COMBINE = 2,
-    MOE_WS_FORWARD = 3
+    MOE_WS_FORWARD = 3,
+    MOE_WS_EXPERTS = 4,
+    MOE_WS_COMBINE = 5
 } moe_ws_kind;
 
 /* ABI version compiled into the library (MOE_ABI_VERSION). */
@@ -112,8 +117,9 @@ int moe_abi_version(void);
 const char* moe_status_string(int status);
 
 /* Bytes of device workspace the given call needs for these dims (written to *bytes).
- * The workspace must be 256-byte aligned. Its first 256 bytes hold the status word;
- * zero them once (moe_clear_status) before first use. */
+ * The workspace must be 256-byte aligned. Its first 256 bytes hold the status word and
+ * a completion counter of the permutation; zero them once (moe_clear_status) before
+ * first use. Every call leaves the counter at zero again. */
 int moe_workspace_size(const moe_dims* dims, int kind, size_t* bytes);
 
 /* Copies the workspace's device status word to *status (host). Synchronises `stream`.
@@ -174,8 +180,10 @@ int moe_permute(const int32_t* topk_ids, const void* x, const moe_dims* dims,
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress); make that first call before any stream capture.
  *   Every call shares the array: calls that overlap on the GPU (two streams, or two
- *   host threads) race and corrupt each other's results. Nothing in it has to be
- *   zeroed: each call writes what it reads.
+ *   host threads) race and corrupt each other's results. Its first word counts the
+ *   CTAs of a call that have finished counting and must be zero when a call starts: it
+ *   is zero when the library loads and every call leaves it at zero; the rest of the
+ *   array is written by each call before it is read.
  * Errors: INVALID_ARG, WORKSPACE (too large), ARCH, CUDA. */
 int moe_permute_noalloc(const int32_t* topk_ids, const void* x, const moe_dims* dims,
                         int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* x_perm,
@@ -216,8 +224,36 @@ int moe_gemm2_combine(const void* h, const float* h_scale, const int32_t* offset
                       const void* w2, const float* w2_scale, const moe_dims* dims,
                       void* out, void* ws, size_t ws_bytes, void* stream);
 
-/* The whole layer: moe_route_topk, moe_permute, moe_gemm1_swiglu, moe_gemm2_combine in
- * sequence on `stream`, with every intermediate in the workspace
+/* Both grouped GEMMs in one persistent launch (the expert MLPs of every group):
+ * h = SwiGLU(GEMM1) exactly as moe_gemm1_swiglu, then y[r] = h[r] . W2[g]^T (fp32
+ * accumulation, bf16 out, unweighted) as the first half of moe_gemm2_combine. GEMM2 work
+ * on a block of rows starts as soon as that block's h is complete, so the two GEMMs
+ * overlap. ([P2] "Modifications", [P4] "Summary", [P5] per-expert dispatch.)
+ *   Inputs as moe_gemm1_swiglu plus w2 / w2_scale as moe_gemm2_combine.
+ *   h [A][I] (+ h_scale [I/128][A] for FP8) and y [A][H] bf16 are outputs.
+ *   ws: moe_workspace_size(MOE_WS_EXPERTS); besides the header it holds per-block
+ *   completion flags that must be zero when a call starts: zero the whole workspace once
+ *   after allocating it; every call leaves the flags at zero.
+ * Errors: INVALID_ARG, WORKSPACE, ARCH, CUDA; TIMEOUT / EXPERT_ID in the status word. */
+int moe_experts(const void* x_perm, const float* x_scale, const int32_t* offsets, const void* w1,
+                const float* w1_scale, const float* gate_scale, const float* up_scale,
+                const void* w2, const float* w2_scale, const moe_dims* dims, void* h,
+                float* h_scale, void* y, void* ws, size_t ws_bytes, void* stream);
+
+/* The routing-weighted combine alone ([P5] slot-specific weighted reduction):
+ *   out[t] = sum_{j<k} topk_w[t][j] * y[inv_perm[t][j]]
+ *          + sum_{s<n_shared} gamma[t][s] * y[offsets[E+s] + t]
+ * in fp32 in that order, one rounding to bf16; gamma as in moe_gemm2_combine.
+ *   y [A][H] bf16 (as written by moe_experts), offsets, inv_perm [T][k], topk_w [T][k],
+ *   shared_w [T][n_sink] (NULL iff n_sink == 0); out [T][H] bf16.
+ *   ws: moe_workspace_size(MOE_WS_COMBINE) (the status header).
+ * Errors: INVALID_ARG, WORKSPACE, ARCH, CUDA; EXPERT_ID in the status word. */
+int moe_combine(const void* y, const int32_t* offsets, const int32_t* inv_perm,
+                const float* topk_w, const float* shared_w, const moe_dims* dims, void* out,
+                void* ws, size_t ws_bytes, void* stream);
+
+/* The whole layer: moe_route_topk, moe_permute, moe_experts and moe_combine in sequence
+ * on `stream`, with every intermediate in the workspace
  * (moe_workspace_size(MOE_WS_FORWARD)).
  *   logits [T][E+n_sink] fp32, x [T][H] bf16, weights and scales as above.
  *   out [T][H] bf16 out.

@@ -82,7 +82,7 @@ def test_workspace_sizes_cover_the_intermediates(L, name):
         need += (H // 128 + I // 128) * A * 4
     assert fwd >= need + 256
     assert fwd % 256 == 0
-    assert moe.moe_workspace_size(d, moe.MOE_WS_GEMM1) == 256
+    assert moe.moe_workspace_size(d, moe.MOE_WS_GEMM1) >= 256
     assert moe.moe_workspace_size(d, moe.MOE_WS_GEMM2_COMBINE) >= A * H * 2
     assert moe.moe_workspace_size(d, moe.MOE_WS_PERMUTE) >= d.T * d.k * 4
 

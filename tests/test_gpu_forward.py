@@ -78,3 +78,47 @@ def test_forward_skewed_routing_one_hot_expert():
     assert set(np.unique(ids.cpu().numpy()).tolist()) == {0, 1, 2, 3}
     ref = oracle_layer(wl, inp).moe_rows(np.arange(200, dtype=np.int32))
     assert_bf16_close(out.float().cpu().numpy(), ref, "skewed")
+
+
+@pytest.mark.parametrize("name", ["oai_swiglu", "decode_t8", "glm_fp8"])
+def test_public_stage_calls_reproduce_forward(name):
+    """moe_route_topk -> moe_permute -> moe_experts -> moe_combine gives moe_forward's
+    output bit for bit (same kernels, deterministic order), and matches the oracle."""
+    wl = W.WORKLOADS[name]
+    if name == "glm_fp8":
+        wl = wl.with_(T=512)
+    inp = W.make_inputs(wl, "cuda")
+    out_f, *_ = run_forward(wl, inp)
+    d = moe.MoeDims.of(wl)
+    fp8 = wl.wdtype == W.WDTYPE_FP8
+    A, G, T = d.A, d.G, wl.T
+    dev = "cuda"
+    ids = torch.empty((T, wl.k), dtype=torch.int32, device=dev)
+    tw = torch.empty((T, wl.k), dtype=torch.float32, device=dev)
+    sw = torch.empty((T, wl.n_sink), dtype=torch.float32, device=dev) if wl.n_sink else None
+    offsets = torch.empty((G + 1,), dtype=torch.int32, device=dev)
+    perm = torch.empty((A,), dtype=torch.int32, device=dev)
+    inv = torch.empty((T, wl.k), dtype=torch.int32, device=dev)
+    xp = torch.empty((A, wl.H), dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev)
+    xs = torch.empty((wl.H // 128, A), dtype=torch.float32, device=dev) if fp8 else None
+    h = torch.empty((A, wl.I), dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev)
+    hs = torch.empty((wl.I // 128, A), dtype=torch.float32, device=dev) if fp8 else None
+    y = torch.empty((A, wl.H), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((T, wl.H), dtype=torch.bfloat16, device=dev)
+    ws_p = moe.alloc_workspace(d, moe.MOE_WS_PERMUTE)
+    ws_e = moe.alloc_workspace(d, moe.MOE_WS_EXPERTS)
+    ws_c = moe.alloc_workspace(d, moe.MOE_WS_COMBINE)
+    for _ in range(2):  # a second pass checks that the experts workspace is left reusable
+        moe.moe_route_topk(inp["logits"], d, ids, tw, sw)
+        moe.moe_permute(ids, inp["x"], d, offsets, perm, inv, xp, xs, ws_p)
+        moe.moe_experts(xp, xs, offsets, inp["w1"], inp["w1_scale"], inp["gate_scale"], inp["up_scale"],
+                        inp["w2"], inp["w2_scale"], d, h, hs, y, ws_e)
+        moe.moe_combine(y, offsets, inv, tw, sw, d, out, ws_c)
+        torch.cuda.synchronize()
+        for ws in (ws_p, ws_e, ws_c):
+            assert moe.moe_read_status(ws) == 0
+        assert torch.equal(out, out_f)
+    toks = sample_tokens(T, 16, seed=2)
+    ref = oracle_layer(wl, inp).moe_rows(toks)
+    got = out.float().cpu().numpy()[toks]
+    (assert_fp8_close if fp8 else assert_bf16_close)(got, ref, name)
