@@ -62,6 +62,10 @@ struct Cfg {
     static constexpr int A_BYTES = 128 * 128;
     static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES;  // sized for GEMM1 (gate + up)
+    // Token rows arrive in boxes of up to 64 rows, and only the boxes a tile's rows reach
+    // are loaded, so a short token block does not pull a full BN-row tile through L2.
+    static constexpr int BOX_ROWS = BN < 64 ? BN : 64;
+    static constexpr int BOX_BYTES = BOX_ROWS * 128;
     // as many stages as fit next to the control block and the largest group table
     static constexpr int STAGE_BUDGET = kSmemLimit - 1024 - 8 * (kMaxGroupsGemm + 1) - 1024 - 4 * 16 * 16 * 3;
     static constexpr int STAGES_RAW = STAGE_BUDGET / STAGE_BYTES;
@@ -69,11 +73,14 @@ struct Cfg {
     static constexpr int ACC_COLS = 2 * BN;  // one TMEM buffer: gate | up (GEMM2 uses the first BN)
     // bf16 hands one buffer per tile to the epilogue, FP8 one per 128-deep K block, so
     // FP8 keeps up to four partial buffers in flight.
-    static constexpr int NBUF = (FP8 && 4 * ACC_COLS <= 512) ? 4 : 2;
+    // At 256 token columns gate | up fill all 512 TMEM columns: one buffer, and the TMA
+    // ring keeps streaming the next tile while the epilogue drains it.
+    static constexpr int NBUF = (FP8 && 4 * ACC_COLS <= 512) ? 4 : (2 * ACC_COLS <= 512 ? 2 : 1);
     static constexpr int TMEM_COLS = pow2_at_least(NBUF * ACC_COLS);
-    // Epilogue warps: two groups of four (one warp per TMEM lane quarter), each group
-    // owning half of the tile's columns.
-    static constexpr int EPI = 8;
+    // Epilogue warps: groups of four (one warp per TMEM lane quarter), each group owning
+    // an equal share of the tile's columns; four groups at 256 columns, whose single
+    // accumulator buffer makes the drain time part of the tile time.
+    static constexpr int EPI = BN >= 256 ? 16 : 8;
     static constexpr int THREADS = 64 + 32 * EPI;
     static constexpr int GROUPS = EPI / 4;
     static constexpr int COLS = BN / GROUPS;  // columns per epilogue warp
@@ -85,6 +92,7 @@ struct Cfg {
     static_assert(TMEM_COLS <= 512, "TMEM holds 512 columns");
     static_assert(COLS % CW == 0 && CW >= 4, "column share must be a multiple of the load width");
     static_assert(!FP8 || COLS <= 32, "FP8 loads a warp's whole column share at once");
+    static_assert(BN % BOX_ROWS == 0 && BN <= 256, "token tile = whole boxes, at most the MMA's N limit");
     static_assert(STAGES >= 2, "at least two pipeline stages");
     // Split-K of GEMM1 is compiled in where it can be chosen (see gemm_split_factor):
     // every tile width except FP8 at 64 columns, whose promotion registers are full.
@@ -179,11 +187,13 @@ __device__ __forceinline__ Tile decode_tile(int L, int T1, const int32_t* blk_st
     return t;
 }
 
+// g * sigmoid(alpha*g) * (u + beta) written as g*(u+beta) / (1 + exp(-alpha*g)): one
+// exponential and one fast reciprocal-multiply. A huge negative g sends the denominator
+// to +inf and the quotient to the limit value 0.
 __device__ __forceinline__ float swiglu_dev(float gate, float up, float alpha, float beta, float limit) {
     const float g = fminf(gate, limit);
     const float u = fminf(fmaxf(up, -limit), limit);
-    const float sig = 1.f / (1.f + __expf(-alpha * g));
-    return g * sig * (u + beta);
+    return __fdividef(g * (u + beta), 1.f + __expf(-alpha * g));
 }
 
 // a0 += p0 * s0, a1 += p1 * s1 as one packed fp32x2 fused multiply-add.
@@ -319,7 +329,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const int all_kb = (g1 ? p.H : p.I) / C::BK;
                 const int kbase = g1 ? tl.ks * all_kb / p.s1 : 0;  // this tile's K blocks
                 const int num_kb = g1 ? (tl.ks + 1) * all_kb / p.s1 - kbase : all_kb;
-                const uint32_t tx = (tl.dual ? 2 : 1) * C::A_BYTES + C::B_BYTES;
+                const int n_box = (max(16, (tl.nrows + 15) & ~15) + C::BOX_ROWS - 1) / C::BOX_ROWS;
+                const uint32_t tx = (tl.dual ? 2 : 1) * C::A_BYTES + n_box * C::BOX_BYTES;
+                auto load_act = [&](uint8_t* st, uint64_t* bar, int kx) {
+                    for (int r = 0; r < n_box; ++r)
+                        tma_load_2d(st + 2 * C::A_BYTES + r * C::BOX_BYTES, ta, bar, kx, tl.row0 + r * C::BOX_ROWS);
+                };
                 // GEMM2 after GEMM1 in the same launch: weights of the first stages go out
                 // before waiting for the block's h rows.
                 const bool dep = chained && !g1;
@@ -332,8 +347,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     const bool dep_ok = wait_counter_geq(p.done1 + tl.blk, p.c1, ab, p.status);
                     uint32_t s2 = st0;
                     for (int k2 = 0; k2 < pre; ++k2) {
-                        tma_load_2d(smem + (size_t)s2 * C::STAGE_BYTES + 2 * C::A_BYTES, ta, &full[s2],
-                                    (kbase + k2) * C::BK, tl.row0);
+                        load_act(smem + (size_t)s2 * C::STAGE_BYTES, &full[s2], (kbase + k2) * C::BK);
                         if (++s2 == (uint32_t)C::STAGES) s2 = 0;
                     }
                     return dep_ok;
@@ -352,7 +366,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     const int kx = (kbase + kb) * C::BK;
                     tma_load_2d(st, tw, &full[stage], kx, tl.a0row);
                     if (tl.dual) tma_load_2d(st + C::A_BYTES, tw, &full[stage], kx, tl.a1row);
-                    if (kb >= pre) tma_load_2d(st + 2 * C::A_BYTES, ta, &full[stage], kx, tl.row0);
+                    if (kb >= pre) load_act(st, &full[stage], kx);
                     pend_mask |= 1u << stage;
                     pend_phase = (pend_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == (uint32_t)C::STAGES) {
@@ -848,8 +862,8 @@ static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
     const uint64_t k1 = p1 ? a.H : a.I, k2 = p2 ? a.I : a.H;
     const uint64_t r1 = p1 ? (uint64_t)a.G * 2 * a.I : (uint64_t)a.G * a.H;
     const uint64_t r2 = p2 ? (uint64_t)a.G * a.H : (uint64_t)a.G * 2 * a.I;
-    if (!make_map(&tmW1, w1, r1, k1, C::FP8, 128) || !make_map(&tmX, x, (uint64_t)a.A, k1, C::FP8, C::BN) ||
-        !make_map(&tmW2, w2, r2, k2, C::FP8, 128) || !make_map(&tmH, hh, (uint64_t)a.A, k2, C::FP8, C::BN))
+    if (!make_map(&tmW1, w1, r1, k1, C::FP8, 128) || !make_map(&tmX, x, (uint64_t)a.A, k1, C::FP8, C::BOX_ROWS) ||
+        !make_map(&tmW2, w2, r2, k2, C::FP8, 128) || !make_map(&tmH, hh, (uint64_t)a.A, k2, C::FP8, C::BOX_ROWS))
         return cudaErrorInvalidValue;
     DevArgs p;
     p.offsets = a.offsets;
@@ -906,7 +920,7 @@ static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
 int gemm_pick_bn(int64_t A, int G, bool fp8) {
     const double avg = G > 0 ? (double)A / (double)G : 0.0;
     int bn = 16;
-    while (bn < 128 && bn < avg) bn <<= 1;  // smallest tile holding an average group
+    while (bn < 256 && bn < avg) bn <<= 1;  // smallest tile holding an average group
     if (fp8 && bn > 64) bn = 64;  // FP8 keeps fp32 promotion registers for gate and up
     return bn;
 }
@@ -961,6 +975,7 @@ cudaError_t launch_moe_gemm(const MoeGemmArgs& a, cudaStream_t stream) {
         case 32: return launch_cfg<Cfg<32, false>>(a, stream);
         case 64: return launch_cfg<Cfg<64, false>>(a, stream);
         case 128: return launch_cfg<Cfg<128, false>>(a, stream);
+        case 256: return launch_cfg<Cfg<256, false>>(a, stream);
         default: return cudaErrorInvalidValue;
     }
 }

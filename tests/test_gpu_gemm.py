@@ -1,6 +1,6 @@
 """Grouped GEMM1 (+ SwiGLU epilogue) and GEMM2 (+ weighted combine) on the GPU against
 the oracle, on synthetic permuted inputs that span several tiles, every token-tile width
-(16/32/64/128 rows), ragged group tails, empty groups and shared groups."""
+(16/32/64/128/256 rows), ragged group tails, empty groups and shared groups."""
 import math
 
 import numpy as np
@@ -68,6 +68,8 @@ GEMM1_CASES = [
     (128, 8, 2, 0, 512, 384, False, {"scales": True}),          # tile 64, per-group gate/up scales
     (512, 8, 2, 0, 512, 256, False, {"skew": 3.0}),             # tile 128, several blocks, ragged tails
     (300, 16, 4, 1, 512, 256, False, {}),                       # a shared group of T rows
+    (1024, 8, 2, 0, 512, 256, False, {"skew": 2.0}),            # tile 256, several blocks, ragged tails
+    (600, 4, 2, 1, 512, 384, False, {"scales": True}),          # tile 256, shared group of 600 rows
     (96, 32, 4, 0, 2048, 768, False, {"oai": True}),            # OAI-SwiGLU shape and parameters
     (512, 8, 2, 0, 512, 256, True, {}),                         # FP8, tile 64
     (40, 32, 4, 1, 512, 256, True, {"glm": True}),              # FP8, tile 16, shared group, L = 10
@@ -112,6 +114,8 @@ GEMM2_CASES = [
     (512, 8, 2, 0, 512, 256, False, False),
     (300, 16, 4, 2, 512, 256, False, True),     # two sink-gated shared groups
     (300, 16, 4, 1, 512, 256, False, False),    # one shared group with weight 1
+    (1024, 8, 2, 0, 512, 256, False, False),    # tile 256
+    (600, 4, 2, 1, 384, 256, False, True),      # tile 256, odd number of 128-row chunks of H
     (512, 8, 2, 0, 512, 256, True, False),
     (40, 32, 4, 1, 512, 256, True, False),
 ]
