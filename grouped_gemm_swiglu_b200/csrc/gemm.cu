@@ -94,6 +94,7 @@ struct Cfg {
     static_assert(!FP8 || COLS <= 32, "FP8 loads a warp's whole column share at once");
     static_assert(BN % BOX_ROWS == 0 && BN <= 256, "token tile = whole boxes, at most the MMA's N limit");
     static_assert(STAGES >= 2, "at least two pipeline stages");
+    static_assert(COLS % 8 == 0, "split-K merges columns in chunks of 8");
     // Split-K of GEMM1 is compiled in where it can be chosen (see gemm_split_factor):
     // every tile width except FP8 at 64 columns, whose promotion registers are full.
     static constexpr bool SPLIT_OK = !(FP8 && BN >= 64);
@@ -144,6 +145,9 @@ struct Tile {
 };
 
 // blk_start: first token block of each group; s_off: group bounds clamped into [0, A].
+// All GEMM1 units are claimed before any GEMM2 tile (interleaving the GEMM2 tiles of a
+// block one or two waves after its GEMM1 units measured slower: they hold their SM while
+// waiting for inputs still in flight).
 template <int BN>
 __device__ __forceinline__ Tile decode_tile(int L, int T1, const int32_t* blk_start, const int32_t* s_off,
                                             const DevArgs& p) {
@@ -203,6 +207,35 @@ __device__ __forceinline__ void ffma2(float& a0, float& a1, float p0, float p1, 
         "fma.rn.f32x2 d, x, y, z;\n\tmov.b64 {%0, %1}, d;\n\t}\n"
         : "+f"(a0), "+f"(a1)
         : "f"(p0), "f"(p1), "f"(s0), "f"(s1));
+}
+
+// Split-K merge: the sums over splits 0..s1-1 of the gate and up partials of CH
+// consecutive columns from `col`, this thread's row. part_tile is the tile's partials,
+// laid out [split][gate, up][bn][128 rows]. Splits are read four at a time with every
+// load of a group issued before its first add: one L2 round trip per four splits.
+template <int CH>
+__device__ __forceinline__ void sum_split_partials(const float* part_tile, int s1, int bn, int col, int row, float* g,
+                                                   float* u) {
+#pragma unroll
+    for (int j = 0; j < CH; ++j) g[j] = u[j] = 0.f;
+#pragma unroll 1
+    for (int k0 = 0; k0 < s1; k0 += 4) {
+        float pg[4][CH], pu[4][CH];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+            for (int j = 0; j < CH; ++j) {
+                const float* q = part_tile + ((size_t)(2 * (k0 + kk)) * bn + col + j) * 128 + row;
+                pg[kk][j] = k0 + kk < s1 ? __ldcg(q) : 0.f;
+                pu[kk][j] = k0 + kk < s1 ? __ldcg(q + (size_t)bn * 128) : 0.f;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < CH; ++j) {
+            g[j] += (pg[0][j] + pg[1][j]) + (pg[2][j] + pg[3][j]);
+            u[j] += (pu[0][j] + pu[1][j]) + (pu[2][j] + pu[3][j]);
+        }
+    }
 }
 
 // Warp-collective bounded wait: lane 0 waits, the verdict is broadcast.
@@ -577,16 +610,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         break;
                     }
                     if (r == 0) continue;  // another split of this tile writes h
-                    for (int j = 0; j < C::COLS; ++j) {
-                        const int n = c0 + j;
-                        if (n >= tl.nrows) break;
-                        float gsum = 0.f, usum = 0.f;
-                        for (int ks = 0; ks < p.s1; ++ks) {
-                            gsum += __ldcg(part_at(tile1, ks, 0, n));
-                            usum += __ldcg(part_at(tile1, ks, 1, n));
+                    const float* ptile = part_at(tile1, 0, 0, 0) - row_local;
+#pragma unroll 1
+                    for (int j0 = 0; j0 < C::COLS && c0 + j0 < tl.nrows; j0 += 8) {
+                        float gs[8], us[8];
+                        sum_split_partials<8>(ptile, p.s1, C::BN, c0 + j0, row_local, gs, us);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int n = c0 + j0 + j;
+                            if (n < tl.nrows) {
+                                const float hv = swiglu_dev(sg * gs[j], su * us[j], p.alpha, p.beta, p.limit);
+                                out[(size_t)(tl.row0 + n) * out_ld + col] = __float2bfloat16_rn(hv);
+                            }
                         }
-                        const float hv = swiglu_dev(sg * gsum, su * usum, p.alpha, p.beta, p.limit);
-                        out[(size_t)(tl.row0 + n) * out_ld + col] = __float2bfloat16_rn(hv);
                     }
                 }
             } else {
@@ -601,11 +637,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 float acc_g[C::COLS], acc_u[C::COLS];
 #pragma unroll
                 for (int j = 0; j < C::COLS; ++j) acc_g[j] = acc_u[j] = 0.f;
-                // h_scale of a GEMM2 tile may have been written by other CTAs of this launch:
-                // acquire the block's counter in this warp and read the scales through L2.
+                // h_scale of a GEMM2 tile is written by the GEMM1 tiles of its block, in
+                // other CTAs of this launch and possibly still running: this warp waits for
+                // the block's counter itself (acquire) before its first scale load, and
+                // reads the scales through L2.
                 if (!g1 && chained) {
-                    if (lane == 0) (void)ld_acquire_gpu(p.done1 + tl.blk);
-                    __syncwarp();
+                    bool dep_ok = true;
+                    if (lane == 0) dep_ok = wait_counter_geq(p.done1 + tl.blk, p.c1, ab, p.status);
+                    dep_ok = __shfl_sync(0xffffffffu, dep_ok ? 1 : 0, 0) != 0;
+                    __syncwarp();  // orders lane 0's acquire before every lane's scale loads
+                    if (!dep_ok) {
+                        ok = false;
+                        break;
+                    }
                 }
                 // This warp's scale products: tab[j] = sa0 * sb[c0+j], tab[COLS+j] = sa1 * sb[c0+j].
                 // The scales of block kb are loaded kPF blocks ahead (a register ring), so the
@@ -700,16 +744,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         break;
                     }
                     if (r == 0) continue;  // another split of this tile writes h
+                    const float* ptile = part_at(tile1, 0, 0, 0) - row_local;
 #pragma unroll
-                    for (int j = 0; j < C::COLS; ++j) {
-                        float gsum = 0.f, usum = 0.f;
-                        for (int ks = 0; ks < p.s1; ++ks) {
-                            gsum += __ldcg(part_at(tile1, ks, 0, c0 + j));
-                            usum += __ldcg(part_at(tile1, ks, 1, c0 + j));
-                        }
-                        acc_g[j] = gsum;
-                        acc_u[j] = usum;
-                    }
+                    for (int j0 = 0; j0 < C::COLS; j0 += 8)
+                        sum_split_partials<8>(ptile, p.s1, C::BN, c0 + j0, row_local, acc_g + j0, acc_u + j0);
                 }
                 if (g1) {
                     // SwiGLU, then 1x128 E4M3 quantisation of h: the block of row r is the
