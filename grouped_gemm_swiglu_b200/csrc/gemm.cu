@@ -496,13 +496,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         // Split-K of GEMM1: this split's partials are in memory. Returns 1 when this CTA
         // holds the last split of the tile (and merges), 0 when another split merges, -1
         // when the CTA aborted. The counter goes back to zero in the merging CTA.
+        // Ordering: the warps' partial stores reach the counting thread through the CTA
+        // barrier (mbarrier arrive = release, wait = acquire, CTA scope); its GPU-scope fence
+        // before the counter increment publishes them, and the merging CTA's fence after
+        // reading the counter orders its loads of the other splits' partials.
         auto split_arrive = [&](int tile1) -> int {
-            __threadfence();
             __syncwarp();
             if (lane == 0) mbar_arrive(epibar);
             if (!warp_wait(epibar, ephase, ab, p.status)) return -1;
             ephase ^= 1;
             if (ew == 0 && lane == 0) {
+                __threadfence();
                 const int old = atomicAdd(p.split_cnt + tile1, 1);
                 const int last = old == p.s1 - 1;
                 if (last) {
@@ -797,14 +801,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
             }
             // GEMM1 tile done: publish its h rows (and scales) to GEMM2 tiles of this block.
-            // Every epilogue thread makes its stores visible at GPU scope and to the async
-            // proxy, the eight warps meet, and one thread releases the block counter. In
-            // FP8 mode this meeting also keeps `red` from being rewritten while read.
+            // The epilogue warps meet (their stores reach the meeting thread through the
+            // CTA-scope mbarrier: arrive = release, wait = acquire), and one thread fences at
+            // GPU scope and for the async proxy and releases the block counter; a reader
+            // acquires the counter and fences the async proxy before its TMA loads. One
+            // fencing thread instead of every thread: under a saturated memory system each
+            // fence waits microseconds for its stores to be acknowledged. In FP8 mode the
+            // meeting also keeps `red` from being rewritten while read.
             if (g1 && (chained || C::FP8)) {
-                if (chained) {
-                    __threadfence();
-                    fence_proxy_async_global();
-                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(epibar);
                 if (!warp_wait(epibar, ephase, ab, p.status)) {
@@ -812,7 +816,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     break;
                 }
                 ephase ^= 1;
-                if (chained && ew == 0 && lane == 0) red_release_add_gpu(p.done1 + tl.blk, 1);
+                if (chained && ew == 0 && lane == 0) {
+                    __threadfence();
+                    fence_proxy_async_global();
+                    red_release_add_gpu(p.done1 + tl.blk, 1);
+                }
             }
         }
     }
