@@ -55,8 +55,8 @@ def _load():
         lib.oracle_quant_1x128.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                                            ctypes.c_void_p, ctypes.c_void_p]
         lib.oracle_route.restype = ctypes.c_int
-        lib.oracle_route.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                     ctypes.c_int, ctypes.c_int, ctypes.c_double,
+        lib.oracle_route.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         lib.oracle_permute.restype = ctypes.c_int
         lib.oracle_permute.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -95,7 +95,8 @@ class _Layer(ctypes.Structure):
                 ("route_scale", ctypes.c_double),
                 ("logits", ctypes.c_void_p), ("x", ctypes.c_void_p), ("w1", ctypes.c_void_p),
                 ("w1_scale", ctypes.c_void_p), ("w2", ctypes.c_void_p), ("w2_scale", ctypes.c_void_p),
-                ("gate_scale", ctypes.c_void_p), ("up_scale", ctypes.c_void_p)]
+                ("gate_scale", ctypes.c_void_p), ("up_scale", ctypes.c_void_p),
+                ("limits", ctypes.c_void_p), ("router_bias", ctypes.c_void_p)]
 
 
 def num_threads() -> int:
@@ -140,15 +141,17 @@ def quant_1x128(values):
     return q, s
 
 
-def route(logits, n_routed: int, k: int, score: int, route_scale: float = 1.0):
-    """logits [T, n_routed + n_sink] float32 -> (ids int32 [T,k], w f64 [T,k], shared_w f64 [T,n_sink])."""
+def route(logits, n_routed: int, k: int, score: int, route_scale: float = 1.0, bias=None):
+    """logits [T, n_routed + n_sink] float32 (+ optional correction bias float32 [n_routed])
+    -> (ids int32 [T,k], w f64 [T,k], shared_w f64 [T,n_sink])."""
     lg = _c(logits, np.float32)
+    b = _c(bias, np.float32)
     T, cols = lg.shape
     S = cols - n_routed
     ids = np.empty((T, k), dtype=np.int32)
     w = np.empty((T, k), dtype=np.float64)
     sw = np.empty((T, max(S, 0)), dtype=np.float64)
-    rc = _load().oracle_route(_ptr(lg), T, n_routed, S, k, score, route_scale, _ptr(ids), _ptr(w),
+    rc = _load().oracle_route(_ptr(lg), _ptr(b), T, n_routed, S, k, score, route_scale, _ptr(ids), _ptr(w),
                               _ptr(sw) if S > 0 else None)
     if rc != 0:
         raise ValueError("oracle_route: invalid arguments")
@@ -175,17 +178,19 @@ class Layer:
     x: uint16 bf16 bits [T,H]; logits float32 [T,E+n_sink];
     w1: [G,2I,H] uint16 (bf16 bits) or uint8 (E4M3); w2: [G,H,I] likewise;
     w1_scale [G,2I/128,H/128] and w2_scale [G,H/128,I/128] float32 for E4M3;
-    gate_scale / up_scale float32 [G] or None.
+    gate_scale / up_scale float32 [G] or None; limits float32 [G] (a clamp per
+    expert) or None; router_bias float32 [E] or None.
     """
 
     def __init__(self, *, T, H, I, E, k, n_sink, n_shared, wdtype, score, alpha, beta, limit,
                  route_scale, logits, x, w1, w2, w1_scale=None, w2_scale=None,
-                 gate_scale=None, up_scale=None):
+                 gate_scale=None, up_scale=None, limits=None, router_bias=None):
         wt = np.uint16 if wdtype == WDTYPE_BF16 else np.uint8
         self._keep = dict(
             logits=_c(logits, np.float32), x=_c(x, np.uint16), w1=_c(w1, wt), w2=_c(w2, wt),
             w1_scale=_c(w1_scale, np.float32), w2_scale=_c(w2_scale, np.float32),
-            gate_scale=_c(gate_scale, np.float32), up_scale=_c(up_scale, np.float32))
+            gate_scale=_c(gate_scale, np.float32), up_scale=_c(up_scale, np.float32),
+            limits=_c(limits, np.float32), router_bias=_c(router_bias, np.float32))
         k_ = self._keep
         self.dims = dict(T=T, H=H, I=I, E=E, k=k, n_sink=n_sink, n_shared=n_shared,
                          wdtype=wdtype, score=score)
@@ -193,7 +198,7 @@ class Layer:
                         float(alpha), float(beta), float(limit), float(route_scale),
                         _ptr(k_["logits"]), _ptr(k_["x"]), _ptr(k_["w1"]), _ptr(k_["w1_scale"]),
                         _ptr(k_["w2"]), _ptr(k_["w2_scale"]), _ptr(k_["gate_scale"]),
-                        _ptr(k_["up_scale"]))
+                        _ptr(k_["up_scale"]), _ptr(k_["limits"]), _ptr(k_["router_bias"]))
 
     def moe_rows(self, tokens) -> np.ndarray:
         tok = _c(tokens, np.int32)

@@ -138,17 +138,27 @@ static double logsigmoid(double x) {
 
 /* Route one gate row ([P3] items 2 and 3).
  *   row: N routed logits followed by S shared-sink logits (fp32).
- *   Selection: k passes of "largest remaining logit"; equal logits go to the lower
+ *   Selection: k passes of "largest remaining key"; equal keys go to the lower
  *   expert id (the ~index half of the sort key); a column is taken at most once
- *   (the "remaining" mask). Ranking is on the raw logit, which orders the routed
- *   columns exactly as sigmoid(logit) does with no correction bias.
+ *   (the "remaining" mask). Without a correction bias the key is the raw logit, which
+ *   orders the routed columns exactly as sigmoid(logit) does. With a bias [N] the key
+ *   is sigmoid(logit) + bias ([P3] item 3: ranking on sigmoid(logits) + bias, sink
+ *   columns take no bias), here in fp64; the weights below still use the raw logits
+ *   of the selected columns ("the value carried out of the top-k loop becomes the
+ *   winner's RAW logit").
  *   Weights, score 0 (softmax renormalised over the selected k):
  *       w_j = exp(l_j - logsumexp(l_sel)).
  *   Weights, score 1 (sigmoid with logsigmoid-logsumexp renorm, sinks included):
  *       lp = logsigmoid(l), w_j = exp(lp_j - logsumexp(lp over sel and sinks)),
  *       the sink terms give the shared weights.
  *   All weights are multiplied by route_scale. Outputs in selection order. */
-static void route_row(const float* row, int N, int S, int k, int score, double route_scale,
+static double route_key(const float* row, const float* bias, int e) {
+    double l = (double)row[e];
+    if (!bias) return l;
+    return 1.0 / (1.0 + exp(-l)) + (double)bias[e];
+}
+
+static void route_row(const float* row, const float* bias, int N, int S, int k, int score, double route_scale,
                       int32_t* ids, double* w, double* shared_w) {
     unsigned char* taken = (unsigned char*)calloc((size_t)N, 1);
     double* lsel = (double*)malloc(sizeof(double) * (size_t)(k + S));
@@ -157,7 +167,7 @@ static void route_row(const float* row, int N, int S, int k, int score, double r
         for (int e = 0; e < N; ++e) {
             if (taken[e]) continue;
             /* strictly greater keeps the lower id on ties, since e increases */
-            if (best < 0 || (double)row[e] > (double)row[best]) best = e;
+            if (best < 0 || route_key(row, bias, e) > route_key(row, bias, best)) best = e;
         }
         taken[best] = 1;
         ids[j] = best;
@@ -180,12 +190,15 @@ static void route_row(const float* row, int N, int S, int k, int score, double r
     free(lsel);
 }
 
-/* Route T rows of logits [T][N+S]. Returns 0, or -1 on invalid sizes. */
-int oracle_route(const float* logits, int T, int N, int S, int k, int score, double route_scale,
-                 int32_t* ids, double* w, double* shared_w) {
+/* Route T rows of logits [T][N+S] (bias [N] or NULL). Returns 0, or -1 on invalid
+ * sizes or a bias with softmax scoring (the pages define the bias for the sigmoid
+ * ranking only). */
+int oracle_route(const float* logits, const float* bias, int T, int N, int S, int k, int score,
+                 double route_scale, int32_t* ids, double* w, double* shared_w) {
     if (T < 0 || N <= 0 || k <= 0 || k > N || S < 0 || (score == 0 && S != 0)) return -1;
+    if (bias && score != 1) return -1;
     for (int t = 0; t < T; ++t)
-        route_row(logits + (int64_t)t * (N + S), N, S, k, score, route_scale,
+        route_row(logits + (int64_t)t * (N + S), bias, N, S, k, score, route_scale,
                   ids + (int64_t)t * k, w + (int64_t)t * k, shared_w ? shared_w + (int64_t)t * S : NULL);
     return 0;
 }
@@ -248,6 +261,8 @@ typedef struct {
     const float* w2_scale;        /* wdtype 1: [E+n_shared][H/128][I/128] */
     const float* gate_scale;      /* [E+n_shared] or NULL (1.0) */
     const float* up_scale;        /* [E+n_shared] or NULL (1.0) */
+    const float* limits;          /* [E+n_shared] clamp per expert, or NULL (limit) */
+    const float* router_bias;     /* [E] correction bias of the ranking, or NULL */
 } oracle_layer;
 
 /* Dequantised weight element. */
@@ -273,13 +288,16 @@ static double w2_at(const oracle_layer* L, int e, int64_t row, int64_t col) {
 static void expert_gemm1(const oracle_layer* L, int e, const double* xv, double* h) {
     double sg = L->gate_scale ? (double)L->gate_scale[e] : 1.0;
     double su = L->up_scale ? (double)L->up_scale[e] : 1.0;
+    /* the clamp limit may be one fp32 value per expert (sglang PR #39920, "Speed Tests
+     * and Profiling": a per-expert fp32 tensor materialised at weight-load time) */
+    double lim = L->limits ? (double)L->limits[e] : L->limit;
     for (int64_t i = 0; i < L->I; ++i) {
         double gate = 0.0, up = 0.0;
         for (int64_t c = 0; c < L->H; ++c) {
             gate += xv[c] * w1_at(L, e, i, c);
             up += xv[c] * w1_at(L, e, L->I + i, c);
         }
-        h[i] = oracle_swiglu(sg * gate, su * up, L->alpha, L->beta, L->limit);
+        h[i] = oracle_swiglu(sg * gate, su * up, L->alpha, L->beta, lim);
     }
 }
 
@@ -322,6 +340,7 @@ static void expert_mlp(const oracle_layer* L, int e, const double* xv, double* y
 int oracle_moe_rows(const oracle_layer* L, const int32_t* tokens, int n_tok, double* out) {
     if (L->n_sink > 0 && L->n_shared > 0 && L->n_sink != L->n_shared) return -1;
     if (L->score == 0 && L->n_sink != 0) return -1;
+    if (L->score == 0 && L->router_bias) return -1;
     int N = L->E, S = L->n_sink;
     int bad = 0;
 #pragma omp parallel for schedule(dynamic, 1)
@@ -334,7 +353,8 @@ int oracle_moe_rows(const oracle_layer* L, const int32_t* tokens, int n_tok, dou
         double* xv = (double*)malloc(sizeof(double) * (size_t)L->H);
         double* y = (double*)malloc(sizeof(double) * (size_t)L->H);
         double* o = out + (int64_t)it * L->H;
-        route_row(L->logits + (int64_t)t * (N + S), N, S, L->k, L->score, L->route_scale, ids, w, sw);
+        route_row(L->logits + (int64_t)t * (N + S), L->router_bias, N, S, L->k, L->score, L->route_scale, ids, w,
+                  sw);
         for (int64_t c = 0; c < L->H; ++c) xv[c] = oracle_bf16_to_double(L->x[(int64_t)t * L->H + c]);
         if (L->wdtype == 1) fp8_roundtrip_row(xv, L->H, xv);
         for (int64_t c = 0; c < L->H; ++c) o[c] = 0.0;

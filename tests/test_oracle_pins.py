@@ -212,6 +212,56 @@ def test_route_rejects_sinks_with_softmax():
         oracle.route(np.zeros((2, 10), np.float32), 8, 2, oracle.SCORE_SOFTMAX)
 
 
+def test_route_zero_bias_keeps_the_raw_logit_order():
+    # sigmoid is increasing, so a zero correction bias ranks exactly like the raw logit
+    rng = np.random.default_rng(21)
+    N, S, k = 64, 2, 6
+    logits = rng.normal(0, 3, (40, N + S)).astype(np.float32)
+    ids0, w0, sw0 = oracle.route(logits, N, k, oracle.SCORE_SIGMOID)
+    ids1, w1, sw1 = oracle.route(logits, N, k, oracle.SCORE_SIGMOID, bias=np.zeros(N, np.float32))
+    assert np.array_equal(ids0, ids1)
+    np.testing.assert_array_equal(w0, w1)
+    np.testing.assert_array_equal(sw0, sw1)
+
+
+def test_route_dominant_bias_forces_the_selection_and_not_the_weights():
+    # sigmoid lies in (0, 1): bias gaps of 10 decide the ranking whatever the logits, and
+    # the weights still come from the raw logits of the selected columns.
+    rng = np.random.default_rng(22)
+    N, S, k = 32, 2, 5
+    logits = rng.normal(0, 4, (24, N + S)).astype(np.float32)
+    bias = (10.0 * rng.permutation(N)).astype(np.float32)
+    ids, w, sw = oracle.route(logits, N, k, oracle.SCORE_SIGMOID, 1.0, bias=bias)
+    want = np.argsort(-bias, kind="stable")[:k]
+    sig = scipy.special.expit(logits.astype(np.float64))
+    for t in range(len(logits)):
+        assert list(ids[t]) == list(want)
+        den = sig[t, want].sum() + sig[t, N:].sum()
+        np.testing.assert_allclose(w[t], sig[t, want] / den, rtol=1e-12)
+        np.testing.assert_allclose(sw[t], sig[t, N:] / den, rtol=1e-12)
+
+
+@pytest.mark.parametrize("scale", [0.02, 0.3])
+def test_route_bias_selection_is_the_top_k_of_sigmoid_plus_bias(scale):
+    rng = np.random.default_rng(23)
+    N, k = 48, 8
+    logits = rng.normal(0, 2, (64, N)).astype(np.float32)
+    bias = rng.normal(0, scale, N).astype(np.float32)
+    ids, _, _ = oracle.route(logits, N, k, oracle.SCORE_SIGMOID, bias=bias)
+    key = scipy.special.expit(logits.astype(np.float64)) + bias.astype(np.float64)
+    for t in range(len(logits)):
+        sel = key[t, ids[t]]
+        rest = np.delete(key[t], ids[t])
+        assert np.all(np.diff(sel) <= 0)          # descending key order
+        assert sel.min() >= rest.max()            # nothing outside beats what is inside
+        assert len(set(ids[t])) == k
+
+
+def test_route_rejects_bias_with_softmax():
+    with pytest.raises(ValueError):
+        oracle.route(np.zeros((2, 8), np.float32), 8, 2, oracle.SCORE_SOFTMAX, bias=np.zeros(8, np.float32))
+
+
 # --------------------------------------------------------------------------- permute
 
 @pytest.mark.parametrize("T,E,k,S", [(37, 8, 2, 0), (100, 16, 4, 1), (5, 300, 8, 2), (1, 4, 4, 0)])
@@ -411,3 +461,48 @@ def test_gemm_pieces_agree_with_dense_reference():
     for t in range(T):
         ref = sum(float(row_w[inv[t, j]]) * (torch.from_numpy(hv[inv[t, j]]) @ torch.from_numpy(_bf16_val(d["w2"][ids[t, j]])).T).numpy() for j in range(k))
         np.testing.assert_allclose(out[t], ref, rtol=1e-11, atol=1e-14)
+
+
+def _dense_mlp_clamped(x, w1, w2, I, L):
+    # alpha = 1, beta = 0: h = silu(min(g, L)) * clamp(u, -L, L), all torch library calls
+    xt = torch.from_numpy(x)
+    g = torch.clamp(xt @ torch.from_numpy(w1[:I]).T, max=L)
+    u = torch.clamp(xt @ torch.from_numpy(w1[I:]).T, min=-L, max=L)
+    return ((torch.nn.functional.silu(g) * u) @ torch.from_numpy(w2).T).numpy()
+
+
+def test_layer_per_expert_limits_clamp_each_expert_with_its_own_value():
+    # k = 1 softmax: every token goes to one expert with weight 1, so the layer output
+    # is that expert's clamped MLP with that expert's limit
+    rng = np.random.default_rng(31)
+    E, I, T = 3, 32, 9
+    limits = np.array([0.25, 0.8, np.inf], np.float32)
+    d = _mk_layer(rng, T=T, H=128, I=I, E=E, k=1, w_mult=2.0)
+    out = oracle.Layer(**d, limits=limits).moe_rows(np.arange(T))
+    ids, _, _ = oracle.route(d["logits"], E, 1, oracle.SCORE_SOFTMAX)
+    x = _bf16_val(d["x"])
+    assert len(set(ids[:, 0])) == E  # every expert (and so every limit) is exercised
+    for t in range(T):
+        e = int(ids[t, 0])
+        ref = _dense_mlp_clamped(x[t:t + 1], _bf16_val(d["w1"][e]), _bf16_val(d["w2"][e]), I, float(limits[e]))
+        np.testing.assert_allclose(out[t:t + 1], ref, rtol=1e-10, atol=1e-12)
+    # a uniform array is the scalar limit (0.75: the same value in fp32 and fp64)
+    uni = oracle.Layer(**dict(d, limit=0.75), limits=np.full(E, 0.75, np.float32)).moe_rows(np.arange(T))
+    sca = oracle.Layer(**dict(d, limit=0.75)).moe_rows(np.arange(T))
+    np.testing.assert_array_equal(uni, sca)
+
+
+def test_layer_router_bias_changes_only_the_selection():
+    # a dominant bias routes every token to the same experts; the output then equals the
+    # sigma-ratio-weighted sum of those experts' dense MLPs (raw-logit weights)
+    rng = np.random.default_rng(32)
+    E, I, T, k = 6, 32, 5, 2
+    d = _mk_layer(rng, T=T, H=128, I=I, E=E, k=k, score=oracle.SCORE_SIGMOID)
+    bias = np.array([0, 0, 50, 0, 40, 0], np.float32)
+    out = oracle.Layer(**d, router_bias=bias).moe_rows(np.arange(T))
+    x = _bf16_val(d["x"])
+    sig = scipy.special.expit(d["logits"].astype(np.float64))
+    wts = sig[:, [2, 4]] / sig[:, [2, 4]].sum(1, keepdims=True)
+    ref = sum(wts[:, j:j + 1] * _dense_mlp(x, _bf16_val(d["w1"][e]), _bf16_val(d["w2"][e]), I)
+              for j, e in enumerate([2, 4]))
+    np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
