@@ -255,10 +255,10 @@ def run_ours(args):
     ws_e = moe.alloc_workspace(d, moe.MOE_WS_EXPERTS, dev)
     ws_c = moe.alloc_workspace(d, moe.MOE_WS_COMBINE, dev)
     stages = {
-        "route": lambda: moe.moe_route_topk(inp["logits"], d, ids, tw, sw),
+        "route": lambda: moe.moe_route_topk(inp["logits"], d, None, ids, tw, sw),
         "permute": lambda: moe.moe_permute(ids, inp["x"], d, offsets, perm, inv, xp, xs, ws_p),
         "experts": lambda: moe.moe_experts(xp, xs, offsets, inp["w1"], inp["w1_scale"], inp["gate_scale"],
-                                           inp["up_scale"], inp["w2"], inp["w2_scale"], d, h, hs, y, ws_e),
+                                           inp["up_scale"], None, inp["w2"], inp["w2_scale"], d, h, hs, y, ws_e),
         "combine": lambda: moe.moe_combine(y, offsets, inv, tw, sw, d, out, ws_c),
     }
     launches_per_step = 5  # router 1, permutation 2, grouped GEMMs 1, combine 1

@@ -18,7 +18,8 @@ from ._lib import (MOE_OK, MOE_SCORE_SIGMOID, MOE_SCORE_SOFTMAX, MOE_WDTYPE_BF16
 
 __all__ = ["MoeDims", "MoeError", "MoELayer", "moe_abi_version", "moe_workspace_size", "moe_read_status",
            "moe_clear_status", "moe_route_topk", "moe_permute", "moe_permute_noalloc", "moe_gemm1_swiglu",
-           "moe_gemm2_combine", "moe_experts", "moe_combine", "moe_forward", "alloc_workspace", "status_string", "lib", "header_functions", "MOE_OK",
+           "moe_gemm2_combine", "moe_experts", "moe_combine", "moe_forward", "alloc_workspace", "status_string", "lib",
+           "header_functions", "MOE_OK",
            "MOE_SCORE_SIGMOID", "MOE_SCORE_SOFTMAX", "MOE_WDTYPE_BF16", "MOE_WDTYPE_FP8_E4M3_BLOCK128",
            "MOE_WS_FORWARD", "MOE_WS_GEMM1", "MOE_WS_GEMM2_COMBINE", "MOE_WS_PERMUTE", "MOE_WS_EXPERTS",
            "MOE_WS_COMBINE"]
@@ -28,21 +29,24 @@ class MoELayer:
     """Weights resident on the GPU plus a reusable workspace; `forward` runs moe_forward.
 
     w1 [G,2I,H] and w2 [G,H,I] are bf16, or uint8 E4M3 codes with w1_scale/w2_scale
-    fp32 block scales; gate_scale/up_scale are optional fp32 [G]. The workspace is
-    sized for `max_tokens` tokens and reused by every call with T <= max_tokens.
+    fp32 block scales; gate_scale/up_scale are optional fp32 [G]; limits is an optional
+    fp32 [G] clamp per expert (else dims.limit); router_bias an optional fp32 [E]
+    correction bias of the ranking. The workspace is sized for `max_tokens` tokens and
+    reused by every call with T <= max_tokens.
     """
 
     def __init__(self, dims: MoeDims, w1, w2, w1_scale=None, w2_scale=None, gate_scale=None, up_scale=None,
-                 max_tokens: int | None = None):
+                 max_tokens: int | None = None, limits=None, router_bias=None):
         self.dims = dims
         self.w1, self.w2, self.w1_scale, self.w2_scale = w1, w2, w1_scale, w2_scale
         self.gate_scale, self.up_scale = gate_scale, up_scale
+        self.limits, self.router_bias = limits, router_bias
         self.max_tokens = dims.T if max_tokens is None else max_tokens
         sized = MoeDims.from_buffer_copy(dims)
         sized.T = self.max_tokens
         self.ws = alloc_workspace(sized, MOE_WS_FORWARD, device=w1.device)
 
-    def forward(self, logits, x, out=None, topk_ids=None, topk_w=None, shared_w=None, stream=None):
+    def forward(self, logits, x, out=None, topk_ids=None, topk_w=None, shared_w=None, packed=None, stream=None):
         T = x.shape[0]
         if T > self.max_tokens:
             raise ValueError(f"T={T} exceeds the workspace size ({self.max_tokens} tokens)")
@@ -50,8 +54,8 @@ class MoELayer:
         d.T = T
         if out is None:
             out = torch.empty((T, d.H), dtype=torch.bfloat16, device=x.device)
-        moe_forward(logits, x, self.w1, self.w1_scale, self.gate_scale, self.up_scale, self.w2, self.w2_scale, d,
-                    out, topk_ids, topk_w, shared_w, self.ws, stream)
+        moe_forward(logits, self.router_bias, x, self.w1, self.w1_scale, self.gate_scale, self.up_scale, self.limits,
+                    self.w2, self.w2_scale, d, out, topk_ids, topk_w, shared_w, packed, self.ws, stream)
         return out
 
     def status(self, stream=None) -> int:

@@ -72,16 +72,16 @@ def lib() -> ctypes.CDLL:
             "moe_workspace_size": ([P, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
             "moe_read_status": ([_VP, ctypes.POINTER(ctypes.c_int32), _VP], ctypes.c_int),
             "moe_clear_status": ([_VP, _VP], ctypes.c_int),
-            "moe_route_topk": ([_VP, P, _VP, _VP, _VP, _VP], ctypes.c_int),
+            "moe_route_topk": ([_VP, P, _VP, _VP, _VP, _VP, _VP, _VP], ctypes.c_int),
             "moe_permute": ([_VP, _VP, P, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
-            "moe_gemm1_swiglu": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, P, _VP, _VP, _VP, ctypes.c_size_t, _VP],
+            "moe_gemm1_swiglu": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, P, _VP, _VP, _VP, ctypes.c_size_t, _VP],
                                  ctypes.c_int),
             "moe_gemm2_combine": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, P, _VP, _VP, ctypes.c_size_t, _VP],
                                   ctypes.c_int),
-            "moe_forward": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, P, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t,
-                             _VP], ctypes.c_int),
-            "moe_experts": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, P, _VP, _VP, _VP, _VP, ctypes.c_size_t,
-                             _VP], ctypes.c_int),
+            "moe_forward": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, P, _VP, _VP, _VP, _VP, _VP, _VP,
+                             ctypes.c_size_t, _VP], ctypes.c_int),
+            "moe_experts": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, P, _VP, _VP, _VP, _VP,
+                             ctypes.c_size_t, _VP], ctypes.c_int),
             "moe_combine": ([_VP, _VP, _VP, _VP, _VP, P, _VP, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
@@ -147,9 +147,9 @@ def moe_clear_status(ws, stream=None) -> None:
     _check("moe_clear_status", lib().moe_clear_status(_p(ws), _s(stream)))
 
 
-def moe_route_topk(logits, dims: MoeDims, topk_ids, topk_w, shared_w=None, stream=None) -> None:
-    _check("moe_route_topk", lib().moe_route_topk(_p(logits), ctypes.byref(dims), _p(topk_ids), _p(topk_w),
-                                                  _p(shared_w), _s(stream)))
+def moe_route_topk(logits, dims: MoeDims, bias, topk_ids, topk_w, shared_w=None, packed=None, stream=None) -> None:
+    _check("moe_route_topk", lib().moe_route_topk(_p(logits), ctypes.byref(dims), _p(bias), _p(topk_ids),
+                                                  _p(topk_w), _p(shared_w), _p(packed), _s(stream)))
 
 
 def moe_permute(topk_ids, x, dims: MoeDims, offsets, perm, inv_perm, x_perm, x_scale, ws, stream=None) -> None:
@@ -158,11 +158,11 @@ def moe_permute(topk_ids, x, dims: MoeDims, offsets, perm, inv_perm, x_perm, x_s
                                             _s(stream)))
 
 
-def moe_gemm1_swiglu(x_perm, x_scale, offsets, w1, w1_scale, gate_scale, up_scale, dims: MoeDims, h, h_scale, ws,
-                     stream=None) -> None:
+def moe_gemm1_swiglu(x_perm, x_scale, offsets, w1, w1_scale, gate_scale, up_scale, limits, dims: MoeDims, h,
+                     h_scale, ws, stream=None) -> None:
     _check("moe_gemm1_swiglu", lib().moe_gemm1_swiglu(_p(x_perm), _p(x_scale), _p(offsets), _p(w1), _p(w1_scale),
-                                                      _p(gate_scale), _p(up_scale), ctypes.byref(dims), _p(h),
-                                                      _p(h_scale), _p(ws), _nbytes(ws), _s(stream)))
+                                                      _p(gate_scale), _p(up_scale), _p(limits), ctypes.byref(dims),
+                                                      _p(h), _p(h_scale), _p(ws), _nbytes(ws), _s(stream)))
 
 
 def moe_gemm2_combine(h, h_scale, offsets, inv_perm, topk_w, shared_w, w2, w2_scale, dims: MoeDims, out, ws,
@@ -172,18 +172,20 @@ def moe_gemm2_combine(h, h_scale, offsets, inv_perm, topk_w, shared_w, w2, w2_sc
                                                         _p(out), _p(ws), _nbytes(ws), _s(stream)))
 
 
-def moe_forward(logits, x, w1, w1_scale, gate_scale, up_scale, w2, w2_scale, dims: MoeDims, out, topk_ids=None,
-                topk_w=None, shared_w=None, ws=None, stream=None) -> None:
-    _check("moe_forward", lib().moe_forward(_p(logits), _p(x), _p(w1), _p(w1_scale), _p(gate_scale), _p(up_scale),
-                                            _p(w2), _p(w2_scale), ctypes.byref(dims), _p(out), _p(topk_ids),
-                                            _p(topk_w), _p(shared_w), _p(ws), _nbytes(ws), _s(stream)))
+def moe_forward(logits, bias, x, w1, w1_scale, gate_scale, up_scale, limits, w2, w2_scale, dims: MoeDims, out,
+                topk_ids=None, topk_w=None, shared_w=None, packed=None, ws=None, stream=None) -> None:
+    _check("moe_forward", lib().moe_forward(_p(logits), _p(bias), _p(x), _p(w1), _p(w1_scale), _p(gate_scale),
+                                            _p(up_scale), _p(limits), _p(w2), _p(w2_scale), ctypes.byref(dims),
+                                            _p(out), _p(topk_ids), _p(topk_w), _p(shared_w), _p(packed), _p(ws),
+                                            _nbytes(ws), _s(stream)))
 
 
-def moe_experts(x_perm, x_scale, offsets, w1, w1_scale, gate_scale, up_scale, w2, w2_scale, dims: MoeDims, h,
-                h_scale, y, ws, stream=None) -> None:
+def moe_experts(x_perm, x_scale, offsets, w1, w1_scale, gate_scale, up_scale, limits, w2, w2_scale, dims: MoeDims,
+                h, h_scale, y, ws, stream=None) -> None:
     _check("moe_experts", lib().moe_experts(_p(x_perm), _p(x_scale), _p(offsets), _p(w1), _p(w1_scale),
-                                            _p(gate_scale), _p(up_scale), _p(w2), _p(w2_scale), ctypes.byref(dims),
-                                            _p(h), _p(h_scale), _p(y), _p(ws), _nbytes(ws), _s(stream)))
+                                            _p(gate_scale), _p(up_scale), _p(limits), _p(w2), _p(w2_scale),
+                                            ctypes.byref(dims), _p(h), _p(h_scale), _p(y), _p(ws), _nbytes(ws),
+                                            _s(stream)))
 
 
 def moe_combine(y, offsets, inv_perm, topk_w, shared_w, dims: MoeDims, out, ws, stream=None) -> None:

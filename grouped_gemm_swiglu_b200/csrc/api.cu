@@ -108,8 +108,15 @@ P* at(void* ws, size_t off) {
 }
 
 // The individual steps, after every check has passed.
-int do_route(const float* logits, const moe_dims* d, int32_t* ids, float* w, float* sw, cudaStream_t s) {
-    return cuda_status(launch_router(logits, d->T, d->E, d->n_sink, d->k, d->score, d->route_scale, ids, w, sw, s));
+int do_route(const float* logits, const float* bias, const moe_dims* d, int32_t* ids, float* w, float* sw,
+             uint32_t* packed, cudaStream_t s) {
+    return cuda_status(launch_router(logits, bias, d->T, d->E, d->n_sink, d->k, d->score, d->route_scale, ids, w, sw,
+                                     packed, s));
+}
+
+// A correction bias is defined for the sigmoid ranking only.
+int check_bias(const moe_dims* d, const float* bias) {
+    return (bias && d->score != MOE_SCORE_SIGMOID) ? MOE_ERR_UNSUPPORTED : MOE_OK;
 }
 
 int do_permute(const int32_t* ids, const void* x, const moe_dims* d, int32_t* offsets, int32_t* perm, int32_t* inv,
@@ -138,7 +145,8 @@ MoeGemmArgs gemm_args(const moe_dims* d, const int32_t* offsets, int* status) {
 }
 
 int do_gemm1(const void* xperm, const float* xscale, const int32_t* offsets, const void* w1, const float* w1s,
-             const float* gs, const float* us, const moe_dims* d, void* h, float* hs, void* ws, cudaStream_t s) {
+             const float* gs, const float* us, const float* limits, const moe_dims* d, void* h, float* hs, void* ws,
+             cudaStream_t s) {
     const Layout L = layout(d, MOE_WS_GEMM1);
     MoeGemmArgs a = gemm_args(d, offsets, at<int>(ws, 0));
     a.split_cnt = L.part ? at<int>(ws, L.splitcnt) : nullptr;
@@ -150,6 +158,7 @@ int do_gemm1(const void* xperm, const float* xscale, const int32_t* offsets, con
     a.w1_scale = w1s;
     a.gate_scale = gs;
     a.up_scale = us;
+    a.limits = limits;
     a.h = h;
     a.h_scale = hs;
     return cuda_status(launch_moe_gemm(a, s));
@@ -220,14 +229,15 @@ int moe_clear_status(void* ws, void* stream) {
     return cuda_status(cudaMemsetAsync(ws, 0, kWsHeader, static_cast<cudaStream_t>(stream)));
 }
 
-int moe_route_topk(const float* logits, const moe_dims* d, int32_t* topk_ids, float* topk_w, float* shared_w,
-                   void* stream) {
+int moe_route_topk(const float* logits, const moe_dims* d, const float* bias, int32_t* topk_ids, float* topk_w,
+                   float* shared_w, uint32_t* packed, void* stream) {
     int rc = check_dims(d);
     if (rc != MOE_OK) return rc;
     if (d->T > 0 && (!logits || !topk_ids || !topk_w)) return MOE_ERR_INVALID_ARG;
     if (d->T > 0 && (d->n_sink > 0) != (shared_w != nullptr)) return MOE_ERR_INVALID_ARG;
+    if ((rc = check_bias(d, bias)) != MOE_OK) return rc;
     if ((rc = check_arch()) != MOE_OK) return rc;
-    return do_route(logits, d, topk_ids, topk_w, shared_w, static_cast<cudaStream_t>(stream));
+    return do_route(logits, bias, d, topk_ids, topk_w, shared_w, packed, static_cast<cudaStream_t>(stream));
 }
 
 int moe_permute(const int32_t* topk_ids, const void* x, const moe_dims* d, int32_t* offsets, int32_t* perm,
@@ -248,8 +258,8 @@ int moe_permute(const int32_t* topk_ids, const void* x, const moe_dims* d, int32
 }
 
 int moe_gemm1_swiglu(const void* x_perm, const float* x_scale, const int32_t* offsets, const void* w1,
-                     const float* w1_scale, const float* gate_scale, const float* up_scale, const moe_dims* d,
-                     void* h, float* h_scale, void* ws, size_t ws_bytes, void* stream) {
+                     const float* w1_scale, const float* gate_scale, const float* up_scale, const float* limits,
+                     const moe_dims* d, void* h, float* h_scale, void* ws, size_t ws_bytes, void* stream) {
     int rc = check_dims(d);
     if (rc != MOE_OK) return rc;
     if (d->T > 0) {
@@ -260,7 +270,7 @@ int moe_gemm1_swiglu(const void* x_perm, const float* x_scale, const int32_t* of
     if ((rc = check_ws(ws, ws_bytes, d, MOE_WS_GEMM1)) != MOE_OK) return rc;
     if ((rc = check_arch()) != MOE_OK) return rc;
     if (d->T == 0) return MOE_OK;
-    return do_gemm1(x_perm, x_scale, offsets, w1, w1_scale, gate_scale, up_scale, d, h, h_scale, ws,
+    return do_gemm1(x_perm, x_scale, offsets, w1, w1_scale, gate_scale, up_scale, limits, d, h, h_scale, ws,
                     static_cast<cudaStream_t>(stream));
 }
 
@@ -284,8 +294,8 @@ int moe_gemm2_combine(const void* h, const float* h_scale, const int32_t* offset
 }
 
 int moe_experts(const void* x_perm, const float* x_scale, const int32_t* offsets, const void* w1,
-                const float* w1_scale, const float* gate_scale, const float* up_scale, const void* w2,
-                const float* w2_scale, const moe_dims* d, void* h, float* h_scale, void* y, void* ws,
+                const float* w1_scale, const float* gate_scale, const float* up_scale, const float* limits,
+                const void* w2, const float* w2_scale, const moe_dims* d, void* h, float* h_scale, void* y, void* ws,
                 size_t ws_bytes, void* stream) {
     int rc = check_dims(d);
     if (rc != MOE_OK) return rc;
@@ -307,6 +317,7 @@ int moe_experts(const void* x_perm, const float* x_scale, const int32_t* offsets
     a.w1_scale = w1_scale;
     a.gate_scale = gate_scale;
     a.up_scale = up_scale;
+    a.limits = limits;
     a.h = h;
     a.h_scale = h_scale;
     a.w2 = w2;
@@ -334,11 +345,13 @@ int moe_combine(const void* y, const int32_t* offsets, const int32_t* inv_perm, 
                       static_cast<cudaStream_t>(stream));
 }
 
-int moe_forward(const float* logits, const void* x, const void* w1, const float* w1_scale, const float* gate_scale,
-                const float* up_scale, const void* w2, const float* w2_scale, const moe_dims* d, void* out,
-                int32_t* topk_ids, float* topk_w, float* shared_w, void* ws, size_t ws_bytes, void* stream) {
+int moe_forward(const float* logits, const float* bias, const void* x, const void* w1, const float* w1_scale,
+                const float* gate_scale, const float* up_scale, const float* limits, const void* w2,
+                const float* w2_scale, const moe_dims* d, void* out, int32_t* topk_ids, float* topk_w,
+                float* shared_w, uint32_t* packed, void* ws, size_t ws_bytes, void* stream) {
     int rc = check_dims(d);
     if (rc != MOE_OK) return rc;
+    if ((rc = check_bias(d, bias)) != MOE_OK) return rc;
     if (d->T > 0) {
         if (!logits || !x || !w1 || !w2 || !out) return MOE_ERR_INVALID_ARG;
         if (is_fp8(d) && (!w1_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
@@ -357,7 +370,7 @@ int moe_forward(const float* logits, const void* x, const void* w1, const float*
     if (d->T == 0) return cuda_status(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (groups(d) + 1), s));
     float* xscale = is_fp8(d) ? at<float>(ws, L.xscale) : nullptr;
     float* hscale = is_fp8(d) ? at<float>(ws, L.hscale) : nullptr;
-    if ((rc = do_route(logits, d, ids, w, sw, s)) != MOE_OK) return rc;
+    if ((rc = do_route(logits, bias, d, ids, w, sw, packed, s)) != MOE_OK) return rc;
     // The counting kernel also clears the GEMM's per-block completion flags.
     int* flags = at<int>(ws, L.flags);
     const size_t clear_words =
@@ -374,6 +387,7 @@ int moe_forward(const float* logits, const void* x, const void* w1, const float*
     a.w1_scale = w1_scale;
     a.gate_scale = gate_scale;
     a.up_scale = up_scale;
+    a.limits = limits;
     a.h = at<void>(ws, L.h);
     a.h_scale = hscale;
     a.w2 = w2;

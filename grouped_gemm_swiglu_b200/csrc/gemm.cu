@@ -120,6 +120,7 @@ struct DevArgs {
     const float* gate_scale;
     const float* up_scale;
     float alpha, beta, limit;
+    const float* limits;    // [G] per-group clamp, or NULL for `limit`
     void* h;                // GEMM1 out / GEMM2 in: [A][I]
     float* h_scale;         // FP8: [I/128][A]
     void* y;                // GEMM2 out: [A][H] bf16
@@ -540,6 +541,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const int out_ld = g1 ? p.I : p.H;
             const float sg = (g1 && p.gate_scale) ? __ldg(p.gate_scale + tl.g) : 1.f;
             const float su = (g1 && p.up_scale) ? __ldg(p.up_scale + tl.g) : 1.f;
+            const float lim = (g1 && p.limits) ? __ldg(p.limits + tl.g) : p.limit;  // this expert's clamp
             if constexpr (!C::FP8) {
                 const uint32_t buf = it % C::NBUF, bph = (it / C::NBUF) & 1;
                 if (!warp_wait(&tfull[buf], bph, ab, p.status)) {
@@ -571,7 +573,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         for (int j = 0; j < C::CW; ++j) {
                             const int n = cc + j;
                             if (n < tl.nrows) {
-                                const float h = swiglu_dev(sg * gv[j], su * uv[j], p.alpha, p.beta, p.limit);
+                                const float h = swiglu_dev(sg * gv[j], su * uv[j], p.alpha, p.beta, lim);
                                 out[(size_t)(tl.row0 + n) * out_ld + col] = __float2bfloat16_rn(h);
                             }
                         }
@@ -623,7 +625,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         for (int j = 0; j < 8; ++j) {
                             const int n = c0 + j0 + j;
                             if (n < tl.nrows) {
-                                const float hv = swiglu_dev(sg * gs[j], su * us[j], p.alpha, p.beta, p.limit);
+                                const float hv = swiglu_dev(sg * gs[j], su * us[j], p.alpha, p.beta, lim);
                                 out[(size_t)(tl.row0 + n) * out_ld + col] = __float2bfloat16_rn(hv);
                             }
                         }
@@ -758,7 +760,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     // 128 intermediate indices of this chunk = the 4 lane quarters.
 #pragma unroll
                     for (int j = 0; j < C::COLS; ++j) {
-                        acc_g[j] = swiglu_dev(sg * acc_g[j], su * acc_u[j], p.alpha, p.beta, p.limit);
+                        acc_g[j] = swiglu_dev(sg * acc_g[j], su * acc_u[j], p.alpha, p.beta, lim);
                         float m = fabsf(acc_g[j]);
 #pragma unroll
                         for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
@@ -927,6 +929,7 @@ static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
     p.alpha = a.alpha;
     p.beta = a.beta;
     p.limit = a.limit;
+    p.limits = a.limits;
     p.h = a.h;
     p.h_scale = a.h_scale;
     p.y = a.y;

@@ -10,8 +10,9 @@
 
 namespace moe {
 
-cudaError_t launch_router(const float* logits, int T, int N, int S, int k, int score, float route_scale,
-                          int32_t* ids, float* w, float* sw, cudaStream_t stream);
+// bias [N] or NULL (rank on the raw logit); packed [T][k] or NULL.
+cudaError_t launch_router(const float* logits, const float* bias, int T, int N, int S, int k, int score,
+                          float route_scale, int32_t* ids, float* w, float* sw, uint32_t* packed, cudaStream_t stream);
 
 // Scratch of the permutation: per 256-token chunk counts/bases [nchunk][E] and the
 // in-chunk rank of every (token, slot) [T][k]. `counter` is one word that must be zero
@@ -46,6 +47,7 @@ struct MoeGemmArgs {
     const float* gate_scale; // [G] or NULL
     const float* up_scale;   // [G] or NULL
     float alpha, beta, limit;
+    const float* limits;     // [G] per-group clamp (replaces limit) or NULL
     void* h;                 // [A][I]
     float* h_scale;          // FP8: [I/128][A]
     const void* w2;          // [G][H][I]

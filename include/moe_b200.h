@@ -14,7 +14,11 @@
  *   [P3] sglang PR #36385 "Enable and fuse the Inkling MoE gate epilogue on Intel XPU",
  *        items 2-3: masked-max top-k, ties to the lower expert id, weights
  *        exp(lp - logsumexp(lp)) with lp = logsigmoid(x), shared-sink columns that
- *        join the normaliser but never the top-k, a scalar routing scale.
+ *        join the normaliser but never the top-k, a scalar routing scale, ranking on
+ *        sigmoid(logit) + bias with the raw logit carried out, the packed
+ *        (id << 16 | bf16 weight) output.
+ *   [P2'] the same sglang PR #39920, "Speed Tests and Profiling": the clamp limit as one
+ *        fp32 value per expert.
  *   [P4] DeepGEMM PR #445 "fix(sm90): support parameterized SwiGLU in FP8 MegaMoE",
  *        "Summary"/"Compatibility": alpha, up_bias (beta) and clamp as explicit
  *        parameters; alpha = 1, beta = 0, no clamp is the standard SwiGLU.
@@ -52,7 +56,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 typedef enum moe_status {
     MOE_OK = 0,
@@ -131,17 +135,24 @@ int moe_clear_status(void* ws, void* stream);
 
 /* Router / gate epilogue ([P3] items 2 and 3).
  *   logits   [T][E + n_sink] fp32, read only. Finite values required.
- *   topk_ids [T][k] int32 out: per token, the k routed columns with the largest logit,
- *            in descending order; equal logits go to the lower id. Ranking is on the raw
- *            logit (no correction bias), which orders like sigmoid(logit).
+ *   bias     [E] fp32 correction bias of the routed columns, or NULL. With NULL the ranking
+ *            key is the raw logit (which orders like sigmoid(logit)); with a bias it is
+ *            sigmoid(logit) + bias[e], both evaluated in fp32 (sigmoid saturates there:
+ *            ties are then broken by the bias, then by the lower id). Sink columns take no
+ *            bias. Sigmoid scoring only (else MOE_ERR_UNSUPPORTED).
+ *   topk_ids [T][k] int32 out: per token, the k routed columns with the largest key,
+ *            in descending order; equal keys go to the lower id.
  *   topk_w   [T][k] fp32 out: routing weights in the same order, times route_scale.
  *            softmax: exp(l_j - logsumexp(l_sel)); sigmoid: exp(lp_j - logsumexp(lp over
- *            the selected and the sink columns)), lp = logsigmoid(l) -- finite even when
- *            every logit is below -104.
+ *            the selected and the sink columns)), lp = logsigmoid(l) of the RAW logit
+ *            (never the biased key) -- finite even when every logit is below -104.
  *   shared_w [T][n_sink] fp32 out (NULL iff n_sink == 0): the sink columns' weights.
- * Errors: INVALID_ARG (sizes, NULL pointers, n_sink > 0 with softmax), ARCH, CUDA. */
-int moe_route_topk(const float* logits, const moe_dims* dims, int32_t* topk_ids,
-                   float* topk_w, float* shared_w, void* stream);
+ *   packed   [T][k] uint32 out, or NULL: (topk_ids << 16) | bf16 bits of topk_w
+ *            (round to nearest even). Ids fit 16 bits (E <= 1024).
+ * Errors: INVALID_ARG (sizes, NULL pointers, n_sink > 0 with softmax), UNSUPPORTED (bias
+ * with softmax), ARCH, CUDA. */
+int moe_route_topk(const float* logits, const moe_dims* dims, const float* bias, int32_t* topk_ids,
+                   float* topk_w, float* shared_w, uint32_t* packed, void* stream);
 
 /* Permute by expert ([P5]: per-expert sorted-token dispatch; [P1]: fused act-quant).
  *   topk_ids [T][k] int32 in: expert ids in [0, E), distinct within a token.
@@ -199,13 +210,15 @@ int moe_permute_noalloc(const int32_t* topk_ids, const void* x, const moe_dims* 
  *   w1        [G][2I][H]: rows [0, I) gate, [I, 2I) up; bf16 or E4M3.
  *   w1_scale  [G][2I/128][H/128] fp32 (FP8 only, else NULL).
  *   gate_scale, up_scale  [G] fp32 per-group scales, or NULL for 1.0.
+ *   limits    [G] fp32 clamp L per group ([P2'] one value per expert), or NULL for
+ *             dims->limit. Each value > 0; +INFINITY disables that group's clamp.
  *   h         [A][I] out: bf16, or E4M3 codes quantised per 1x128 block like x_perm.
  *   h_scale   [I/128][A] fp32 out (FP8 only, else NULL).
  * Errors: INVALID_ARG, WORKSPACE, ARCH, CUDA; TIMEOUT in the status word. */
 int moe_gemm1_swiglu(const void* x_perm, const float* x_scale, const int32_t* offsets,
                      const void* w1, const float* w1_scale, const float* gate_scale,
-                     const float* up_scale, const moe_dims* dims, void* h, float* h_scale,
-                     void* ws, size_t ws_bytes, void* stream);
+                     const float* up_scale, const float* limits, const moe_dims* dims, void* h,
+                     float* h_scale, void* ws, size_t ws_bytes, void* stream);
 
 /* Grouped GEMM2 and the routing-weighted combine ([P5]: slot-specific weighted
  * reduction in fp32). y[r] = h[r] . W2[g]^T for each row r of group g (fp32
@@ -229,7 +242,7 @@ int moe_gemm2_combine(const void* h, const float* h_scale, const int32_t* offset
  * accumulation, bf16 out, unweighted) as the first half of moe_gemm2_combine. GEMM2 work
  * on a block of rows starts as soon as that block's h is complete, so the two GEMMs
  * overlap. ([P2] "Modifications", [P4] "Summary", [P5] per-expert dispatch.)
- *   Inputs as moe_gemm1_swiglu plus w2 / w2_scale as moe_gemm2_combine.
+ *   Inputs as moe_gemm1_swiglu (limits included) plus w2 / w2_scale as moe_gemm2_combine.
  *   h [A][I] (+ h_scale [I/128][A] for FP8) and y [A][H] bf16 are outputs.
  *   ws: moe_workspace_size(MOE_WS_EXPERTS); besides the header it holds per-block
  *   completion flags that must be zero when a call starts: zero the whole workspace once
@@ -237,8 +250,8 @@ int moe_gemm2_combine(const void* h, const float* h_scale, const int32_t* offset
  * Errors: INVALID_ARG, WORKSPACE, ARCH, CUDA; TIMEOUT / EXPERT_ID in the status word. */
 int moe_experts(const void* x_perm, const float* x_scale, const int32_t* offsets, const void* w1,
                 const float* w1_scale, const float* gate_scale, const float* up_scale,
-                const void* w2, const float* w2_scale, const moe_dims* dims, void* h,
-                float* h_scale, void* y, void* ws, size_t ws_bytes, void* stream);
+                const float* limits, const void* w2, const float* w2_scale, const moe_dims* dims,
+                void* h, float* h_scale, void* y, void* ws, size_t ws_bytes, void* stream);
 
 /* The routing-weighted combine alone ([P5] slot-specific weighted reduction):
  *   out[t] = sum_{j<k} topk_w[t][j] * y[inv_perm[t][j]]
@@ -255,15 +268,17 @@ int moe_combine(const void* y, const int32_t* offsets, const int32_t* inv_perm,
 /* The whole layer: moe_route_topk, moe_permute, moe_experts and moe_combine in sequence
  * on `stream`, with every intermediate in the workspace
  * (moe_workspace_size(MOE_WS_FORWARD)).
- *   logits [T][E+n_sink] fp32, x [T][H] bf16, weights and scales as above.
+ *   logits [T][E+n_sink] fp32, bias [E] or NULL, x [T][H] bf16, weights, scales and
+ *   limits as above.
  *   out [T][H] bf16 out.
- *   topk_ids / topk_w / shared_w: optional outputs ([T][k], [T][k], [T][n_sink]); pass
- *   NULL to keep them in the workspace.
+ *   topk_ids / topk_w / shared_w / packed: optional outputs ([T][k], [T][k], [T][n_sink],
+ *   [T][k]); pass NULL to keep the first three in the workspace and skip `packed`.
  * Errors: as the four calls. */
-int moe_forward(const float* logits, const void* x, const void* w1, const float* w1_scale,
-                const float* gate_scale, const float* up_scale, const void* w2,
-                const float* w2_scale, const moe_dims* dims, void* out, int32_t* topk_ids,
-                float* topk_w, float* shared_w, void* ws, size_t ws_bytes, void* stream);
+int moe_forward(const float* logits, const float* bias, const void* x, const void* w1,
+                const float* w1_scale, const float* gate_scale, const float* up_scale,
+                const float* limits, const void* w2, const float* w2_scale, const moe_dims* dims,
+                void* out, int32_t* topk_ids, float* topk_w, float* shared_w, uint32_t* packed,
+                void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -36,4 +36,5 @@ def oracle_layer_from_inputs(wl, host: dict) -> Layer:
                  wdtype=wl.wdtype, score=wl.score, alpha=wl.alpha, beta=wl.beta, limit=wl.limit,
                  route_scale=wl.route_scale, logits=host["logits"], x=host["x"], w1=host["w1"], w2=host["w2"],
                  w1_scale=host.get("w1_scale"), w2_scale=host.get("w2_scale"),
-                 gate_scale=host.get("gate_scale"), up_scale=host.get("up_scale"))
+                 gate_scale=host.get("gate_scale"), up_scale=host.get("up_scale"),
+                 limits=host.get("limits"), router_bias=host.get("router_bias"))

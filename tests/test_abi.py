@@ -26,7 +26,7 @@ def test_every_header_function_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert moe.moe_abi_version() == 1
+    assert moe.moe_abi_version() == 2
     for code in range(-7, 1):
         assert moe.status_string(code)
     assert "unknown" in moe.status_string(-99)
@@ -50,13 +50,13 @@ def test_invalid_dims_rejected(L, bad):
         moe.moe_workspace_size(d, moe.MOE_WS_FORWARD)
     assert ei.value.status == -1
     # the entry points reject the same dims before any CUDA call
-    assert L.moe_route_topk(None, ctypes.byref(d), None, None, None, None) == -1
+    assert L.moe_route_topk(None, ctypes.byref(d), None, None, None, None, None, None) == -1
 
 
 def test_null_pointers_and_small_workspace_rejected(L):
     d = _dims()
-    assert L.moe_route_topk(None, ctypes.byref(d), None, None, None, None) == -1
-    assert L.moe_forward(*([None] * 8), ctypes.byref(d), None, None, None, None, None, 0, None) == -1
+    assert L.moe_route_topk(None, ctypes.byref(d), None, None, None, None, None, None) == -1
+    assert L.moe_forward(*([None] * 10), ctypes.byref(d), None, None, None, None, None, None, 0, None) == -1
     fake = 1 << 20  # never dereferenced: the checks fail first
     n = moe.moe_workspace_size(d, moe.MOE_WS_PERMUTE)
     rc = L.moe_permute(fake, fake, ctypes.byref(d), fake, fake, fake, fake, None, fake, n - 1, None)
@@ -66,7 +66,7 @@ def test_null_pointers_and_small_workspace_rejected(L):
     rc = L.moe_permute(fake, fake + 2, ctypes.byref(d), fake, fake, fake, fake, None, fake, n, None)
     assert rc == -1  # x not 16-byte aligned
     # sink weights pointer must match n_sink
-    rc = L.moe_route_topk(fake, ctypes.byref(d), fake, fake, fake, None)
+    rc = L.moe_route_topk(fake, ctypes.byref(d), None, fake, fake, fake, None, None)
     assert rc == -1
 
 
@@ -91,3 +91,13 @@ def test_no_clamp_is_infinite_limit():
     d = moe.MoeDims.of(W.WORKLOADS["tiny"])
     assert math.isinf(d.limit) and d.limit > 0
     assert moe.MoeDims.of(W.WORKLOADS["oai_swiglu"]).limit == pytest.approx(7.0)
+
+
+def test_router_bias_needs_sigmoid_scoring(L):
+    """A correction bias is defined for the sigmoid ranking only: rejected before any CUDA call."""
+    fake = 1 << 20
+    d = _dims(score=moe.MOE_SCORE_SOFTMAX, n_sink=0)
+    assert L.moe_route_topk(fake, ctypes.byref(d), fake, fake, fake, None, None, None) == -2
+    ws_n = moe.moe_workspace_size(d, moe.MOE_WS_FORWARD)
+    assert L.moe_forward(fake, fake, fake, fake, None, None, None, None, fake, None, ctypes.byref(d), fake,
+                         None, None, None, None, fake, ws_n, None) == -2

@@ -65,7 +65,8 @@ def test_forward_empty_batch():
     d = moe.MoeDims.of(wl, T=0)
     ws = moe.alloc_workspace(moe.MoeDims.of(wl), moe.MOE_WS_FORWARD)
     out = torch.empty((0, wl.H), dtype=torch.bfloat16, device="cuda")
-    moe.moe_forward(inp["logits"][:0], inp["x"][:0], inp["w1"], None, None, None, inp["w2"], None, d, out, ws=ws)
+    moe.moe_forward(inp["logits"][:0], None, inp["x"][:0], inp["w1"], None, None, None, None, inp["w2"], None, d, out,
+                    ws=ws)
     assert moe.moe_read_status(ws) == 0
 
 
@@ -109,9 +110,9 @@ def test_public_stage_calls_reproduce_forward(name):
     ws_e = moe.alloc_workspace(d, moe.MOE_WS_EXPERTS)
     ws_c = moe.alloc_workspace(d, moe.MOE_WS_COMBINE)
     for _ in range(2):  # a second pass checks that the experts workspace is left reusable
-        moe.moe_route_topk(inp["logits"], d, ids, tw, sw)
+        moe.moe_route_topk(inp["logits"], d, None, ids, tw, sw)
         moe.moe_permute(ids, inp["x"], d, offsets, perm, inv, xp, xs, ws_p)
-        moe.moe_experts(xp, xs, offsets, inp["w1"], inp["w1_scale"], inp["gate_scale"], inp["up_scale"],
+        moe.moe_experts(xp, xs, offsets, inp["w1"], inp["w1_scale"], inp["gate_scale"], inp["up_scale"], None,
                         inp["w2"], inp["w2_scale"], d, h, hs, y, ws_e)
         moe.moe_combine(y, offsets, inv, tw, sw, d, out, ws_c)
         torch.cuda.synchronize()
@@ -122,3 +123,40 @@ def test_public_stage_calls_reproduce_forward(name):
     ref = oracle_layer(wl, inp).moe_rows(toks)
     got = out.float().cpu().numpy()[toks]
     (assert_fp8_close if fp8 else assert_bf16_close)(got, ref, name)
+
+
+def test_forward_with_router_bias_expert_limits_and_packed_output():
+    """moe_forward with a correction bias on the ranking, a clamp per expert and the packed
+    routing output, against the oracle given the same bias and limits (decode shape:
+    sigmoid scoring with sinks gating the shared experts)."""
+    from oracle.torch_io import host_inputs, oracle_layer_from_inputs
+    wl = W.WORKLOADS["decode_t64"]
+    inp = W.make_inputs(wl, "cuda")
+    g = torch.Generator(device="cuda").manual_seed(11)
+    bias = torch.randn((wl.E,), generator=g, device="cuda") * 0.05
+    limits = 0.5 + 2 * torch.rand((wl.E + wl.n_shared,), generator=g, device="cuda")  # pre-activation std ~1.3
+    d = moe.MoeDims.of(wl)
+    layer = moe.MoELayer(d, inp["w1"], inp["w2"], limits=limits, router_bias=bias)
+    T = wl.T
+    ids = torch.empty((T, wl.k), dtype=torch.int32, device="cuda")
+    tw = torch.empty((T, wl.k), dtype=torch.float32, device="cuda")
+    sw = torch.empty((T, wl.n_sink), dtype=torch.float32, device="cuda")
+    packed = torch.empty((T, wl.k), dtype=torch.int32, device="cuda")
+    out = layer.forward(inp["logits"], inp["x"], topk_ids=ids, topk_w=tw, shared_w=sw, packed=packed)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    o_ids, o_w, o_sw = oracle.route(f32(inp["logits"]), wl.E, wl.k, wl.score, wl.route_scale, bias=f32(bias))
+    assert np.array_equal(ids.cpu().numpy(), o_ids)
+    assert np.abs(tw.cpu().numpy() - o_w).max() <= 1e-6 and np.abs(sw.cpu().numpy() - o_sw).max() <= 1e-6
+    pk = packed.cpu().numpy().view(np.uint32)
+    wb = tw.cpu().to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16).astype(np.uint32)
+    assert np.array_equal(pk >> 16, o_ids.astype(np.uint32)) and np.array_equal(pk & 0xFFFF, wb)
+    host = host_inputs(inp)
+    host["router_bias"], host["limits"] = f32(bias), f32(limits)
+    ref = oracle_layer_from_inputs(wl, host).moe_rows(np.arange(T, dtype=np.int32))
+    assert_bf16_close(out.float().cpu().numpy(), ref, "bias + limits")
+    # the limits bite: without them the output differs by more than the tolerance
+    host0 = host_inputs(inp)
+    host0["router_bias"] = f32(bias)
+    ref0 = oracle_layer_from_inputs(wl, host0).moe_rows(np.arange(8, dtype=np.int32))
+    assert np.abs(ref0 - ref[:8]).max() > 0.05 * np.abs(ref[:8]).max()

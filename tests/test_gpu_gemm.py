@@ -15,7 +15,7 @@ from helpers import assert_bf16_close, assert_fp8_close, bits16, e4m3_to_np, f32
 pytestmark = pytest.mark.gpu
 
 
-def make_case(T, E, k, S, H, I, fp8, seed, gate_up_mult=1.0, scales=False, sinks=False, skew=0.0):
+def make_case(T, E, k, S, H, I, fp8, seed, gate_up_mult=1.0, scales=False, sinks=False, skew=0.0, limits=False):
     ids = W.random_topk_ids(T, E, k, seed=seed, skew=skew)
     offsets, perm, inv = oracle.permute(ids.numpy(), E, S)
     A = T * (k + S)
@@ -39,6 +39,12 @@ def make_case(T, E, k, S, H, I, fp8, seed, gate_up_mult=1.0, scales=False, sinks
         c["xp"], c["hp"] = xf.to(torch.bfloat16), hf.to(torch.bfloat16)
     c["gate_scale"] = (0.52 + 0.7 * torch.rand((G,), generator=g, device="cuda")) if scales else None
     c["up_scale"] = (0.52 + 0.7 * torch.rand((G,), generator=g, device="cuda")) if scales else None
+    # a clamp per expert: small enough to bite on the pre-activations (std ~0.45), one group unclamped
+    c["limits"] = None
+    if limits:
+        lim = 0.2 + 0.8 * torch.rand((G,), generator=g, device="cuda")
+        lim[G // 2] = float("inf")
+        c["limits"] = lim
     c["topk_w"] = torch.rand((T, k), generator=g, device="cuda")
     c["shared_w"] = torch.rand((T, S), generator=g, device="cuda") if (sinks and S) else None
     return c
@@ -58,7 +64,7 @@ def oracle_of(c, d):
                         x=np.zeros((c["T"], c["H"]), np.uint16),
                         w1=u8(c["w1"]) if fp8 else bits16(c["w1"]), w2=u8(c["w2"]) if fp8 else bits16(c["w2"]),
                         w1_scale=f32(c["w1_scale"]), w2_scale=f32(c["w2_scale"]),
-                        gate_scale=f32(c["gate_scale"]), up_scale=f32(c["up_scale"]))
+                        gate_scale=f32(c["gate_scale"]), up_scale=f32(c["up_scale"]), limits=f32(c.get("limits")))
 
 
 GEMM1_CASES = [
@@ -74,6 +80,8 @@ GEMM1_CASES = [
     (512, 8, 2, 0, 512, 256, True, {}),                         # FP8, tile 64
     (40, 32, 4, 1, 512, 256, True, {"glm": True}),              # FP8, tile 16, shared group, L = 10
     (200, 8, 2, 0, 1024, 512, True, {"oai": True, "scales": True}),
+    (128, 8, 2, 1, 512, 384, False, {"limits": True}),          # a clamp per expert (shared group too)
+    (300, 16, 4, 0, 512, 256, True, {"limits": True, "scales": True}),  # FP8, tile 32, clamp per expert
 ]
 
 
@@ -81,7 +89,7 @@ GEMM1_CASES = [
 def test_gemm1_swiglu(T, E, k, S, H, I, fp8, extra):
     oai, glm = extra.get("oai", False), extra.get("glm", False)
     c = make_case(T, E, k, S, H, I, fp8, seed=T + E + H, gate_up_mult=4.0 if oai else 1.0,
-                  scales=extra.get("scales", False), skew=extra.get("skew", 0.0))
+                  scales=extra.get("scales", False), skew=extra.get("skew", 0.0), limits=extra.get("limits", False))
     d = dims_of(c, alpha=1.702 if oai else 1.0, beta=1.0 if oai else 0.0,
                 limit=7.0 if oai else (10.0 if glm else math.inf))
     A = c["A"]
@@ -89,7 +97,8 @@ def test_gemm1_swiglu(T, E, k, S, H, I, fp8, extra):
     hs = torch.zeros((I // 128, A), dtype=torch.float32, device="cuda") if fp8 else None
     ws = moe.alloc_workspace(d, moe.MOE_WS_GEMM1)
     offsets = torch.from_numpy(c["offsets"]).cuda()
-    moe.moe_gemm1_swiglu(c["xp"], c["xs"], offsets, c["w1"], c["w1_scale"], c["gate_scale"], c["up_scale"], d,
+    moe.moe_gemm1_swiglu(c["xp"], c["xs"], offsets, c["w1"], c["w1_scale"], c["gate_scale"], c["up_scale"],
+                         c["limits"], d,
                          h, hs, ws)
     assert moe.moe_read_status(ws) == 0
     n = int(c["offsets"][-1])
