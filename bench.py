@@ -359,6 +359,36 @@ def run_ours(args):
     h2d = x_h.numel() * x_h.element_size() + lg_h.numel() * lg_h.element_size()
     d2h = out_h.numel() * out_h.element_size()
 
+    # ---- the fused gate GEMV + router (decode-sized batches, outside the layer step): x . W_gate
+    # with a seeded bf16 gate weight [E + n_sink][H], then the routing, in one launch
+    gate = None
+    if T <= 16:
+        gg = torch.Generator(device=dev).manual_seed(1)
+        w_gate = (torch.randn((wl.E + wl.n_sink, wl.H), generator=gg, device=dev) * 0.05).to(torch.bfloat16)
+        ws_g = moe.alloc_workspace(d, moe.MOE_WS_GATE_ROUTE, dev)
+        lg_g = torch.empty((T, wl.E + wl.n_sink), dtype=torch.float32, device=dev)
+        gate_fn = lambda: moe.moe_gate_route(inp["x"], w_gate, d, None, lg_g, ids, tw, sw, None, ws_g)  # noqa: E731
+        for _ in range(3):
+            gate_fn()
+        g_gate = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_gate):
+            gate_fn()
+        gt = []
+        for _ in range(max(1, min(K, 200))):
+            flush.zero_()
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            g_gate.replay()
+            b_.record(stream)
+            gt.append((a_, b_))
+        torch.cuda.synchronize(dev)
+        assert moe.moe_read_status(ws_g) == 0
+        gate = {"ms": max_over_ranks(sum(x.elapsed_time(y) for x, y in gt) / len(gt)),
+                "what": "moe_gate_route: gate GEMV over E + n_sink columns fused with the router, one launch, "
+                        "graph replay, L2 flushed; compare stages_ms.route (router alone, logits given)",
+                "w_gate_bytes": w_gate.numel() * 2}
+        del g_gate
+
     # ---- roofline of the dominant kernel: both grouped GEMMs (moe_experts, one launch)
     off = offsets.cpu().numpy()
     used = int(((off[1:] - off[:-1]) > 0).sum())
@@ -392,7 +422,7 @@ def run_ours(args):
             "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "roofline": roof, "clocks": clocks, "gpu_launches": 2 * launches_per_step * K,
-            "stages_ms": st, "forward_ms_per_step": fwd_ms, "experts_touched": used,
+            "stages_ms": st, "forward_ms_per_step": fwd_ms, "experts_touched": used, "gate_route": gate,
             "timing": "CUDA graph replays: value from the moe_forward graph; stages from one graph per public "
                       "call with device events between the launches",
             "layer_tflops": wl.flops() / (ms / 1e3) / 1e12,

@@ -21,6 +21,7 @@ MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_ARCH",
                 -4: "MOE_ERR_WORKSPACE", -5: "MOE_ERR_EXPERT_ID", -6: "MOE_ERR_TIMEOUT", -7: "MOE_ERR_CUDA"}
 MOE_WS_PERMUTE, MOE_WS_GEMM1, MOE_WS_GEMM2_COMBINE, MOE_WS_FORWARD, MOE_WS_EXPERTS, MOE_WS_COMBINE = 0, 1, 2, 3, 4, 5
+MOE_WS_GATE_ROUTE = 6
 MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
 MOE_WDTYPE_BF16, MOE_WDTYPE_FP8_E4M3_BLOCK128 = 0, 1
 
@@ -83,6 +84,7 @@ def lib() -> ctypes.CDLL:
             "moe_experts": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, P, _VP, _VP, _VP, _VP,
                              ctypes.c_size_t, _VP], ctypes.c_int),
             "moe_combine": ([_VP, _VP, _VP, _VP, _VP, P, _VP, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
+            "moe_gate_route": ([_VP, _VP, P, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -150,6 +152,13 @@ def moe_clear_status(ws, stream=None) -> None:
 def moe_route_topk(logits, dims: MoeDims, bias, topk_ids, topk_w, shared_w=None, packed=None, stream=None) -> None:
     _check("moe_route_topk", lib().moe_route_topk(_p(logits), ctypes.byref(dims), _p(bias), _p(topk_ids),
                                                   _p(topk_w), _p(shared_w), _p(packed), _s(stream)))
+
+
+def moe_gate_route(x, w_gate, dims: MoeDims, bias, logits, topk_ids, topk_w, shared_w, packed, ws,
+                   stream=None) -> None:
+    _check("moe_gate_route", lib().moe_gate_route(_p(x), _p(w_gate), ctypes.byref(dims), _p(bias), _p(logits),
+                                                  _p(topk_ids), _p(topk_w), _p(shared_w), _p(packed), _p(ws),
+                                                  _nbytes(ws), _s(stream)))
 
 
 def moe_permute(topk_ids, x, dims: MoeDims, offsets, perm, inv_perm, x_perm, x_scale, ws, stream=None) -> None:

@@ -58,7 +58,7 @@ bool is_fp8(const moe_dims* d) { return d->wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK12
 // Sub-buffers of a workspace, as byte offsets from its start.
 struct Layout {
     size_t ids = 0, w = 0, sw = 0, offsets = 0, perm = 0, inv = 0, xperm = 0, xscale = 0, h = 0, hscale = 0,
-           flags = 0, splitcnt = 0, part = 0, pscratch = 0, y = 0, total = 0;
+           flags = 0, splitcnt = 0, part = 0, pscratch = 0, y = 0, logits = 0, total = 0;
 };
 
 Layout layout(const moe_dims* d, int kind) {
@@ -90,6 +90,7 @@ Layout layout(const moe_dims* d, int kind) {
     }
     if (kind == MOE_WS_FORWARD || kind == MOE_WS_PERMUTE) L.pscratch = take(permute_scratch_bytes(d->T, d->k, d->E));
     if (kind == MOE_WS_FORWARD || kind == MOE_WS_GEMM2_COMBINE) L.y = take(A * H * 2);
+    if (kind == MOE_WS_GATE_ROUTE) L.logits = take(T * (size_t)(d->E + d->n_sink) * 4);
     L.total = off;
     return L;
 }
@@ -209,7 +210,7 @@ int moe_workspace_size(const moe_dims* dims, int kind, size_t* bytes) {
     if (!bytes) return MOE_ERR_INVALID_ARG;
     int rc = check_dims(dims);
     if (rc != MOE_OK) return rc;
-    if (kind < MOE_WS_PERMUTE || kind > MOE_WS_COMBINE) return MOE_ERR_INVALID_ARG;
+    if (kind < MOE_WS_PERMUTE || kind > MOE_WS_GATE_ROUTE) return MOE_ERR_INVALID_ARG;
     *bytes = layout(dims, kind).total;
     return MOE_OK;
 }
@@ -238,6 +239,28 @@ int moe_route_topk(const float* logits, const moe_dims* d, const float* bias, in
     if ((rc = check_bias(d, bias)) != MOE_OK) return rc;
     if ((rc = check_arch()) != MOE_OK) return rc;
     return do_route(logits, bias, d, topk_ids, topk_w, shared_w, packed, static_cast<cudaStream_t>(stream));
+}
+
+int moe_gate_route(const void* x, const void* w_gate, const moe_dims* d, const float* bias, float* logits,
+                   int32_t* topk_ids, float* topk_w, float* shared_w, uint32_t* packed, void* ws, size_t ws_bytes,
+                   void* stream) {
+    int rc = check_dims(d);
+    if (rc != MOE_OK) return rc;
+    if (d->T > 0) {
+        if (!x || !w_gate || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+        if ((d->n_sink > 0) != (shared_w != nullptr)) return MOE_ERR_INVALID_ARG;
+        if (!aligned(x, 16) || !aligned(w_gate, 16)) return MOE_ERR_INVALID_ARG;
+    }
+    if ((rc = check_bias(d, bias)) != MOE_OK) return rc;
+    if (d->T > kGateMaxTokens) return MOE_ERR_UNSUPPORTED;
+    if ((rc = check_ws(ws, ws_bytes, d, MOE_WS_GATE_ROUTE)) != MOE_OK) return rc;
+    if ((rc = check_arch()) != MOE_OK) return rc;
+    const Layout L = layout(d, MOE_WS_GATE_ROUTE);
+    float* lg = logits ? logits : at<float>(ws, L.logits);
+    unsigned int* counter = at<unsigned int>(ws, kWsGateCtrOffset);
+    return cuda_status(launch_gate_route(x, w_gate, bias, d->T, d->H, d->E, d->n_sink, d->k, d->score,
+                                         d->route_scale, lg, topk_ids, topk_w, shared_w, packed, counter,
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 int moe_permute(const int32_t* topk_ids, const void* x, const moe_dims* d, int32_t* offsets, int32_t* perm,

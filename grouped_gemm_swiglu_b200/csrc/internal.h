@@ -14,6 +14,14 @@ namespace moe {
 cudaError_t launch_router(const float* logits, const float* bias, int T, int N, int S, int k, int score,
                           float route_scale, int32_t* ids, float* w, float* sw, uint32_t* packed, cudaStream_t stream);
 
+// Fused gate GEMV + router for T <= kGateMaxTokens: logits[T][N+S] = x[T][H] . wg[N+S][H]^T
+// (bf16 in, fp32 accumulation), then the router. `counter`: one word, zero when idle,
+// left at zero.
+constexpr int kGateMaxTokens = 16;
+cudaError_t launch_gate_route(const void* x, const void* wg, const float* bias, int T, int H, int N, int S, int k,
+                              int score, float route_scale, float* logits, int32_t* ids, float* w, float* sw,
+                              uint32_t* packed, unsigned int* counter, cudaStream_t stream);
+
 // Scratch of the permutation: per 256-token chunk counts/bases [nchunk][E] and the
 // in-chunk rank of every (token, slot) [T][k]. `counter` is one word that must be zero
 // before the first call; every call leaves it at zero.

@@ -20,18 +20,24 @@
 
 namespace moe {
 
+// Logit loads: through the read-only path when the logits are an input of the launch,
+// through L2 when other CTAs of the same launch wrote them (the fused gate GEMV).
+template <bool COHERENT>
+__device__ __forceinline__ float load_logit(const float* p) {
+    if constexpr (COHERENT) return __ldcg(p);
+    else return __ldg(p);
+}
+
+// Routes token t with one warp (all 32 lanes must call it).
 // CPL = columns per lane (N <= 32*CPL). Lane l holds columns c*32 + l, c < CPL.
 // BIAS: rank on sigmoid(logit) + bias instead of the raw logit (a separate instance, so
 // the unbiased router keeps one value per column in registers).
-template <int CPL, bool BIAS>
-__global__ void __launch_bounds__(256) router_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
-                                                     int T, int N, int S, int k, int score, float route_scale,
-                                                     int32_t* __restrict__ ids, float* __restrict__ w,
-                                                     float* __restrict__ sw, uint32_t* __restrict__ packed) {
+template <int CPL, bool BIAS, bool COHERENT>
+__device__ __forceinline__ void route_token(const float* __restrict__ row, const float* __restrict__ bias, int t,
+                                            int N, int S, int k, int score, float route_scale,
+                                            int32_t* __restrict__ ids, float* __restrict__ w,
+                                            float* __restrict__ sw, uint32_t* __restrict__ packed) {
     const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (t >= T) return;
-    const float* row = logits + (size_t)t * (size_t)(N + S);
 
     float v[CPL];                 // raw logits: the value carried out of the selection
     float key[BIAS ? CPL : 1];    // BIAS: sigmoid(logit) + bias; else the key is v itself
@@ -40,7 +46,7 @@ __global__ void __launch_bounds__(256) router_kernel(const float* __restrict__ l
     for (int c = 0; c < CPL; ++c) {
         const int col = c * 32 + lane;
         if (col < N) {
-            v[c] = __ldg(row + col);
+            v[c] = load_logit<COHERENT>(row + col);
             if constexpr (BIAS) key[c] = __fadd_rn(__fdiv_rn(1.f, 1.f + expf(-v[c])), __ldg(bias + col));
             live |= 1u << c;
         } else {
@@ -90,7 +96,7 @@ __global__ void __launch_bounds__(256) router_kernel(const float* __restrict__ l
     const bool active = lane < k + S;
     float x = 0.f;
     if (lane < k) x = my_v;
-    else if (lane < k + S) x = __ldg(row + N + (lane - k));
+    else if (lane < k + S) x = load_logit<COHERENT>(row + N + (lane - k));
     float lp = x;
     if (score == MOE_SCORE_SIGMOID) lp = fminf(x, 0.f) - log1pf(expf(-fabsf(x)));  // logsigmoid
     float m = active ? lp : -FLT_MAX;
@@ -114,6 +120,110 @@ __global__ void __launch_bounds__(256) router_kernel(const float* __restrict__ l
     }
 }
 
+template <int CPL, bool BIAS>
+__global__ void __launch_bounds__(256) router_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
+                                                     int T, int N, int S, int k, int score, float route_scale,
+                                                     int32_t* __restrict__ ids, float* __restrict__ w,
+                                                     float* __restrict__ sw, uint32_t* __restrict__ packed) {
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    route_token<CPL, BIAS, false>(logits + (size_t)t * (size_t)(N + S), bias, t, N, S, k, score, route_scale, ids, w,
+                                  sw, packed);
+}
+
+// ---------------------------------------------------------------- fused gate GEMV + router
+// The 258-column gate GEMM and its epilogue in one launch for decode-sized batches
+// (sglang PR #36385: the fused gate GEMV path taken at <= 4 tokens; the op is
+// submission-bound there). logits[t][c] = sum_h x[t][h] * wg[c][h], fp32 accumulation
+// of the bf16 products. Each CTA computes kGateCols columns for every token, a column
+// split over kGateSplit warps (H/kGateSplit elements each, 16-byte loads), the partial
+// sums added in a fixed order. The CTA that finishes last (an atomic counter, then
+// reset to zero) routes every token from the finished logits.
+constexpr int kGateCols = 2;
+constexpr int kGateSplit = 4;  // warps per column: 8 warps = kGateCols * kGateSplit
+
+template <int TMAX, int CPL, bool BIAS>
+__global__ void __launch_bounds__(256) gate_route_kernel(const __nv_bfloat16* __restrict__ x,
+                                                         const __nv_bfloat16* __restrict__ wg,
+                                                         const float* __restrict__ bias, int T, int H, int N, int S,
+                                                         int k, int score, float route_scale, float* logits,
+                                                         int32_t* __restrict__ ids, float* __restrict__ w,
+                                                         float* __restrict__ sw, uint32_t* __restrict__ packed,
+                                                         unsigned int* counter) {
+    __shared__ float part[kGateCols][kGateSplit][TMAX];
+    __shared__ int s_last;
+    const int C = N + S;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int col_local = warp / kGateSplit, piece = warp % kGateSplit;
+    const int col = blockIdx.x * kGateCols + col_local;
+    const int len = H / kGateSplit;  // a multiple of 32 (H is a multiple of 128)
+    float acc[TMAX];
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) acc[t] = 0.f;
+    if (col < C) {
+        const __nv_bfloat16* wr = wg + (size_t)col * H + (size_t)piece * len;
+        for (int i = lane * 8; i < len; i += 32 * 8) {
+            const uint4 wv = __ldg(reinterpret_cast<const uint4*>(wr + i));
+            const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wv);
+            float wf[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __bfloat1622float2(w2[j]);
+                wf[2 * j] = f.x;
+                wf[2 * j + 1] = f.y;
+            }
+#pragma unroll
+            for (int t = 0; t < TMAX; ++t) {
+                if (t < T) {
+                    const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + (size_t)piece * len + i));
+                    const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 f = __bfloat1622float2(x2[j]);
+                        acc[t] = fmaf(f.x, wf[2 * j], acc[t]);
+                        acc[t] = fmaf(f.y, wf[2 * j + 1], acc[t]);
+                    }
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int t = 0; t < TMAX; ++t) part[col_local][piece][t] = acc[t];
+    }
+    __syncthreads();
+    if (threadIdx.x < kGateCols * TMAX) {
+        const int cl = threadIdx.x / TMAX, t = threadIdx.x % TMAX;
+        const int c = blockIdx.x * kGateCols + cl;
+        if (c < C && t < T) {
+            float v = 0.f;
+#pragma unroll
+            for (int q = 0; q < kGateSplit; ++q) v += part[cl][q][t];
+            logits[(size_t)t * C + c] = v;
+        }
+    }
+    // Publish this CTA's logits (fence before the count), and let the last CTA route.
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned int done = atomicAdd(counter, 1u);
+        s_last = done == gridDim.x - 1;
+        if (s_last) {
+            __threadfence();
+            atomicExch(counter, 0u);
+        }
+    }
+    __syncthreads();
+    if (!s_last) return;
+    for (int t = warp; t < T; t += blockDim.x >> 5)
+        route_token<CPL, BIAS, true>(logits + (size_t)t * C, bias, t, N, S, k, score, route_scale, ids, w, sw, packed);
+}
+
 cudaError_t launch_router(const float* logits, const float* bias, int T, int N, int S, int k, int score,
                           float route_scale, int32_t* ids, float* w, float* sw, uint32_t* packed, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
@@ -132,6 +242,45 @@ cudaError_t launch_router(const float* logits, const float* bias, int T, int N, 
     else MOE_ROUTER(32);
 #undef MOE_ROUTER
     return cudaGetLastError();
+}
+
+template <int TMAX>
+static cudaError_t launch_gate_t(const void* x, const void* wg, const float* bias, int T, int H, int N, int S, int k,
+                                 int score, float route_scale, float* logits, int32_t* ids, float* w, float* sw,
+                                 uint32_t* packed, unsigned int* counter, cudaStream_t stream) {
+    const int C = N + S;
+    dim3 grid((C + kGateCols - 1) / kGateCols), block(256);
+    auto xb = static_cast<const __nv_bfloat16*>(x);
+    auto wb = static_cast<const __nv_bfloat16*>(wg);
+#define MOE_GATE(CPL)                                                                                              \
+    (bias ? gate_route_kernel<TMAX, CPL, true><<<grid, block, 0, stream>>>(xb, wb, bias, T, H, N, S, k, score,     \
+                                                                           route_scale, logits, ids, w, sw, packed, \
+                                                                           counter)                                \
+          : gate_route_kernel<TMAX, CPL, false><<<grid, block, 0, stream>>>(xb, wb, bias, T, H, N, S, k, score,    \
+                                                                            route_scale, logits, ids, w, sw,        \
+                                                                            packed, counter))
+    if (N <= 32) MOE_GATE(1);
+    else if (N <= 64) MOE_GATE(2);
+    else if (N <= 128) MOE_GATE(4);
+    else if (N <= 256) MOE_GATE(8);
+    else if (N <= 512) MOE_GATE(16);
+    else MOE_GATE(32);
+#undef MOE_GATE
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gate_route(const void* x, const void* wg, const float* bias, int T, int H, int N, int S, int k,
+                              int score, float route_scale, float* logits, int32_t* ids, float* w, float* sw,
+                              uint32_t* packed, unsigned int* counter, cudaStream_t stream) {
+    if (T == 0) return cudaSuccess;
+    if (T <= 1) return launch_gate_t<1>(x, wg, bias, T, H, N, S, k, score, route_scale, logits, ids, w, sw, packed,
+                                        counter, stream);
+    if (T <= 4) return launch_gate_t<4>(x, wg, bias, T, H, N, S, k, score, route_scale, logits, ids, w, sw, packed,
+                                        counter, stream);
+    if (T <= 8) return launch_gate_t<8>(x, wg, bias, T, H, N, S, k, score, route_scale, logits, ids, w, sw, packed,
+                                        counter, stream);
+    return launch_gate_t<kGateMaxTokens>(x, wg, bias, T, H, N, S, k, score, route_scale, logits, ids, w, sw, packed,
+                                         counter, stream);
 }
 
 }  // namespace moe

@@ -111,7 +111,8 @@ typedef enum moe_ws_kind {
     MOE_WS_GEMM2_COMBINE = 2,
     MOE_WS_FORWARD = 3,
     MOE_WS_EXPERTS = 4,
-    MOE_WS_COMBINE = 5
+    MOE_WS_COMBINE = 5,
+    MOE_WS_GATE_ROUTE = 6
 } moe_ws_kind;
 
 /* ABI version compiled into the library (MOE_ABI_VERSION). */
@@ -153,6 +154,26 @@ int moe_clear_status(void* ws, void* stream);
  * with softmax), ARCH, CUDA. */
 int moe_route_topk(const float* logits, const moe_dims* dims, const float* bias, int32_t* topk_ids,
                    float* topk_w, float* shared_w, uint32_t* packed, void* stream);
+
+/* Gate GEMV fused with the router, for decode-sized batches ([P3]: the gate's fused GEMV
+ * path taken at <= 4 tokens, where the op is submission-bound; item 3 for the epilogue).
+ * One launch computes
+ *   logits[t][c] = sum_h x[t][h] * w_gate[c][h]     (bf16 products, fp32 accumulation;
+ *                                                    per column, per-warp partial sums over
+ *                                                    H/4 elements added in a fixed order)
+ * for the E routed and n_sink sink columns, then routes every token exactly as
+ * moe_route_topk does on those logits.
+ *   x        [T][H] bf16, 16-byte aligned; T <= 16 (larger T: a GEMM, then moe_route_topk;
+ *            UNSUPPORTED here).
+ *   w_gate   [E + n_sink][H] bf16, 16-byte aligned (row c = gate column c).
+ *   bias, topk_ids, topk_w, shared_w, packed   as moe_route_topk.
+ *   logits   [T][E + n_sink] fp32 out, or NULL to keep them in the workspace.
+ *   ws       moe_workspace_size(MOE_WS_GATE_ROUTE): the header (a completion counter that
+ *            every call leaves at zero) and room for the logits.
+ * Errors: INVALID_ARG, UNSUPPORTED (T > 16, bias with softmax), WORKSPACE, ARCH, CUDA. */
+int moe_gate_route(const void* x, const void* w_gate, const moe_dims* dims, const float* bias,
+                   float* logits, int32_t* topk_ids, float* topk_w, float* shared_w,
+                   uint32_t* packed, void* ws, size_t ws_bytes, void* stream);
 
 /* Permute by expert ([P5]: per-expert sorted-token dispatch; [P1]: fused act-quant).
  *   topk_ids [T][k] int32 in: expert ids in [0, E), distinct within a token.

@@ -58,6 +58,9 @@ def _load():
         lib.oracle_route.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+        lib.oracle_gate_logits.restype = ctypes.c_int
+        lib.oracle_gate_logits.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_void_p]
         lib.oracle_permute.restype = ctypes.c_int
         lib.oracle_permute.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
@@ -156,6 +159,18 @@ def route(logits, n_routed: int, k: int, score: int, route_scale: float = 1.0, b
     if rc != 0:
         raise ValueError("oracle_route: invalid arguments")
     return ids, w, sw
+
+
+def gate_logits(x_bits, w_bits):
+    """Gate GEMV: x bf16 bits [T,H], w bf16 bits [C,H] -> fp64 logits [T,C]."""
+    x = _c(x_bits, np.uint16)
+    w = _c(w_bits, np.uint16)
+    T, H = x.shape
+    C = w.shape[0]
+    out = np.empty((T, C), dtype=np.float64)
+    if _load().oracle_gate_logits(_ptr(x), _ptr(w), T, H, C, _ptr(out)) != 0:
+        raise ValueError("oracle_gate_logits: invalid sizes")
+    return out
 
 
 def permute(ids, E: int, n_shared: int = 0):

@@ -203,6 +203,21 @@ int oracle_route(const float* logits, const float* bias, int T, int N, int S, in
     return 0;
 }
 
+/* Gate GEMV in front of the router ([P3]: the 258-column gate GEMM whose output the
+ * epilogue routes, fused with it at <= 4 tokens): logits[t][c] = sum_h x[t][h] * w[c][h]
+ * with bf16 inputs and fp64 sums. x [T][H], w [C][H] bf16 bits; out [T][C] fp64. */
+int oracle_gate_logits(const uint16_t* x, const uint16_t* w, int T, int H, int C, double* out) {
+    if (T < 0 || H <= 0 || C <= 0) return -1;
+    for (int t = 0; t < T; ++t)
+        for (int c = 0; c < C; ++c) {
+            double acc = 0.0;
+            for (int h = 0; h < H; ++h)
+                acc += oracle_bf16_to_double(x[(int64_t)t * H + h]) * oracle_bf16_to_double(w[(int64_t)c * H + h]);
+            out[(int64_t)t * C + c] = acc;
+        }
+    return 0;
+}
+
 /* ------------------------------------------------------------------------- */
 /* Permutation by expert                                                      */
 /* ------------------------------------------------------------------------- */

@@ -101,3 +101,15 @@ def test_router_bias_needs_sigmoid_scoring(L):
     ws_n = moe.moe_workspace_size(d, moe.MOE_WS_FORWARD)
     assert L.moe_forward(fake, fake, fake, fake, None, None, None, None, fake, None, ctypes.byref(d), fake,
                          None, None, None, None, fake, ws_n, None) == -2
+
+
+def test_gate_route_checks(L):
+    """The fused gate GEMV + router takes T <= 16 and sizes its workspace for the logits."""
+    fake = 1 << 20
+    d = _dims(T=17)
+    n = moe.moe_workspace_size(d, moe.MOE_WS_GATE_ROUTE)
+    assert n >= 256 + 17 * (d.E + d.n_sink) * 4
+    assert L.moe_gate_route(fake, fake, ctypes.byref(d), None, None, fake, fake, None, None, fake, n, None) == -2
+    d = _dims(T=4)
+    assert L.moe_gate_route(fake, fake + 8, ctypes.byref(d), None, None, fake, fake, None, None, fake, n,
+                            None) == -1  # w_gate not 16-byte aligned

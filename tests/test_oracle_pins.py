@@ -262,6 +262,16 @@ def test_route_rejects_bias_with_softmax():
         oracle.route(np.zeros((2, 8), np.float32), 8, 2, oracle.SCORE_SOFTMAX, bias=np.zeros(8, np.float32))
 
 
+def test_gate_logits_match_torch_fp64_matmul():
+    # bf16 values are exact in fp64; torch's own bf16 -> fp64 conversion and matmul
+    rng = np.random.default_rng(24)
+    x = torch.from_numpy(rng.normal(0, 1, (5, 512))).to(torch.bfloat16)
+    w = torch.from_numpy(rng.normal(0, 0.05, (258, 512))).to(torch.bfloat16)
+    got = oracle.gate_logits(x.view(torch.int16).numpy().view(np.uint16), w.view(torch.int16).numpy().view(np.uint16))
+    ref = (x.double() @ w.double().T).numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-13, atol=1e-13)
+
+
 # --------------------------------------------------------------------------- permute
 
 @pytest.mark.parametrize("T,E,k,S", [(37, 8, 2, 0), (100, 16, 4, 1), (5, 300, 8, 2), (1, 4, 4, 0)])
