@@ -21,6 +21,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     int n_sink, int64_t A, uint16_t* __restrict__ out, int* status) {
     __shared__ int s_row[32];
     __shared__ float s_w[32];
+    pdl_trigger();
+    pdl_wait();
     const int t = blockIdx.x;
     const int nd = k + n_shared;
     if (threadIdx.x < nd) {
@@ -74,10 +76,8 @@ cudaError_t launch_combine(const void* y, const int32_t* offsets, const int32_t*
                            void* out, int* status, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
     dim3 grid(T, (H / 8 + kCombineThreads - 1) / kCombineThreads);
-    combine_kernel<<<grid, kCombineThreads, 0, stream>>>(static_cast<const uint16_t*>(y), offsets, inv, topk_w,
-                                                         shared_w, T, H, k, E, n_shared, n_sink, A,
-                                                         static_cast<uint16_t*>(out), status);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, grid, dim3(kCombineThreads), 0, stream, static_cast<const uint16_t*>(y), offsets,
+                      inv, topk_w, shared_w, T, H, k, E, n_shared, n_sink, A, static_cast<uint16_t*>(out), status);
 }
 
 }  // namespace moe

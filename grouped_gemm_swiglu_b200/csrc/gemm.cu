@@ -296,6 +296,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
+    // Everything above is private to the SM; the offsets (and all other global data) come
+    // from the previous kernels on the stream.
+    pdl_wait();
     // Token blocks per group and their running start: blk_start[g] = sum_{g'<g} ceil(n_g'/BN).
     // The offsets may come from the caller: group bounds are clamped into [0, A] (and a
     // bad array is flagged), so no tile ever reads or writes a row outside the matrices.
@@ -827,6 +830,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
     }
 
+    pdl_trigger();  // this CTA has no tiles left: the next kernel may launch
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -962,8 +966,7 @@ static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
         }
     }
     if (smem > (size_t)limit) return cudaErrorInvalidValue;
-    moe_gemm_kernel<C><<<num_sms(), C::THREADS, smem, stream>>>(tmW1, tmX, tmW2, tmH, p);
-    return cudaGetLastError();
+    return launch_pdl(moe_gemm_kernel<C>, dim3(num_sms()), dim3(C::THREADS), smem, stream, tmW1, tmX, tmW2, tmH, p);
 }
 
 int gemm_pick_bn(int64_t A, int G, bool fp8) {

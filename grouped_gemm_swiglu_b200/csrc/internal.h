@@ -10,6 +10,36 @@
 
 namespace moe {
 
+// Programmatic dependent launch. Every kernel of the library is launched with
+// launch_pdl, so it may start while the previous kernel on the stream is finishing; each
+// kernel calls pdl_wait() before it touches global memory (which waits for the previous
+// grid to complete and its writes to be visible), so the order of completion stays that
+// of the stream and only launch latency and prologues overlap. pdl_trigger() lets the
+// next kernel launch: the small kernels call it on entry, the grouped-GEMM kernel when a
+// CTA runs out of tiles. A dependent grid starts only after every CTA of its predecessor
+// has triggered or exited, so it never takes resources that a pending predecessor CTA
+// needs. Without the launch attribute (or with a plain predecessor) both are no-ops.
+#ifdef __CUDACC__
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+#endif
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // bias [N] or NULL (rank on the raw logit); packed [T][k] or NULL.
 cudaError_t launch_router(const float* logits, const float* bias, int T, int N, int S, int k, int score,
                           float route_scale, int32_t* ids, float* w, float* sw, uint32_t* packed, cudaStream_t stream);

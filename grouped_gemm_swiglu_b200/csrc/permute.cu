@@ -66,7 +66,9 @@ __global__ void __launch_bounds__(256) permute_count_kernel(const int32_t* __res
     uint32_t* flags = sm;                                      // [8][E] membership bitmaps
     uint16_t* pre = reinterpret_cast<uint16_t*>(sm + 8 * E);  // [8][E] rows of earlier warps
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_trigger();
     for (int i = threadIdx.x; i < 8 * E; i += blockDim.x) flags[i] = 0;
+    pdl_wait();
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < zero_words; i += (size_t)gridDim.x * blockDim.x)
         zero[i] = 0;
     __syncthreads();
@@ -141,6 +143,8 @@ __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
     int64_t A, int32_t* __restrict__ perm, int32_t* __restrict__ inv, void* __restrict__ x_perm,
     float* __restrict__ x_scale, int* status) {
     __shared__ int s_dst[32];
+    pdl_trigger();
+    pdl_wait();
     const int t = blockIdx.x;
     const int nd = k + n_shared;
     if (threadIdx.x < nd) {
@@ -226,19 +230,14 @@ cudaError_t launch_permute(const int32_t* ids, const void* x, int T, int H, int 
         err = cudaFuncSetAttribute(permute_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
         if (err != cudaSuccess) return err;
     }
-    permute_count_kernel<<<nchunk, 256, sm1, stream>>>(ids, T, k, E, n_shared, cnt, rank, offsets, counter, status,
-                                                       zero, zero ? zero_words : 0);
+    err = launch_pdl(permute_count_kernel, dim3(nchunk), dim3(256), sm1, stream, ids, T, k, E, n_shared, cnt, rank,
+                     offsets, counter, status, zero, zero ? zero_words : (size_t)0);
+    if (err != cudaSuccess) return err;
     const int64_t A = (int64_t)T * (k + n_shared);
     dim3 grid(T, (H / 8 + kScatterThreads - 1) / kScatterThreads);
-    if (fp8)
-        permute_scatter_kernel<true><<<grid, kScatterThreads, 0, stream>>>(
-            ids, rank, cnt, offsets, static_cast<const uint16_t*>(x), T, H, k, E, n_shared, A, perm, inv, x_perm,
-            x_scale, status);
-    else
-        permute_scatter_kernel<false><<<grid, kScatterThreads, 0, stream>>>(
-            ids, rank, cnt, offsets, static_cast<const uint16_t*>(x), T, H, k, E, n_shared, A, perm, inv, x_perm,
-            x_scale, status);
-    return cudaGetLastError();
+    return launch_pdl(fp8 ? permute_scatter_kernel<true> : permute_scatter_kernel<false>, grid, dim3(kScatterThreads),
+                      0, stream, ids, static_cast<const int32_t*>(rank), static_cast<const int32_t*>(cnt), offsets,
+                      static_cast<const uint16_t*>(x), T, H, k, E, n_shared, A, perm, inv, x_perm, x_scale, status);
 }
 
 }  // namespace moe

@@ -125,6 +125,8 @@ __global__ void __launch_bounds__(256) router_kernel(const float* __restrict__ l
                                                      int T, int N, int S, int k, int score, float route_scale,
                                                      int32_t* __restrict__ ids, float* __restrict__ w,
                                                      float* __restrict__ sw, uint32_t* __restrict__ packed) {
+    pdl_trigger();
+    pdl_wait();
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
     route_token<CPL, BIAS, false>(logits + (size_t)t * (size_t)(N + S), bias, t, N, S, k, score, route_scale, ids, w,
@@ -154,6 +156,8 @@ __global__ void __launch_bounds__(256) gate_route_kernel(const __nv_bfloat16* __
     __shared__ int s_last;
     const int C = N + S;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_trigger();
+    pdl_wait();
     const int col_local = warp / kGateSplit, piece = warp % kGateSplit;
     const int col = blockIdx.x * kGateCols + col_local;
     const int len = H / kGateSplit;  // a multiple of 32 (H is a multiple of 128)
@@ -229,19 +233,16 @@ cudaError_t launch_router(const float* logits, const float* bias, int T, int N, 
     if (T == 0) return cudaSuccess;
     const int warps = 8;
     dim3 grid((T + warps - 1) / warps), block(32 * warps);
-#define MOE_ROUTER(CPL)                                                                                        \
-    (bias ? router_kernel<CPL, true><<<grid, block, 0, stream>>>(logits, bias, T, N, S, k, score, route_scale, ids, \
-                                                                  w, sw, packed)                                  \
-          : router_kernel<CPL, false><<<grid, block, 0, stream>>>(logits, bias, T, N, S, k, score, route_scale,   \
-                                                                   ids, w, sw, packed))
+#define MOE_ROUTER(CPL)                                                                                          \
+    return launch_pdl(bias ? router_kernel<CPL, true> : router_kernel<CPL, false>, grid, block, 0, stream, logits, \
+                      bias, T, N, S, k, score, route_scale, ids, w, sw, packed)
     if (N <= 32) MOE_ROUTER(1);
-    else if (N <= 64) MOE_ROUTER(2);
-    else if (N <= 128) MOE_ROUTER(4);
-    else if (N <= 256) MOE_ROUTER(8);
-    else if (N <= 512) MOE_ROUTER(16);
-    else MOE_ROUTER(32);
+    if (N <= 64) MOE_ROUTER(2);
+    if (N <= 128) MOE_ROUTER(4);
+    if (N <= 256) MOE_ROUTER(8);
+    if (N <= 512) MOE_ROUTER(16);
+    MOE_ROUTER(32);
 #undef MOE_ROUTER
-    return cudaGetLastError();
 }
 
 template <int TMAX>
@@ -252,21 +253,16 @@ static cudaError_t launch_gate_t(const void* x, const void* wg, const float* bia
     dim3 grid((C + kGateCols - 1) / kGateCols), block(256);
     auto xb = static_cast<const __nv_bfloat16*>(x);
     auto wb = static_cast<const __nv_bfloat16*>(wg);
-#define MOE_GATE(CPL)                                                                                              \
-    (bias ? gate_route_kernel<TMAX, CPL, true><<<grid, block, 0, stream>>>(xb, wb, bias, T, H, N, S, k, score,     \
-                                                                           route_scale, logits, ids, w, sw, packed, \
-                                                                           counter)                                \
-          : gate_route_kernel<TMAX, CPL, false><<<grid, block, 0, stream>>>(xb, wb, bias, T, H, N, S, k, score,    \
-                                                                            route_scale, logits, ids, w, sw,        \
-                                                                            packed, counter))
+#define MOE_GATE(CPL)                                                                                         \
+    return launch_pdl(bias ? gate_route_kernel<TMAX, CPL, true> : gate_route_kernel<TMAX, CPL, false>, grid, block, \
+                      0, stream, xb, wb, bias, T, H, N, S, k, score, route_scale, logits, ids, w, sw, packed, counter)
     if (N <= 32) MOE_GATE(1);
-    else if (N <= 64) MOE_GATE(2);
-    else if (N <= 128) MOE_GATE(4);
-    else if (N <= 256) MOE_GATE(8);
-    else if (N <= 512) MOE_GATE(16);
-    else MOE_GATE(32);
+    if (N <= 64) MOE_GATE(2);
+    if (N <= 128) MOE_GATE(4);
+    if (N <= 256) MOE_GATE(8);
+    if (N <= 512) MOE_GATE(16);
+    MOE_GATE(32);
 #undef MOE_GATE
-    return cudaGetLastError();
 }
 
 cudaError_t launch_gate_route(const void* x, const void* wg, const float* bias, int T, int H, int N, int S, int k,
