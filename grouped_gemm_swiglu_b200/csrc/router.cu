@@ -140,11 +140,14 @@ __global__ void __launch_bounds__(256) router_kernel(const float* __restrict__ l
 // of the bf16 products. Each CTA computes kGateCols columns for every token, a column
 // split over kGateSplit warps (H/kGateSplit elements each, 16-byte loads), the partial
 // sums added in a fixed order. The CTA that finishes last (an atomic counter, then
-// reset to zero) routes every token from the finished logits.
+// reset to zero) routes every token from the finished logits. XSMEM: the CTA first copies
+// x into shared memory (one coalesced pass), so the dot products read every token's row
+// from there instead of from L2 once per 8-element chunk.
 constexpr int kGateCols = 2;
 constexpr int kGateSplit = 4;  // warps per column: 8 warps = kGateCols * kGateSplit
+constexpr size_t kGateXSmemMax = 96 * 1024;
 
-template <int TMAX, int CPL, bool BIAS>
+template <int TMAX, int CPL, bool BIAS, bool XSMEM>
 __global__ void __launch_bounds__(256) gate_route_kernel(const __nv_bfloat16* __restrict__ x,
                                                          const __nv_bfloat16* __restrict__ wg,
                                                          const float* __restrict__ bias, int T, int H, int N, int S,
@@ -154,10 +157,19 @@ __global__ void __launch_bounds__(256) gate_route_kernel(const __nv_bfloat16* __
                                                          unsigned int* counter) {
     __shared__ float part[kGateCols][kGateSplit][TMAX];
     __shared__ int s_last;
+    extern __shared__ __align__(16) uint8_t gate_sm[];
     const int C = N + S;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_trigger();
     pdl_wait();
+    const __nv_bfloat16* xs = x;
+    if constexpr (XSMEM) {
+        uint4* dst = reinterpret_cast<uint4*>(gate_sm);
+        const int nvec = T * H / 8;
+        for (int v = threadIdx.x; v < nvec; v += blockDim.x) dst[v] = __ldg(reinterpret_cast<const uint4*>(x) + v);
+        __syncthreads();
+        xs = reinterpret_cast<const __nv_bfloat16*>(gate_sm);
+    }
     const int col_local = warp / kGateSplit, piece = warp % kGateSplit;
     const int col = blockIdx.x * kGateCols + col_local;
     const int len = H / kGateSplit;  // a multiple of 32 (H is a multiple of 128)
@@ -166,6 +178,7 @@ __global__ void __launch_bounds__(256) gate_route_kernel(const __nv_bfloat16* __
     for (int t = 0; t < TMAX; ++t) acc[t] = 0.f;
     if (col < C) {
         const __nv_bfloat16* wr = wg + (size_t)col * H + (size_t)piece * len;
+#pragma unroll 4
         for (int i = lane * 8; i < len; i += 32 * 8) {
             const uint4 wv = __ldg(reinterpret_cast<const uint4*>(wr + i));
             const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wv);
@@ -179,7 +192,8 @@ __global__ void __launch_bounds__(256) gate_route_kernel(const __nv_bfloat16* __
 #pragma unroll
             for (int t = 0; t < TMAX; ++t) {
                 if (t < T) {
-                    const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + (size_t)piece * len + i));
+                    const uint4* xp = reinterpret_cast<const uint4*>(xs + (size_t)t * H + (size_t)piece * len + i);
+                    const uint4 xv = XSMEM ? *xp : __ldg(xp);
                     const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
@@ -253,9 +267,20 @@ static cudaError_t launch_gate_t(const void* x, const void* wg, const float* bia
     dim3 grid((C + kGateCols - 1) / kGateCols), block(256);
     auto xb = static_cast<const __nv_bfloat16*>(x);
     auto wb = static_cast<const __nv_bfloat16*>(wg);
-#define MOE_GATE(CPL)                                                                                         \
-    return launch_pdl(bias ? gate_route_kernel<TMAX, CPL, true> : gate_route_kernel<TMAX, CPL, false>, grid, block, \
-                      0, stream, xb, wb, bias, T, H, N, S, k, score, route_scale, logits, ids, w, sw, packed, counter)
+    const size_t xbytes = (size_t)T * H * 2;
+    const bool xsmem = T >= 2 && xbytes <= kGateXSmemMax;  // one token: nothing to share, skip the copy
+#define MOE_GATE(CPL)                                                                                                \
+    {                                                                                                                \
+        auto kern = xsmem ? (bias ? gate_route_kernel<TMAX, CPL, true, true> : gate_route_kernel<TMAX, CPL, false, true>) \
+                          : (bias ? gate_route_kernel<TMAX, CPL, true, false>                                        \
+                                  : gate_route_kernel<TMAX, CPL, false, false>);                                     \
+        if (xsmem && xbytes > 48 * 1024) {                                                                           \
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGateXSmemMax); \
+            if (e != cudaSuccess) return e;                                                                          \
+        }                                                                                                            \
+        return launch_pdl(kern, grid, block, xsmem ? xbytes : (size_t)0, stream, xb, wb, bias, T, H, N, S, k, score,  \
+                          route_scale, logits, ids, w, sw, packed, counter);                                         \
+    }
     if (N <= 32) MOE_GATE(1);
     if (N <= 64) MOE_GATE(2);
     if (N <= 128) MOE_GATE(4);
