@@ -21,6 +21,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 
 WDTYPE_BF16 = 0
 WDTYPE_FP8 = 1
+WDTYPE_INT4 = 2
 SCORE_SOFTMAX = 0
 SCORE_SIGMOID = 1
 
@@ -61,6 +62,9 @@ def _load():
         lib.oracle_gate_logits.restype = ctypes.c_int
         lib.oracle_gate_logits.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, ctypes.c_void_p]
+        lib.oracle_int4_at.restype = ctypes.c_double
+        lib.oracle_int4_at.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                       ctypes.c_int64]
         lib.oracle_permute.restype = ctypes.c_int
         lib.oracle_permute.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
@@ -161,6 +165,19 @@ def route(logits, n_routed: int, k: int, score: int, route_scale: float = 1.0, b
     return ids, w, sw
 
 
+def int4_dequant(packed, scale_bits):
+    """INT4 group-32 weights: packed uint8 [rows, K/2], bf16 scale bits [rows, K/32] -> fp64 [rows, K]."""
+    p = _c(packed, np.uint8)
+    s = _c(scale_bits, np.uint16)
+    rows, K = p.shape[0], p.shape[1] * 2
+    lib = _load()
+    out = np.empty((rows, K), dtype=np.float64)
+    for r in range(rows):
+        for c in range(K):
+            out[r, c] = lib.oracle_int4_at(_ptr(p), _ptr(s), K, r, c)
+    return out
+
+
 def gate_logits(x_bits, w_bits):
     """Gate GEMV: x bf16 bits [T,H], w bf16 bits [C,H] -> fp64 logits [T,C]."""
     x = _c(x_bits, np.uint16)
@@ -201,9 +218,10 @@ class Layer:
                  route_scale, logits, x, w1, w2, w1_scale=None, w2_scale=None,
                  gate_scale=None, up_scale=None, limits=None, router_bias=None):
         wt = np.uint16 if wdtype == WDTYPE_BF16 else np.uint8
+        st = np.uint16 if wdtype == WDTYPE_INT4 else np.float32  # INT4 group scales are bf16 bits
         self._keep = dict(
             logits=_c(logits, np.float32), x=_c(x, np.uint16), w1=_c(w1, wt), w2=_c(w2, wt),
-            w1_scale=_c(w1_scale, np.float32), w2_scale=_c(w2_scale, np.float32),
+            w1_scale=_c(w1_scale, st), w2_scale=_c(w2_scale, st),
             gate_scale=_c(gate_scale, np.float32), up_scale=_c(up_scale, np.float32),
             limits=_c(limits, np.float32), router_bias=_c(router_bias, np.float32))
         k_ = self._keep

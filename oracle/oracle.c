@@ -264,36 +264,66 @@ int oracle_permute(const int32_t* ids, int T, int k, int E, int n_shared,
 
 typedef struct {
     int32_t T, H, I, E, k, n_sink, n_shared;
-    int32_t wdtype;               /* 0: bf16 weights; 1: E4M3 with 128x128 fp32 block scales */
+    int32_t wdtype;               /* 0: bf16 weights; 1: E4M3 with 128x128 fp32 block scales;
+                                     2: INT4 group-32 with bf16 scales (activations bf16) */
     int32_t score;                /* 0: softmax renorm; 1: sigmoid + logsigmoid-LSE renorm */
     int32_t pad_;
     double alpha, beta, limit, route_scale;
     const float* logits;          /* [T][E + n_sink] fp32 */
     const uint16_t* x;            /* [T][H] bf16 bits */
     const void* w1;               /* [E+n_shared][2I][H]; rows [0,I) gate, [I,2I) up */
-    const float* w1_scale;        /* wdtype 1: [E+n_shared][2I/128][H/128] */
+    const void* w1_scale;         /* wdtype 1: fp32 [E+n_shared][2I/128][H/128];
+                                     wdtype 2: bf16 bits [E+n_shared][2I][H/32] */
     const void* w2;               /* [E+n_shared][H][I] */
-    const float* w2_scale;        /* wdtype 1: [E+n_shared][H/128][I/128] */
+    const void* w2_scale;         /* wdtype 1: fp32 [E+n_shared][H/128][I/128];
+                                     wdtype 2: bf16 bits [E+n_shared][H][I/32] */
     const float* gate_scale;      /* [E+n_shared] or NULL (1.0) */
     const float* up_scale;        /* [E+n_shared] or NULL (1.0) */
     const float* limits;          /* [E+n_shared] clamp per expert, or NULL (limit) */
     const float* router_bias;     /* [E] correction bias of the ranking, or NULL */
 } oracle_layer;
 
+/* Round to bf16, nearest even, a value exactly representable in binary32 (finite). */
+static double round_bf16(double v) {
+    float f = (float)v;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    u &= 0xFFFF0000u;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* INT4 group-32 element (batchgen PR #239 commit notes): packed [rows][K/2] bytes, the
+ * low nibble holding the even K index and the high nibble the odd one; scale [rows][K/32]
+ * bf16; value (nibble - 8) * scale, taken in bf16 as the dot products consume it (the
+ * product has at most 12 significant bits, so it is exact before that rounding). */
+double oracle_int4_at(const uint8_t* packed, const uint16_t* scale, int64_t K, int64_t row, int64_t col) {
+    uint8_t b = packed[row * (K / 2) + col / 2];
+    int n = (col & 1) ? (b >> 4) : (b & 0xF);
+    double s = oracle_bf16_to_double(scale[row * (K / 32) + col / 32]);
+    return round_bf16((double)(n - 8) * s);
+}
+
 /* Dequantised weight element. */
 static double w1_at(const oracle_layer* L, int e, int64_t row, int64_t col) {
     int64_t idx = ((int64_t)e * 2 * L->I + row) * L->H + col;
     if (L->wdtype == 0) return oracle_bf16_to_double(((const uint16_t*)L->w1)[idx]);
+    if (L->wdtype == 2)
+        return oracle_int4_at((const uint8_t*)L->w1, (const uint16_t*)L->w1_scale, L->H, (int64_t)e * 2 * L->I + row,
+                              col);
     int64_t nbr = 2 * L->I / 128, nbc = L->H / 128;
-    double s = L->w1_scale[((int64_t)e * nbr + row / 128) * nbc + col / 128];
+    double s = ((const float*)L->w1_scale)[((int64_t)e * nbr + row / 128) * nbc + col / 128];
     return oracle_e4m3_decode(((const uint8_t*)L->w1)[idx]) * s;
 }
 
 static double w2_at(const oracle_layer* L, int e, int64_t row, int64_t col) {
     int64_t idx = ((int64_t)e * L->H + row) * L->I + col;
     if (L->wdtype == 0) return oracle_bf16_to_double(((const uint16_t*)L->w2)[idx]);
+    if (L->wdtype == 2)
+        return oracle_int4_at((const uint8_t*)L->w2, (const uint16_t*)L->w2_scale, L->I, (int64_t)e * L->H + row, col);
     int64_t nbr = L->H / 128, nbc = L->I / 128;
-    double s = L->w2_scale[((int64_t)e * nbr + row / 128) * nbc + col / 128];
+    double s = ((const float*)L->w2_scale)[((int64_t)e * nbr + row / 128) * nbc + col / 128];
     return oracle_e4m3_decode(((const uint8_t*)L->w2)[idx]) * s;
 }
 
@@ -401,7 +431,7 @@ int oracle_gemm1_rows(const oracle_layer* L, int64_t A, const void* xp, const fl
         if (r < 0 || r >= A) { bad = 1; continue; }
         double* xv = (double*)malloc(sizeof(double) * (size_t)L->H);
         for (int64_t c = 0; c < L->H; ++c) {
-            if (L->wdtype == 0) xv[c] = oracle_bf16_to_double(((const uint16_t*)xp)[r * L->H + c]);
+            if (L->wdtype != 1) xv[c] = oracle_bf16_to_double(((const uint16_t*)xp)[r * L->H + c]);
             else xv[c] = oracle_e4m3_decode(((const uint8_t*)xp)[r * L->H + c]) * (double)xs[(c / 128) * A + r];
         }
         expert_gemm1(L, row_expert[it], xv, h + (int64_t)it * L->I);
@@ -435,7 +465,7 @@ int oracle_gemm2_rows(const oracle_layer* L, int64_t A, const void* hp, const fl
             while (g < G && !(offsets[g] <= r && r < offsets[g + 1])) ++g;
             if (g == G) { bad = 1; break; }
             for (int64_t i = 0; i < L->I; ++i) {
-                if (L->wdtype == 0) hv[i] = oracle_bf16_to_double(((const uint16_t*)hp)[r * L->I + i]);
+                if (L->wdtype != 1) hv[i] = oracle_bf16_to_double(((const uint16_t*)hp)[r * L->I + i]);
                 else hv[i] = oracle_e4m3_decode(((const uint8_t*)hp)[r * L->I + i]) * (double)hs[(i / 128) * A + r];
             }
             expert_gemm2(L, g, hv, y);

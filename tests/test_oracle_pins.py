@@ -516,3 +516,49 @@ def test_layer_router_bias_changes_only_the_selection():
     ref = sum(wts[:, j:j + 1] * _dense_mlp(x, _bf16_val(d["w1"][e]), _bf16_val(d["w2"][e]), I)
               for j, e in enumerate([2, 4]))
     np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- INT4 group-32 weights
+
+def _torch_int4_dequant(packed, scale_bits):
+    """The pages' rule with torch ops: low nibble = even K, high = odd K, (nibble - 8) * scale
+    as a bf16 product (torch multiplies bf16 in fp32 and rounds to bf16 once)."""
+    p = torch.from_numpy(packed.astype(np.int32))
+    n = torch.stack([(p & 0xF) - 8, (p >> 4) - 8], dim=-1).reshape(p.shape[0], -1)
+    s = torch.from_numpy(scale_bits.view(np.int16)).view(torch.bfloat16).repeat_interleave(32, dim=1)
+    return n.to(torch.bfloat16) * s
+
+
+def test_int4_dequant_follows_the_nibble_order_and_group_scale():
+    rng = np.random.default_rng(41)
+    packed = rng.integers(0, 256, (6, 64), dtype=np.uint8)  # K = 128: 4 groups of 32
+    scales = _bf16_bits(rng.normal(0, 0.3, (6, 4)))
+    packed[0, 0], packed[0, 1] = 0x2F, 0x80  # K 0..3: nibbles 15, 2, 0, 8 -> 7s, -6s, -8s, 0
+    got = oracle.int4_dequant(packed, scales)
+    ref = _torch_int4_dequant(packed, scales).double().numpy()
+    np.testing.assert_array_equal(got, ref)
+    s0 = float(_bf16_val(scales[0, 0]))
+    # byte 0x2F: low nibble 15 is K 0 (+7 s), high nibble 2 is K 1 (-6 s); byte 0x80: 0 -> -8 s, 8 -> 0
+    assert got[0, 2] == -8 * s0 and got[0, 3] == 0.0   # powers of two times s: exact in bf16
+    np.testing.assert_allclose(got[0, :2], [7 * s0, -6 * s0], rtol=2 ** -8)
+
+
+def test_layer_int4_equals_bf16_layer_with_dequantised_weights():
+    # the INT4 layer must compute exactly the bf16 layer whose weights are the dequantised
+    # INT4 weights (the same fp64 arithmetic on the same values)
+    rng = np.random.default_rng(42)
+    T, H, I, E, k, S = 6, 128, 64, 4, 2, 1
+    G = E + S
+    w1p = rng.integers(0, 256, (G, 2 * I, H // 2), dtype=np.uint8)
+    w2p = rng.integers(0, 256, (G, H, I // 2), dtype=np.uint8)
+    w1s = _bf16_bits(np.abs(rng.normal(0.01, 0.003, (G, 2 * I, H // 32))))
+    w2s = _bf16_bits(np.abs(rng.normal(0.01, 0.003, (G, H, I // 32))))
+    x = _bf16_bits(rng.normal(0, 1, (T, H)))
+    logits = rng.normal(0, 1, (T, E)).astype(np.float32)
+    common = dict(T=T, H=H, I=I, E=E, k=k, n_sink=0, n_shared=S, score=oracle.SCORE_SOFTMAX, alpha=1.702, beta=1.0,
+                  limit=7.0, route_scale=1.0, logits=logits, x=x)
+    q = oracle.Layer(**common, wdtype=oracle.WDTYPE_INT4, w1=w1p, w2=w2p, w1_scale=w1s, w2_scale=w2s)
+    w1b = np.stack([_torch_int4_dequant(w1p[g], w1s[g]).view(torch.int16).numpy().view(np.uint16) for g in range(G)])
+    w2b = np.stack([_torch_int4_dequant(w2p[g], w2s[g]).view(torch.int16).numpy().view(np.uint16) for g in range(G)])
+    b = oracle.Layer(**common, wdtype=oracle.WDTYPE_BF16, w1=w1b, w2=w2b)
+    np.testing.assert_array_equal(q.moe_rows(np.arange(T)), b.moe_rows(np.arange(T)))
