@@ -25,7 +25,8 @@ int check_dims(const moe_dims* d) {
     if (d->n_sink < 0 || d->k + d->n_sink > kMaxSlots) return MOE_ERR_INVALID_ARG;
     if (d->n_shared < 0 || d->k + d->n_shared > kMaxSlots) return MOE_ERR_INVALID_ARG;
     if (d->score != MOE_SCORE_SOFTMAX && d->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
-    if (d->wdtype != MOE_WDTYPE_BF16 && d->wdtype != MOE_WDTYPE_FP8_E4M3_BLOCK128) return MOE_ERR_INVALID_ARG;
+    if (d->wdtype != MOE_WDTYPE_BF16 && d->wdtype != MOE_WDTYPE_FP8_E4M3_BLOCK128 && d->wdtype != MOE_WDTYPE_INT4_G32)
+        return MOE_ERR_INVALID_ARG;
     if (d->n_sink > 0 && d->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
     if (d->n_sink > 0 && d->n_shared > 0 && d->n_shared != d->n_sink) return MOE_ERR_INVALID_ARG;
     if (!std::isfinite(d->alpha) || !std::isfinite(d->beta) || !std::isfinite(d->route_scale))
@@ -54,6 +55,7 @@ int64_t rows_A(const moe_dims* d) { return (int64_t)d->T * (d->k + d->n_shared);
 int groups(const moe_dims* d) { return d->E + d->n_shared; }
 size_t act_elt(const moe_dims* d) { return d->wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128 ? 1 : 2; }
 bool is_fp8(const moe_dims* d) { return d->wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128; }
+bool is_int4(const moe_dims* d) { return d->wdtype == MOE_WDTYPE_INT4_G32; }
 
 // Sub-buffers of a workspace, as byte offsets from its start.
 struct Layout {
@@ -85,8 +87,8 @@ Layout layout(const moe_dims* d, int kind) {
     // block flags and split-K counters are adjacent so one clear covers both
     if (kind == MOE_WS_FORWARD || kind == MOE_WS_EXPERTS) L.flags = take(gemm_block_flags_bytes(A, G));
     if (kind == MOE_WS_FORWARD || kind == MOE_WS_EXPERTS || kind == MOE_WS_GEMM1) {
-        L.splitcnt = take(gemm_split_counter_bytes(A, G, H, I, is_fp8(d)));
-        L.part = take(gemm_split_scratch_bytes(A, G, H, I, is_fp8(d)));
+        L.splitcnt = take(gemm_split_counter_bytes(A, G, H, I, d->wdtype));
+        L.part = take(gemm_split_scratch_bytes(A, G, H, I, d->wdtype));
     }
     if (kind == MOE_WS_FORWARD || kind == MOE_WS_PERMUTE) L.pscratch = take(permute_scratch_bytes(d->T, d->k, d->E));
     if (kind == MOE_WS_FORWARD || kind == MOE_WS_GEMM2_COMBINE) L.y = take(A * H * 2);
@@ -136,6 +138,7 @@ MoeGemmArgs gemm_args(const moe_dims* d, const int32_t* offsets, int* status) {
     a.H = d->H;
     a.I = d->I;
     a.fp8 = is_fp8(d);
+    a.int4 = d->wdtype == MOE_WDTYPE_INT4_G32;
     a.alpha = d->alpha;
     a.beta = d->beta;
     a.limit = d->limit;
@@ -145,7 +148,7 @@ MoeGemmArgs gemm_args(const moe_dims* d, const int32_t* offsets, int* status) {
     return a;
 }
 
-int do_gemm1(const void* xperm, const float* xscale, const int32_t* offsets, const void* w1, const float* w1s,
+int do_gemm1(const void* xperm, const float* xscale, const int32_t* offsets, const void* w1, const void* w1s,
              const float* gs, const float* us, const float* limits, const moe_dims* d, void* h, float* hs, void* ws,
              cudaStream_t s) {
     const Layout L = layout(d, MOE_WS_GEMM1);
@@ -172,7 +175,7 @@ int do_combine(const void* y, const int32_t* offsets, const int32_t* inv, const 
 }
 
 int do_gemm2_combine(const void* h, const float* hs, const int32_t* offsets, const int32_t* inv, const float* topk_w,
-                     const float* shared_w, const void* w2, const float* w2s, const moe_dims* d, void* out, void* y,
+                     const float* shared_w, const void* w2, const void* w2s, const moe_dims* d, void* out, void* y,
                      int* status, cudaStream_t s) {
     MoeGemmArgs a = gemm_args(d, offsets, status);
     a.run_gemm2 = true;
@@ -281,13 +284,14 @@ int moe_permute(const int32_t* topk_ids, const void* x, const moe_dims* d, int32
 }
 
 int moe_gemm1_swiglu(const void* x_perm, const float* x_scale, const int32_t* offsets, const void* w1,
-                     const float* w1_scale, const float* gate_scale, const float* up_scale, const float* limits,
+                     const void* w1_scale, const float* gate_scale, const float* up_scale, const float* limits,
                      const moe_dims* d, void* h, float* h_scale, void* ws, size_t ws_bytes, void* stream) {
     int rc = check_dims(d);
     if (rc != MOE_OK) return rc;
     if (d->T > 0) {
         if (!x_perm || !offsets || !w1 || !h) return MOE_ERR_INVALID_ARG;
         if (is_fp8(d) && (!x_scale || !w1_scale || !h_scale)) return MOE_ERR_INVALID_ARG;
+        if (is_int4(d) && (!w1_scale || !aligned(w1_scale, 4))) return MOE_ERR_INVALID_ARG;
         if (!aligned(x_perm, 16) || !aligned(w1, 16) || !aligned(h, 16)) return MOE_ERR_INVALID_ARG;
     }
     if ((rc = check_ws(ws, ws_bytes, d, MOE_WS_GEMM1)) != MOE_OK) return rc;
@@ -298,7 +302,7 @@ int moe_gemm1_swiglu(const void* x_perm, const float* x_scale, const int32_t* of
 }
 
 int moe_gemm2_combine(const void* h, const float* h_scale, const int32_t* offsets, const int32_t* inv_perm,
-                      const float* topk_w, const float* shared_w, const void* w2, const float* w2_scale,
+                      const float* topk_w, const float* shared_w, const void* w2, const void* w2_scale,
                       const moe_dims* d, void* out, void* ws, size_t ws_bytes, void* stream) {
     int rc = check_dims(d);
     if (rc != MOE_OK) return rc;
@@ -306,6 +310,7 @@ int moe_gemm2_combine(const void* h, const float* h_scale, const int32_t* offset
         if (!h || !offsets || !inv_perm || !topk_w || !w2 || !out) return MOE_ERR_INVALID_ARG;
         if ((d->n_sink > 0) != (shared_w != nullptr)) return MOE_ERR_INVALID_ARG;
         if (is_fp8(d) && (!h_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
+        if (is_int4(d) && (!w2_scale || !aligned(w2_scale, 4))) return MOE_ERR_INVALID_ARG;
         if (!aligned(h, 16) || !aligned(w2, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
     }
     if ((rc = check_ws(ws, ws_bytes, d, MOE_WS_GEMM2_COMBINE)) != MOE_OK) return rc;
@@ -317,14 +322,16 @@ int moe_gemm2_combine(const void* h, const float* h_scale, const int32_t* offset
 }
 
 int moe_experts(const void* x_perm, const float* x_scale, const int32_t* offsets, const void* w1,
-                const float* w1_scale, const float* gate_scale, const float* up_scale, const float* limits,
-                const void* w2, const float* w2_scale, const moe_dims* d, void* h, float* h_scale, void* y, void* ws,
+                const void* w1_scale, const float* gate_scale, const float* up_scale, const float* limits,
+                const void* w2, const void* w2_scale, const moe_dims* d, void* h, float* h_scale, void* y, void* ws,
                 size_t ws_bytes, void* stream) {
     int rc = check_dims(d);
     if (rc != MOE_OK) return rc;
     if (d->T > 0) {
         if (!x_perm || !offsets || !w1 || !w2 || !h || !y) return MOE_ERR_INVALID_ARG;
         if (is_fp8(d) && (!x_scale || !w1_scale || !w2_scale || !h_scale)) return MOE_ERR_INVALID_ARG;
+        if (is_int4(d) && (!w1_scale || !w2_scale || !aligned(w1_scale, 4) || !aligned(w2_scale, 4)))
+            return MOE_ERR_INVALID_ARG;
         if (!aligned(x_perm, 16) || !aligned(w1, 16) || !aligned(w2, 16) || !aligned(h, 16) || !aligned(y, 16))
             return MOE_ERR_INVALID_ARG;
     }
@@ -368,9 +375,9 @@ int moe_combine(const void* y, const int32_t* offsets, const int32_t* inv_perm, 
                       static_cast<cudaStream_t>(stream));
 }
 
-int moe_forward(const float* logits, const float* bias, const void* x, const void* w1, const float* w1_scale,
+int moe_forward(const float* logits, const float* bias, const void* x, const void* w1, const void* w1_scale,
                 const float* gate_scale, const float* up_scale, const float* limits, const void* w2,
-                const float* w2_scale, const moe_dims* d, void* out, int32_t* topk_ids, float* topk_w,
+                const void* w2_scale, const moe_dims* d, void* out, int32_t* topk_ids, float* topk_w,
                 float* shared_w, uint32_t* packed, void* ws, size_t ws_bytes, void* stream) {
     int rc = check_dims(d);
     if (rc != MOE_OK) return rc;
@@ -378,6 +385,8 @@ int moe_forward(const float* logits, const float* bias, const void* x, const voi
     if (d->T > 0) {
         if (!logits || !x || !w1 || !w2 || !out) return MOE_ERR_INVALID_ARG;
         if (is_fp8(d) && (!w1_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
+        if (is_int4(d) && (!w1_scale || !w2_scale || !aligned(w1_scale, 4) || !aligned(w2_scale, 4)))
+            return MOE_ERR_INVALID_ARG;
         if (!aligned(x, 16) || !aligned(w1, 16) || !aligned(w2, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
         if (shared_w && d->n_sink == 0) return MOE_ERR_INVALID_ARG;
     }
@@ -397,7 +406,7 @@ int moe_forward(const float* logits, const float* bias, const void* x, const voi
     // The counting kernel also clears the GEMM's per-block completion flags.
     int* flags = at<int>(ws, L.flags);
     const size_t clear_words =
-        (L.splitcnt + gemm_split_counter_bytes(rows_A(d), groups(d), d->H, d->I, is_fp8(d)) - L.flags) / sizeof(int);
+        (L.splitcnt + gemm_split_counter_bytes(rows_A(d), groups(d), d->H, d->I, d->wdtype) - L.flags) / sizeof(int);
     if ((rc = do_permute(ids, x, d, offsets, at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv), at<void>(ws, L.xperm),
                          xscale, at<void>(ws, L.pscratch), status, s, flags, clear_words)) != MOE_OK)
         return rc;

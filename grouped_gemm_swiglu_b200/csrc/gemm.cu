@@ -54,14 +54,22 @@ constexpr int pow2_at_least(int v) {
     return p;
 }
 
-template <int BN_, bool FP8_>
+template <int BN_, bool FP8_, bool INT4_ = false>
 struct Cfg {
     static constexpr int BN = BN_;
     static constexpr bool FP8 = FP8_;
+    // INT4 group-32 weights: TMA brings the packed bytes (RAW_BYTES per 128x64 block),
+    // dequantisation warps write the bf16 tiles the MMA reads; everything else is bf16.
+    static constexpr bool INT4 = INT4_;
     static constexpr int BK = FP8 ? 128 : 64;  // K elements per stage: one 128-byte row
     static constexpr int A_BYTES = 128 * 128;
     static constexpr int B_BYTES = BN * 128;
-    static constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES;  // sized for GEMM1 (gate + up)
+    static constexpr int RAW_BYTES = INT4 ? 128 * 32 : 0;
+    static constexpr int RAW_OFF = 2 * A_BYTES + B_BYTES;  // packed A0, A1 after the bf16 tiles and B
+    static constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES + 2 * RAW_BYTES;  // sized for GEMM1 (gate + up)
+    // Dequantisation warps: 8 for decode-sized tiles (one weight row of one of the two tiles
+    // per thread, the epilogue then has 4 warps), else 4 (one row of both tiles per thread).
+    static constexpr int DQ = INT4 ? (BN <= 32 ? 8 : 4) : 0;
     // Token rows arrive in boxes of up to 64 rows, and only the boxes a tile's rows reach
     // are loaded, so a short token block does not pull a full BN-row tile through L2.
     static constexpr int BOX_ROWS = BN < 64 ? BN : 64;
@@ -80,8 +88,8 @@ struct Cfg {
     // Epilogue warps: groups of four (one warp per TMEM lane quarter), each group owning
     // an equal share of the tile's columns; four groups at 256 columns, whose single
     // accumulator buffer makes the drain time part of the tile time.
-    static constexpr int EPI = BN >= 256 ? 16 : 8;
-    static constexpr int THREADS = 64 + 32 * EPI;
+    static constexpr int EPI = BN >= 256 ? 16 : ((INT4 && BN <= 32) ? 4 : 8);
+    static constexpr int THREADS = 64 + 32 * EPI + 32 * DQ;
     static constexpr int GROUPS = EPI / 4;
     static constexpr int COLS = BN / GROUPS;  // columns per epilogue warp
     static constexpr int CW = COLS < 16 ? COLS : 16;  // TMEM load width (columns)
@@ -94,13 +102,15 @@ struct Cfg {
     static_assert(!FP8 || COLS <= 32, "FP8 loads a warp's whole column share at once");
     static_assert(BN % BOX_ROWS == 0 && BN <= 256, "token tile = whole boxes, at most the MMA's N limit");
     static_assert(STAGES >= 2, "at least two pipeline stages");
+    static_assert(!(INT4 && FP8), "INT4 weights take bf16 activations");
     static_assert(COLS % 8 == 0, "split-K merges columns in chunks of 8");
     // Split-K of GEMM1 is compiled in where it can be chosen (see gemm_split_factor):
     // every tile width except FP8 at 64 columns, whose promotion registers are full.
     static constexpr bool SPLIT_OK = !(FP8 && BN >= 64);
 
-    // full/empty per stage, tfull/tempty per TMEM buffer, ring_full/ring_empty x kRing, drain, epibar
-    static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 2 * kRing + 2;
+    // full/empty per stage, tfull/tempty per TMEM buffer, ring_full/ring_empty x kRing, drain,
+    // epibar, and for INT4 raw_full per stage (packed bytes and token rows landed)
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 2 * kRing + 2 + (INT4 ? STAGES : 0);
     static constexpr size_t ctrl_bytes() {
         return 8 * NUM_BARS + 16 + 4 * kRing + 16 + 4 * RED_FLOATS + 16 + 4 * SCT_FLOATS;
     }
@@ -115,8 +125,8 @@ struct DevArgs {
     int c1;      // GEMM1 tiles per token block: I/128 (0 = phase absent)
     int c2;      // GEMM2 tiles per token block: ceil(H/256), each two 128-row chunks of H (0 = absent)
     const float* x_scale;   // FP8: [H/128][A]
-    const float* w1_scale;  // FP8: [G][2I/128][H/128]
-    const float* w2_scale;  // FP8: [G][H/128][I/128]
+    const void* w1_scale;   // FP8: fp32 [G][2I/128][H/128]; INT4: bf16 [G][2I][H/32]
+    const void* w2_scale;   // FP8: fp32 [G][H/128][I/128]; INT4: bf16 [G][H][I/32]
     const float* gate_scale;
     const float* up_scale;
     float alpha, beta, limit;
@@ -239,6 +249,53 @@ __device__ __forceinline__ void sum_split_partials(const float* part_tile, int s
     }
 }
 
+// INT4 group-32 dequantisation of one 64-deep weight row segment into the bf16 tile the
+// MMA reads (batchgen PR #239 commit notes: low nibble = even K, value (nibble - 8) *
+// scale with one bf16 scale per 32 K, taken in bf16).
+//   raw: the row's 32 packed bytes; sc: its two group scales (bf16 bits, K 0-31, 32-63);
+//   dst: the row (128 bytes) of the 128B-swizzled K-major tile; r: the row index in the tile.
+// Each byte becomes one bf16x2 pair: the bf16 with bits 0x4300 | n is exactly 128 + n, so
+// subtracting 136 gives n - 8 exactly, and one packed bf16 multiply (round to nearest
+// even) gives the weight. lo / hi hold the low / high nibbles of the word's four bytes
+// (one per byte); a byte permute puts byte j's pair in bytes 0 and 2 of one word.
+__device__ __forceinline__ uint32_t byte_perm(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t int4_pair_bf16(uint32_t lo, uint32_t hi, int byte, __nv_bfloat162 s) {
+    // selector: result byte 0 = byte `byte` of lo, byte 2 = byte `byte` of hi (index 4 + byte)
+    const uint32_t u = (byte_perm(lo, hi, (uint32_t)byte | ((uint32_t)(4 + byte) << 8)) & 0x00FF00FFu) | 0x43004300u;
+    __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&u);
+    v = __hmul2(__hsub2(v, __float2bfloat162_rn(136.f)), s);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void dequant_int4_row(const uint8_t* raw, uint32_t sc, uint8_t* dst, int r) {
+    __nv_bfloat162 s[2];
+    s[0] = __halves2bfloat162(__ushort_as_bfloat16((unsigned short)(sc & 0xFFFFu)),
+                              __ushort_as_bfloat16((unsigned short)(sc & 0xFFFFu)));
+    s[1] = __halves2bfloat162(__ushort_as_bfloat16((unsigned short)(sc >> 16)),
+                              __ushort_as_bfloat16((unsigned short)(sc >> 16)));
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const uint4 q = *reinterpret_cast<const uint4*>(raw + 16 * half);
+        const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {  // 16-byte chunk (8 K elements) 4*half + c of the row
+            const uint32_t lo = qw[c] & 0x0F0F0F0Fu, hi = (qw[c] >> 4) & 0x0F0F0F0Fu;
+            uint4 o;
+            o.x = int4_pair_bf16(lo, hi, 0, s[half]);
+            o.y = int4_pair_bf16(lo, hi, 1, s[half]);
+            o.z = int4_pair_bf16(lo, hi, 2, s[half]);
+            o.w = int4_pair_bf16(lo, hi, 3, s[half]);
+            const int chunk = (4 * half + c) ^ (r & 7);  // 128-byte swizzle: chunk XOR row mod 8
+            *reinterpret_cast<uint4*>(dst + chunk * 16) = o;
+        }
+    }
+}
+
 // Warp-collective bounded wait: lane 0 waits, the verdict is broadcast.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, PipeAbort* ab, int* status) {
     bool ok = true;
@@ -263,7 +320,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint64_t* ring_empty = ring_full + kRing;
     uint64_t* drain = ring_empty + kRing;
     uint64_t* epibar = drain + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epibar + 1);
+    uint64_t* raw_full = epibar + 1;  // INT4 only: [STAGES]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(raw_full + (C::INT4 ? C::STAGES : 0));
     PipeAbort* ab = reinterpret_cast<PipeAbort*>(tmem_slot + 1);
     int* ring = reinterpret_cast<int*>(tmem_slot + 4);
     float* red = reinterpret_cast<float*>(ring + kRing + 4);
@@ -276,7 +334,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], C::INT4 ? C::DQ : 1);  // INT4: the dequantisation warps complete it
+            if (C::INT4) mbar_init(&raw_full[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < C::NBUF; ++b) {
@@ -285,7 +344,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         for (int r = 0; r < kRing; ++r) {
             mbar_init(&ring_full[r], 1);
-            mbar_init(&ring_empty[r], 1 + C::EPI);
+            mbar_init(&ring_empty[r], 1 + C::EPI + C::DQ);
         }
         mbar_init(drain, 1);
         mbar_init(epibar, C::EPI);
@@ -367,7 +426,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const int kbase = g1 ? tl.ks * all_kb / p.s1 : 0;  // this tile's K blocks
                 const int num_kb = g1 ? (tl.ks + 1) * all_kb / p.s1 - kbase : all_kb;
                 const int n_box = (max(16, (tl.nrows + 15) & ~15) + C::BOX_ROWS - 1) / C::BOX_ROWS;
-                const uint32_t tx = (tl.dual ? 2 : 1) * C::A_BYTES + n_box * C::BOX_BYTES;
+                const uint32_t tx = (tl.dual ? 2 : 1) * (C::INT4 ? C::RAW_BYTES : C::A_BYTES) + n_box * C::BOX_BYTES;
                 auto load_act = [&](uint8_t* st, uint64_t* bar, int kx) {
                     for (int r = 0; r < n_box; ++r)
                         tma_load_2d(st + 2 * C::A_BYTES + r * C::BOX_BYTES, ta, bar, kx, tl.row0 + r * C::BOX_ROWS);
@@ -384,7 +443,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     const bool dep_ok = wait_counter_geq(p.done1 + tl.blk, p.c1, ab, p.status);
                     uint32_t s2 = st0;
                     for (int k2 = 0; k2 < pre; ++k2) {
-                        load_act(smem + (size_t)s2 * C::STAGE_BYTES, &full[s2], (kbase + k2) * C::BK);
+                        load_act(smem + (size_t)s2 * C::STAGE_BYTES, C::INT4 ? &raw_full[s2] : &full[s2],
+                                 (kbase + k2) * C::BK);
                         if (++s2 == (uint32_t)C::STAGES) s2 = 0;
                     }
                     return dep_ok;
@@ -399,11 +459,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         break;
                     }
                     uint8_t* st = smem + (size_t)stage * C::STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full[stage], tx);
+                    uint64_t* bar = C::INT4 ? &raw_full[stage] : &full[stage];
+                    mbar_arrive_expect_tx(bar, tx);
                     const int kx = (kbase + kb) * C::BK;
-                    tma_load_2d(st, tw, &full[stage], kx, tl.a0row);
-                    if (tl.dual) tma_load_2d(st + C::A_BYTES, tw, &full[stage], kx, tl.a1row);
-                    if (kb >= pre) load_act(st, &full[stage], kx);
+                    if constexpr (C::INT4) {  // packed weight bytes: x is a byte offset (2 K per byte)
+                        tma_load_2d(st + C::RAW_OFF, tw, bar, kx / 2, tl.a0row);
+                        if (tl.dual) tma_load_2d(st + C::RAW_OFF + C::RAW_BYTES, tw, bar, kx / 2, tl.a1row);
+                    } else {
+                        tma_load_2d(st, tw, bar, kx, tl.a0row);
+                        if (tl.dual) tma_load_2d(st + C::A_BYTES, tw, bar, kx, tl.a1row);
+                    }
+                    if (kb >= pre) load_act(st, bar, kx);
                     pend_mask |= 1u << stage;
                     pend_phase = (pend_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == (uint32_t)C::STAGES) {
@@ -415,7 +481,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             }
             // Never leave with a copy in flight: wait for the last fill of every stage.
             for (int s = 0; s < C::STAGES; ++s)
-                if ((pend_mask >> s) & 1u) mbar_wait_drain(&full[s], (pend_phase >> s) & 1u);
+                if ((pend_mask >> s) & 1u)
+                    mbar_wait_drain(C::INT4 ? &raw_full[s] : &full[s], (pend_phase >> s) & 1u);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -486,6 +553,60 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             mbar_wait_drain(drain, 0);
         }
         __syncwarp();
+    } else if (C::INT4 && warp >= 2 + C::EPI) {
+        // ------------------------------------------------------------ INT4 dequantisation
+        // Thread dt converts weight row r = dt % 128 of tile dt / 128 (A0, A1; with 4 warps
+        // both tiles) of every stage, in the same tile order as the MMA, then the warp
+        // completes the stage's `full` barrier.
+        const int dt = (warp - 2 - C::EPI) * 32 + lane;
+        const int r = dt % 128;
+        constexpr int kTileStep = C::DQ * 32 / 128;  // tiles apart that one thread converts
+        uint32_t stage = 0, phase = 0;
+        bool ok = true;
+        for (int i = 0; ok; ++i) {
+            const int slot = i % kRing;
+            if (!warp_wait(&ring_full[slot], (i / kRing) & 1, ab, p.status)) break;
+            const int L = ring[slot];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ring_empty[slot]);
+            if (L < 0) break;
+            const Tile tl = decode_tile<C::BN>(L, T1, blk_start, s_off, p);
+            const bool g1 = tl.phase == 1;
+            const int K = g1 ? p.H : p.I;
+            const int all_kb = K / C::BK;
+            const int kbase = g1 ? tl.ks * all_kb / p.s1 : 0;
+            const int num_kb = g1 ? (tl.ks + 1) * all_kb / p.s1 - kbase : all_kb;
+            // this row's bf16 group scales: [rows][K/32], two groups (one 32-bit word) per stage
+            const uint32_t* sc = static_cast<const uint32_t*>(g1 ? p.w1_scale : p.w2_scale);
+            const int t0 = dt / 128;  // first tile of this thread (0 = A0, 1 = A1)
+            const bool has0 = t0 == 0 || tl.dual;
+            const bool has1 = kTileStep == 1 && tl.dual;  // a second tile (A1) when 4 warps cover both
+            const uint32_t* sc0 = sc + (size_t)((t0 == 0 ? tl.a0row : tl.a1row) + r) * (K / 64) + kbase;
+            const uint32_t* sc1 = sc + (size_t)(tl.a1row + r) * (K / 64) + kbase;
+            uint32_t s0 = has0 ? __ldg(sc0) : 0u, s1 = has1 ? __ldg(sc1) : 0u;
+            for (int kb = 0; kb < num_kb; ++kb) {
+                // the next stage's scales are loaded before this stage's bytes are awaited
+                const bool more = kb + 1 < num_kb;
+                const uint32_t n0 = (more && has0) ? __ldg(sc0 + kb + 1) : 0u;
+                const uint32_t n1 = (more && has1) ? __ldg(sc1 + kb + 1) : 0u;
+                if (!warp_wait(&raw_full[stage], phase, ab, p.status)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* st = smem + (size_t)stage * C::STAGE_BYTES;
+                if (has0) dequant_int4_row(st + C::RAW_OFF + t0 * C::RAW_BYTES + r * 32, s0, st + t0 * C::A_BYTES + r * 128, r);
+                if (has1) dequant_int4_row(st + C::RAW_OFF + C::RAW_BYTES + r * 32, s1, st + C::A_BYTES + r * 128, r);
+                fence_proxy_async_smem();  // these generic writes are read by the MMA (async proxy)
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[stage]);
+                if (++stage == (uint32_t)C::STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+                s0 = n0;
+                s1 = n1;
+            }
+        }
     } else {
         // ------------------------------------------------------------ epilogue
         const int ew = warp - 2;
@@ -640,7 +761,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const int num_kb = g1 ? (tl.ks + 1) * kblocks / p.s1 - kbase : kblocks;
                 const float* act_scale = g1 ? p.x_scale : p.h_scale;
                 // block scales of A0 and A1: weight row block a_row / 128 of the [G*rows/128][K/128] grid
-                const float* wscale = g1 ? p.w1_scale : p.w2_scale;
+                const float* wscale = static_cast<const float*>(g1 ? p.w1_scale : p.w2_scale);
                 const float* wsg = wscale + (size_t)(tl.a0row / 128) * kblocks + kbase;
                 const float* wsu = wscale + (size_t)(tl.a1row / 128) * kblocks + kbase;
                 float acc_g[C::COLS], acc_u[C::COLS];
@@ -876,6 +997,21 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
+// INT4 weights: rows x K/2 packed bytes, box = 128 rows x 32 bytes (64 K), no swizzle: the
+// dequantisation warps read each row's 32 bytes and write the swizzled bf16 tile.
+static bool make_map_int4(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {K / 2, rows};
+    cuuint64_t strides[1] = {K / 2};
+    cuuint32_t box[2] = {32, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // 2D K-major tensor map: rows x K elements, box = box_rows x 128 bytes, 128B swizzle.
 static bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, bool fp8, uint32_t box_rows) {
     auto enc = tensor_map_encoder();
@@ -914,8 +1050,11 @@ static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
     const uint64_t k1 = p1 ? a.H : a.I, k2 = p2 ? a.I : a.H;
     const uint64_t r1 = p1 ? (uint64_t)a.G * 2 * a.I : (uint64_t)a.G * a.H;
     const uint64_t r2 = p2 ? (uint64_t)a.G * a.H : (uint64_t)a.G * 2 * a.I;
-    if (!make_map(&tmW1, w1, r1, k1, C::FP8, 128) || !make_map(&tmX, x, (uint64_t)a.A, k1, C::FP8, C::BOX_ROWS) ||
-        !make_map(&tmW2, w2, r2, k2, C::FP8, 128) || !make_map(&tmH, hh, (uint64_t)a.A, k2, C::FP8, C::BOX_ROWS))
+    auto wmap = [&](CUtensorMap* m, const void* base, uint64_t rows, uint64_t K) {
+        return C::INT4 ? make_map_int4(m, base, rows, K) : make_map(m, base, rows, K, C::FP8, 128);
+    };
+    if (!wmap(&tmW1, w1, r1, k1) || !make_map(&tmX, x, (uint64_t)a.A, k1, C::FP8, C::BOX_ROWS) ||
+        !wmap(&tmW2, w2, r2, k2) || !make_map(&tmH, hh, (uint64_t)a.A, k2, C::FP8, C::BOX_ROWS))
         return cudaErrorInvalidValue;
     DevArgs p;
     p.offsets = a.offsets;
@@ -940,7 +1079,9 @@ static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
     p.tile_ctr = a.tile_ctr;
     p.exit_ctr = a.exit_ctr;
     p.done1 = (p1 && p2) ? a.done1 : nullptr;
-    p.s1 = p1 ? gemm_split_factor(a.A, a.G, a.H, a.I, C::FP8) : 1;
+    p.s1 = p1 ? gemm_split_factor(a.A, a.G, a.H, a.I,
+                                  C::INT4 ? MOE_WDTYPE_INT4_G32 : (C::FP8 ? MOE_WDTYPE_FP8_E4M3_BLOCK128 : MOE_WDTYPE_BF16))
+              : 1;
     p.part = a.part;
     p.split_cnt = a.split_cnt;
     if (p.s1 > 1 && (!p.part || !p.split_cnt)) return cudaErrorInvalidValue;
@@ -969,11 +1110,12 @@ static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
     return launch_pdl(moe_gemm_kernel<C>, dim3(num_sms()), dim3(C::THREADS), smem, stream, tmW1, tmX, tmW2, tmH, p);
 }
 
-int gemm_pick_bn(int64_t A, int G, bool fp8) {
+int gemm_pick_bn(int64_t A, int G, int wdtype) {
     const double avg = G > 0 ? (double)A / (double)G : 0.0;
     int bn = 16;
     while (bn < 256 && bn < avg) bn <<= 1;  // smallest tile holding an average group
-    if (fp8 && bn > 64) bn = 64;  // FP8 keeps fp32 promotion registers for gate and up
+    if (wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128 && bn > 64) bn = 64;  // fp32 promotion registers for gate and up
+    if (wdtype == MOE_WDTYPE_INT4_G32 && bn > 128) bn = 128;  // the dequantisation warps need their threads
     return bn;
 }
 
@@ -987,9 +1129,10 @@ size_t gemm_block_flags_bytes(int64_t A, int G) {
 
 // Split GEMM1's K range when its tiles cannot fill two waves of the 148 SMs (decode-sized
 // batches), keeping at least two K blocks per split.
-int gemm_split_factor(int64_t A, int G, int H, int I, bool fp8) {
+int gemm_split_factor(int64_t A, int G, int H, int I, int wdtype) {
     constexpr int64_t kTarget = 2 * 148;
-    const int bn = gemm_pick_bn(A, G, fp8);
+    const bool fp8 = wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128;
+    const int bn = gemm_pick_bn(A, G, wdtype);
     const int64_t tiles = gemm_max_blocks(A, G, bn) * (I / 128);
     const int kb = H / (fp8 ? 128 : 64);
     if (fp8 && bn >= 64) return 1;  // the kernel variant has no split-K path
@@ -998,22 +1141,32 @@ int gemm_split_factor(int64_t A, int G, int H, int I, bool fp8) {
     return s;
 }
 
-size_t gemm_split_scratch_bytes(int64_t A, int G, int H, int I, bool fp8) {
-    const int s = gemm_split_factor(A, G, H, I, fp8);
+size_t gemm_split_scratch_bytes(int64_t A, int G, int H, int I, int wdtype) {
+    const int s = gemm_split_factor(A, G, H, I, wdtype);
     if (s == 1) return 0;
-    const int bn = gemm_pick_bn(A, G, fp8);
+    const int bn = gemm_pick_bn(A, G, wdtype);
     return (size_t)gemm_max_blocks(A, G, bn) * (I / 128) * s * 2 * bn * 128 * sizeof(float);
 }
 
-size_t gemm_split_counter_bytes(int64_t A, int G, int H, int I, bool fp8) {
-    if (gemm_split_factor(A, G, H, I, fp8) == 1) return 0;
-    const int bn = gemm_pick_bn(A, G, fp8);
+size_t gemm_split_counter_bytes(int64_t A, int G, int H, int I, int wdtype) {
+    if (gemm_split_factor(A, G, H, I, wdtype) == 1) return 0;
+    const int bn = gemm_pick_bn(A, G, wdtype);
     return (size_t)gemm_max_blocks(A, G, bn) * (I / 128) * sizeof(int);
 }
 
 cudaError_t launch_moe_gemm(const MoeGemmArgs& a, cudaStream_t stream) {
     if (a.A == 0 || a.G == 0 || (!a.run_gemm1 && !a.run_gemm2)) return cudaSuccess;
-    const int bn = gemm_pick_bn(a.A, a.G, a.fp8);
+    const int wdtype = a.int4 ? MOE_WDTYPE_INT4_G32 : (a.fp8 ? MOE_WDTYPE_FP8_E4M3_BLOCK128 : MOE_WDTYPE_BF16);
+    const int bn = gemm_pick_bn(a.A, a.G, wdtype);
+    if (a.int4) {
+        switch (bn) {
+            case 16: return launch_cfg<Cfg<16, false, true>>(a, stream);
+            case 32: return launch_cfg<Cfg<32, false, true>>(a, stream);
+            case 64: return launch_cfg<Cfg<64, false, true>>(a, stream);
+            case 128: return launch_cfg<Cfg<128, false, true>>(a, stream);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     if (a.fp8) {
         switch (bn) {
             case 16: return launch_cfg<Cfg<16, true>>(a, stream);

@@ -77,11 +77,12 @@ struct MoeGemmArgs {
     int64_t A;               // rows of x_perm / h / y
     int H, I;
     bool fp8;
+    bool int4;               // INT4 group-32 weights (bf16 activations)
     bool run_gemm1, run_gemm2;
     const void* x_perm;      // [A][H]
     const float* x_scale;    // FP8: [H/128][A]
     const void* w1;          // [G][2I][H]
-    const float* w1_scale;   // FP8: [G][2I/128][H/128]
+    const void* w1_scale;    // FP8: fp32 [G][2I/128][H/128]; INT4: bf16 [G][2I][H/32]
     const float* gate_scale; // [G] or NULL
     const float* up_scale;   // [G] or NULL
     float alpha, beta, limit;
@@ -89,7 +90,7 @@ struct MoeGemmArgs {
     void* h;                 // [A][I]
     float* h_scale;          // FP8: [I/128][A]
     const void* w2;          // [G][H][I]
-    const float* w2_scale;   // FP8: [G][H/128][I/128]
+    const void* w2_scale;    // FP8: fp32 [G][H/128][I/128]; INT4: bf16 [G][H][I/32]
     void* y;                 // [A][H] bf16
     unsigned int* tile_ctr;  // zero when idle; left at zero
     unsigned int* exit_ctr;  // zero when idle; left at zero
@@ -99,15 +100,15 @@ struct MoeGemmArgs {
     int* status;
 };
 
-int gemm_pick_bn(int64_t A, int G, bool fp8);
+int gemm_pick_bn(int64_t A, int G, int wdtype);
 // Upper bound on token blocks: every non-empty group adds at most one partial block.
 int64_t gemm_max_blocks(int64_t A, int G, int bn);
 size_t gemm_block_flags_bytes(int64_t A, int G);
-// GEMM1 split-K factor (1, 2 or 4) for these sizes, and the scratch it needs: fp32
+// Tile width, GEMM1 split-K factor (1, 2 or 4) for these sizes and weight format (moe_wdtype), and the scratch it needs: fp32
 // partials [tiles][splits][2][BN][128] plus one counter per GEMM1 tile.
-int gemm_split_factor(int64_t A, int G, int H, int I, bool fp8);
-size_t gemm_split_scratch_bytes(int64_t A, int G, int H, int I, bool fp8);
-size_t gemm_split_counter_bytes(int64_t A, int G, int H, int I, bool fp8);
+int gemm_split_factor(int64_t A, int G, int H, int I, int wdtype);
+size_t gemm_split_scratch_bytes(int64_t A, int G, int H, int I, int wdtype);
+size_t gemm_split_counter_bytes(int64_t A, int G, int H, int I, int wdtype);
 cudaError_t launch_moe_gemm(const MoeGemmArgs& a, cudaStream_t stream);
 
 int num_sms();

@@ -17,6 +17,9 @@ Workloads (synthetic stand-ins; no checkpoint or evaluation data is used):
   decode_t{1,8,64}  H=4096, I=1024, 256 routed + 2 sink-gated shared experts, top-8,
                 sigmoid+LSE with sinks, Zipf(1.2) expert popularity, row 0 all logits
                 below -104 with exact ties at the top-8 boundary (sglang PR #36385, item 2).
+  decode_t{1,64}_int4  the decode shapes with INT4 group-32 weights (batchgen PR #239 commit
+                notes: packed nibbles, one bf16 scale per 32 K); uniform nibbles and scales
+                drawn so that the weights' spread matches the bf16 workloads (std ~0.02).
 """
 from __future__ import annotations
 
@@ -27,6 +30,7 @@ import torch
 
 WDTYPE_BF16 = 0
 WDTYPE_FP8 = 1
+WDTYPE_INT4 = 2
 SCORE_SOFTMAX = 0
 SCORE_SIGMOID = 1
 
@@ -92,6 +96,10 @@ WORKLOADS = {
                           score=SCORE_SIGMOID, zipf_s=1.2, special_row=True),
     "decode_t64": Workload("decode_t64", T=64, H=4096, I=1024, E=256, k=8, n_sink=2, n_shared=2,
                            score=SCORE_SIGMOID, zipf_s=1.2, special_row=True),
+    "decode_t1_int4": Workload("decode_t1_int4", T=1, H=4096, I=1024, E=256, k=8, n_sink=2, n_shared=2,
+                               wdtype=WDTYPE_INT4, score=SCORE_SIGMOID, zipf_s=1.2, special_row=True),
+    "decode_t64_int4": Workload("decode_t64_int4", T=64, H=4096, I=1024, E=256, k=8, n_sink=2, n_shared=2,
+                                wdtype=WDTYPE_INT4, score=SCORE_SIGMOID, zipf_s=1.2, special_row=True),
 }
 
 
@@ -109,6 +117,17 @@ def fp8_block_quantize_weights(w: torch.Tensor):
     s = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
     q = (blk / s[..., :, None, :, None]).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
     return q.reshape(*lead, R, C).view(torch.uint8), s.to(torch.float32).contiguous()
+
+
+def random_int4_weights(gen, shape, device, std: float):
+    """Offline INT4 group-32 weight format (an input format, not a step of the layer):
+    uniform random bytes [.., R, C/2] (two nibbles each, low nibble = even column) and one
+    bf16 scale per row and 32 columns [.., R, C/32], drawn around std / 4.6 (the standard
+    deviation of nibble - 8 for uniform nibbles) so the weights have std close to `std`."""
+    *lead, R, C = shape
+    packed = torch.randint(0, 256, (*lead, R, C // 2), generator=gen, device=device, dtype=torch.int32)
+    scale = (std / 4.6) * (0.75 + 0.5 * torch.rand((*lead, R, C // 32), generator=gen, device=device))
+    return packed.to(torch.uint8).contiguous(), scale.to(torch.bfloat16).contiguous()
 
 
 def _special_row(gen, n_cols: int, k: int, device) -> torch.Tensor:
@@ -130,7 +149,8 @@ def make_inputs(wl: Workload, device="cpu", seed: int | None = None) -> dict:
     """Draw every input of one layer pass on `device` with a seeded torch generator.
 
     Returns torch tensors: x bf16 [T,H]; logits fp32 [T,E+n_sink]; w1 [G,2I,H] and
-    w2 [G,H,I] (bf16, or uint8 E4M3 codes with w1_scale/w2_scale fp32 block scales);
+    w2 [G,H,I] (bf16, or uint8 E4M3 codes with w1_scale/w2_scale fp32 block scales, or
+    INT4 packed bytes [G,2I,H/2] / [G,H,I/2] with bf16 group scales [G,2I,H/32] / [G,H,I/32]);
     gate_scale/up_scale fp32 [G] or None. Gate logits are x.W_r in fp64 rounded to fp32.
     """
     seed = wl.seed if seed is None else seed
@@ -164,6 +184,10 @@ def make_inputs(wl: Workload, device="cpu", seed: int | None = None) -> dict:
         if wl.wdtype == WDTYPE_FP8:
             q1, s1 = fp8_block_quantize_weights(w1)
             q2, s2 = fp8_block_quantize_weights(w2)
+            w1_parts.append(q1); w2_parts.append(q2); s1_parts.append(s1); s2_parts.append(s2)
+        elif wl.wdtype == WDTYPE_INT4:
+            q1, s1 = random_int4_weights(gen, (n, 2 * I, H), dev, wl.w_std * wl.gate_up_mult)
+            q2, s2 = random_int4_weights(gen, (n, H, I), dev, wl.w_std)
             w1_parts.append(q1); w2_parts.append(q2); s1_parts.append(s1); s2_parts.append(s2)
         else:
             w1_parts.append(w1.to(torch.bfloat16)); w2_parts.append(w2.to(torch.bfloat16))

@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 2
+#define MOE_ABI_VERSION 3
 
 typedef enum moe_status {
     MOE_OK = 0,
@@ -78,8 +78,11 @@ typedef enum moe_score_fn {
 
 typedef enum moe_wdtype {
     MOE_WDTYPE_BF16 = 0,             /* bf16 weights and activations                       */
-    MOE_WDTYPE_FP8_E4M3_BLOCK128 = 1 /* E4M3 weights with one fp32 scale per 128x128 block;
+    MOE_WDTYPE_FP8_E4M3_BLOCK128 = 1, /* E4M3 weights with one fp32 scale per 128x128 block;
                                         E4M3 activations with one fp32 scale per 1x128 block */
+    MOE_WDTYPE_INT4_G32 = 2          /* [P5] INT4 weights, two per byte (low nibble = even K),
+                                        one bf16 scale per 32 K per row, value
+                                        bf16((nibble - 8) * scale); bf16 activations       */
 } moe_wdtype;
 
 /* Problem statement. All fields are read on every call.
@@ -228,8 +231,10 @@ int moe_permute_noalloc(const int32_t* topk_ids, const void* x, const moe_dims* 
  *   h[r][i] = min(gate, L) * sigmoid(alpha * min(gate, L)) * (clamp(up, -L, L) + beta)
  * accumulated in fp32 (FP8: per 128-deep K block, times x_scale * w1_scale).
  *   x_perm, x_scale, offsets   as written by moe_permute (A = offsets[G]).
- *   w1        [G][2I][H]: rows [0, I) gate, [I, 2I) up; bf16 or E4M3.
- *   w1_scale  [G][2I/128][H/128] fp32 (FP8 only, else NULL).
+ *   w1        [G][2I][H]: rows [0, I) gate, [I, 2I) up; bf16 or E4M3, or for INT4 [G][2I][H/2]
+ *             packed bytes (16-byte aligned).
+ *   w1_scale  FP8: fp32 [G][2I/128][H/128]; INT4: bf16 [G][2I][H/32] (4-byte aligned);
+ *             else NULL.
  *   gate_scale, up_scale  [G] fp32 per-group scales, or NULL for 1.0.
  *   limits    [G] fp32 clamp L per group ([P2'] one value per expert), or NULL for
  *             dims->limit. Each value > 0; +INFINITY disables that group's clamp.
@@ -237,7 +242,7 @@ int moe_permute_noalloc(const int32_t* topk_ids, const void* x, const moe_dims* 
  *   h_scale   [I/128][A] fp32 out (FP8 only, else NULL).
  * Errors: INVALID_ARG, WORKSPACE, ARCH, CUDA; TIMEOUT in the status word. */
 int moe_gemm1_swiglu(const void* x_perm, const float* x_scale, const int32_t* offsets,
-                     const void* w1, const float* w1_scale, const float* gate_scale,
+                     const void* w1, const void* w1_scale, const float* gate_scale,
                      const float* up_scale, const float* limits, const moe_dims* dims, void* h,
                      float* h_scale, void* ws, size_t ws_bytes, void* stream);
 
@@ -250,12 +255,13 @@ int moe_gemm1_swiglu(const void* x_perm, const float* x_scale, const int32_t* of
  * summed in fp32 in that fixed order and rounded once to bf16.
  *   h, h_scale, offsets  as written by moe_gemm1_swiglu / moe_permute.
  *   inv_perm [T][k], topk_w [T][k], shared_w [T][n_sink] (NULL iff n_sink == 0).
- *   w2       [G][H][I] bf16 or E4M3; w2_scale [G][H/128][I/128] fp32 (FP8 only).
+ *   w2       [G][H][I] bf16 or E4M3, or INT4 [G][H][I/2] packed bytes; w2_scale FP8: fp32
+ *            [G][H/128][I/128], INT4: bf16 [G][H][I/32]; else NULL.
  *   out      [T][H] bf16 out.
  * Errors: INVALID_ARG, WORKSPACE, ARCH, CUDA; TIMEOUT in the status word. */
 int moe_gemm2_combine(const void* h, const float* h_scale, const int32_t* offsets,
                       const int32_t* inv_perm, const float* topk_w, const float* shared_w,
-                      const void* w2, const float* w2_scale, const moe_dims* dims,
+                      const void* w2, const void* w2_scale, const moe_dims* dims,
                       void* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Both grouped GEMMs in one persistent launch (the expert MLPs of every group):
@@ -270,8 +276,8 @@ int moe_gemm2_combine(const void* h, const float* h_scale, const int32_t* offset
  *   after allocating it; every call leaves the flags at zero.
  * Errors: INVALID_ARG, WORKSPACE, ARCH, CUDA; TIMEOUT / EXPERT_ID in the status word. */
 int moe_experts(const void* x_perm, const float* x_scale, const int32_t* offsets, const void* w1,
-                const float* w1_scale, const float* gate_scale, const float* up_scale,
-                const float* limits, const void* w2, const float* w2_scale, const moe_dims* dims,
+                const void* w1_scale, const float* gate_scale, const float* up_scale,
+                const float* limits, const void* w2, const void* w2_scale, const moe_dims* dims,
                 void* h, float* h_scale, void* y, void* ws, size_t ws_bytes, void* stream);
 
 /* The routing-weighted combine alone ([P5] slot-specific weighted reduction):
@@ -296,8 +302,8 @@ int moe_combine(const void* y, const int32_t* offsets, const int32_t* inv_perm,
  *   [T][k]); pass NULL to keep the first three in the workspace and skip `packed`.
  * Errors: as the four calls. */
 int moe_forward(const float* logits, const float* bias, const void* x, const void* w1,
-                const float* w1_scale, const float* gate_scale, const float* up_scale,
-                const float* limits, const void* w2, const float* w2_scale, const moe_dims* dims,
+                const void* w1_scale, const float* gate_scale, const float* up_scale,
+                const float* limits, const void* w2, const void* w2_scale, const moe_dims* dims,
                 void* out, int32_t* topk_ids, float* topk_w, float* shared_w, uint32_t* packed,
                 void* ws, size_t ws_bytes, void* stream);
 

@@ -26,7 +26,7 @@ def test_every_header_function_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert moe.moe_abi_version() == 2
+    assert moe.moe_abi_version() == 3
     for code in range(-7, 1):
         assert moe.status_string(code)
     assert "unknown" in moe.status_string(-99)

@@ -12,7 +12,7 @@ from helpers import assert_bf16_close, assert_fp8_close, f32, oracle_layer, samp
 
 pytestmark = pytest.mark.gpu
 
-FULL = ["tiny", "oai_swiglu", "decode_t1", "decode_t8", "decode_t64"]
+FULL = ["tiny", "oai_swiglu", "decode_t1", "decode_t8", "decode_t64", "decode_t1_int4", "decode_t64_int4"]
 SAMPLED = {"qwen3_30b_a3b": 48, "glm_fp8": 24}
 
 

@@ -15,7 +15,8 @@ from helpers import assert_bf16_close, assert_fp8_close, bits16, e4m3_to_np, f32
 pytestmark = pytest.mark.gpu
 
 
-def make_case(T, E, k, S, H, I, fp8, seed, gate_up_mult=1.0, scales=False, sinks=False, skew=0.0, limits=False):
+def make_case(T, E, k, S, H, I, fp8, seed, gate_up_mult=1.0, scales=False, sinks=False, skew=0.0, limits=False,
+              int4=False):
     ids = W.random_topk_ids(T, E, k, seed=seed, skew=skew)
     offsets, perm, inv = oracle.permute(ids.numpy(), E, S)
     A = T * (k + S)
@@ -25,8 +26,14 @@ def make_case(T, E, k, S, H, I, fp8, seed, gate_up_mult=1.0, scales=False, sinks
     w2f = torch.randn((G, H, I), generator=g, device="cuda") * 0.02
     xf = torch.randn((A, H), generator=g, device="cuda")
     hf = torch.randn((A, I), generator=g, device="cuda")
-    c = dict(T=T, E=E, k=k, S=S, H=H, I=I, A=A, G=G, fp8=fp8, ids=ids, offsets=offsets, perm=perm, inv=inv)
-    if fp8:
+    c = dict(T=T, E=E, k=k, S=S, H=H, I=I, A=A, G=G, fp8=fp8, int4=int4, ids=ids, offsets=offsets, perm=perm,
+             inv=inv)
+    if int4:  # INT4 group-32 weights, bf16 activations
+        c["w1"], c["w1_scale"] = W.random_int4_weights(g, (G, 2 * I, H), "cuda", 0.02 * gate_up_mult)
+        c["w2"], c["w2_scale"] = W.random_int4_weights(g, (G, H, I), "cuda", 0.02)
+        c["xs"] = c["hs"] = None
+        c["xp"], c["hp"] = xf.to(torch.bfloat16), hf.to(torch.bfloat16)
+    elif fp8:
         c["w1"], c["w1_scale"] = W.fp8_block_quantize_weights(w1f)
         c["w2"], c["w2_scale"] = W.fp8_block_quantize_weights(w2f)
         q, s = oracle.quant_1x128(xf.cpu().numpy())
@@ -52,12 +59,20 @@ def make_case(T, E, k, S, H, I, fp8, seed, gate_up_mult=1.0, scales=False, sinks
 
 def dims_of(c, alpha=1.0, beta=0.0, limit=math.inf):
     return moe.MoeDims(T=c["T"], H=c["H"], I=c["I"], E=c["E"], k=c["k"], n_sink=c["S"] if c["shared_w"] is not None else 0,
-                       n_shared=c["S"], wdtype=1 if c["fp8"] else 0, score=1, alpha=alpha, beta=beta,
+                       n_shared=c["S"], wdtype=2 if c.get("int4") else (1 if c["fp8"] else 0), score=1, alpha=alpha,
+                       beta=beta,
                        limit=limit, route_scale=1.0)
 
 
 def oracle_of(c, d):
     fp8 = c["fp8"]
+    if c.get("int4"):
+        return oracle.Layer(T=c["T"], H=c["H"], I=c["I"], E=c["E"], k=c["k"], n_sink=d.n_sink, n_shared=c["S"],
+                            wdtype=oracle.WDTYPE_INT4, score=1, alpha=d.alpha, beta=d.beta, limit=d.limit,
+                            route_scale=1.0, logits=np.zeros((c["T"], c["E"] + d.n_sink), np.float32),
+                            x=np.zeros((c["T"], c["H"]), np.uint16), w1=u8(c["w1"]), w2=u8(c["w2"]),
+                            w1_scale=bits16(c["w1_scale"]), w2_scale=bits16(c["w2_scale"]),
+                            gate_scale=f32(c["gate_scale"]), up_scale=f32(c["up_scale"]), limits=f32(c.get("limits")))
     return oracle.Layer(T=c["T"], H=c["H"], I=c["I"], E=c["E"], k=c["k"], n_sink=d.n_sink, n_shared=c["S"],
                         wdtype=1 if fp8 else 0, score=1, alpha=d.alpha, beta=d.beta, limit=d.limit,
                         route_scale=1.0, logits=np.zeros((c["T"], c["E"] + d.n_sink), np.float32),
@@ -82,6 +97,10 @@ GEMM1_CASES = [
     (200, 8, 2, 0, 1024, 512, True, {"oai": True, "scales": True}),
     (128, 8, 2, 1, 512, 384, False, {"limits": True}),          # a clamp per expert (shared group too)
     (300, 16, 4, 0, 512, 256, True, {"limits": True, "scales": True}),  # FP8, tile 32, clamp per expert
+    (8, 64, 4, 0, 256, 256, False, {"int4": True}),            # INT4 group-32 weights: tile 16, split-K
+    (64, 16, 4, 0, 512, 256, False, {"int4": True}),           # INT4, tile 32
+    (300, 16, 4, 1, 512, 384, False, {"int4": True, "oai": True, "scales": True}),  # INT4, shared group
+    (512, 8, 2, 0, 512, 256, False, {"int4": True, "skew": 3.0, "limits": True}),   # INT4, tile 128
 ]
 
 
@@ -89,7 +108,8 @@ GEMM1_CASES = [
 def test_gemm1_swiglu(T, E, k, S, H, I, fp8, extra):
     oai, glm = extra.get("oai", False), extra.get("glm", False)
     c = make_case(T, E, k, S, H, I, fp8, seed=T + E + H, gate_up_mult=4.0 if oai else 1.0,
-                  scales=extra.get("scales", False), skew=extra.get("skew", 0.0), limits=extra.get("limits", False))
+                  scales=extra.get("scales", False), skew=extra.get("skew", 0.0), limits=extra.get("limits", False),
+                  int4=extra.get("int4", False))
     d = dims_of(c, alpha=1.702 if oai else 1.0, beta=1.0 if oai else 0.0,
                 limit=7.0 if oai else (10.0 if glm else math.inf))
     A = c["A"]
@@ -127,12 +147,17 @@ GEMM2_CASES = [
     (600, 4, 2, 1, 384, 256, False, True),      # tile 256, odd number of 128-row chunks of H
     (512, 8, 2, 0, 512, 256, True, False),
     (40, 32, 4, 1, 512, 256, True, False),
+    (8, 64, 4, 0, 256, 256, "int4", False),     # INT4 weights, tile 16
+    (300, 16, 4, 2, 512, 256, "int4", True),    # INT4, sink-gated shared groups
+    (512, 8, 2, 0, 384, 256, "int4", False),    # INT4, tile 128, odd chunk count of H
 ]
 
 
 @pytest.mark.parametrize("T,E,k,S,H,I,fp8,sinks", GEMM2_CASES)
 def test_gemm2_combine(T, E, k, S, H, I, fp8, sinks):
-    c = make_case(T, E, k, S, H, I, fp8, seed=3 * T + E, sinks=sinks)
+    int4 = fp8 == "int4"
+    fp8 = fp8 is True
+    c = make_case(T, E, k, S, H, I, fp8, seed=3 * T + E, sinks=sinks, int4=int4)
     d = dims_of(c)
     out = torch.zeros((T, H), dtype=torch.bfloat16, device="cuda")
     ws = moe.alloc_workspace(d, moe.MOE_WS_GEMM2_COMBINE)
