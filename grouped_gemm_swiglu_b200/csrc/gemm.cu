@@ -58,17 +58,21 @@ template <int BN_, bool FP8_, bool INT4_ = false>
 struct Cfg {
     static constexpr int BN = BN_;
     static constexpr bool FP8 = FP8_;
-    // INT4 group-32 weights: TMA brings the packed bytes (RAW_BYTES per 128x64 block),
-    // dequantisation warps write the bf16 tiles the MMA reads; everything else is bf16.
+    // INT4 group-32 weights: TMA brings the packed bytes (RAW_BYTES per 128x64 block) and
+    // dequantisation warps write the bf16 weight tiles into tensor memory, where the MMA
+    // takes its A operand; shared memory then holds only the token tile and packed bytes.
     static constexpr bool INT4 = INT4_;
     static constexpr int BK = FP8 ? 128 : 64;  // K elements per stage: one 128-byte row
     static constexpr int A_BYTES = 128 * 128;
     static constexpr int B_BYTES = BN * 128;
     static constexpr int RAW_BYTES = INT4 ? 128 * 32 : 0;
-    static constexpr int RAW_OFF = 2 * A_BYTES + B_BYTES;  // packed A0, A1 after the bf16 tiles and B
-    static constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES + 2 * RAW_BYTES;  // sized for GEMM1 (gate + up)
+    static constexpr int B_OFF = INT4 ? 0 : 2 * A_BYTES;  // token tile within a stage
+    static constexpr int RAW_OFF = B_OFF + B_BYTES;        // INT4: packed A0, A1 after the token tile
+    static constexpr int STAGE_BYTES = INT4 ? B_BYTES + 2 * RAW_BYTES : 2 * A_BYTES + B_BYTES;  // GEMM1-sized
+    static constexpr int A_TMEM_COLS = 64;  // INT4: one stage's bf16 A0 | A1 (128 x 64 K, two K per column)
     // Dequantisation warps: 8 for decode-sized tiles (one weight row of one of the two tiles
     // per thread, the epilogue then has 4 warps), else 4 (one row of both tiles per thread).
+    // A warp may only touch its TMEM lane quarter (warp % 4): its rows follow that quarter.
     static constexpr int DQ = INT4 ? (BN <= 32 ? 8 : 4) : 0;
     // Token rows arrive in boxes of up to 64 rows, and only the boxes a tile's rows reach
     // are loaded, so a short token block does not pull a full BN-row tile through L2.
@@ -76,15 +80,18 @@ struct Cfg {
     static constexpr int BOX_BYTES = BOX_ROWS * 128;
     // as many stages as fit next to the control block and the largest group table
     static constexpr int STAGE_BUDGET = kSmemLimit - 1024 - 8 * (kMaxGroupsGemm + 1) - 1024 - 4 * 16 * 16 * 3;
-    static constexpr int STAGES_RAW = STAGE_BUDGET / STAGE_BYTES;
-    static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
     static constexpr int ACC_COLS = 2 * BN;  // one TMEM buffer: gate | up (GEMM2 uses the first BN)
     // bf16 hands one buffer per tile to the epilogue, FP8 one per 128-deep K block, so
     // FP8 keeps up to four partial buffers in flight.
     // At 256 token columns gate | up fill all 512 TMEM columns: one buffer, and the TMA
     // ring keeps streaming the next tile while the epilogue drains it.
     static constexpr int NBUF = (FP8 && 4 * ACC_COLS <= 512) ? 4 : (2 * ACC_COLS <= 512 ? 2 : 1);
-    static constexpr int TMEM_COLS = pow2_at_least(NBUF * ACC_COLS);
+    static constexpr int STAGES_SMEM = STAGE_BUDGET / STAGE_BYTES;
+    static constexpr int STAGES_TMEM = INT4 ? (512 - NBUF * ACC_COLS) / A_TMEM_COLS : 8;  // INT4: A tiles in TMEM
+    static constexpr int STAGES_RAW = STAGES_SMEM < STAGES_TMEM ? STAGES_SMEM : STAGES_TMEM;
+    static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+    static constexpr int A_TMEM = NBUF * ACC_COLS;  // INT4: first TMEM column of the A tiles
+    static constexpr int TMEM_COLS = pow2_at_least(NBUF * ACC_COLS + (INT4 ? STAGES * A_TMEM_COLS : 0));
     // Epilogue warps: groups of four (one warp per TMEM lane quarter), each group owning
     // an equal share of the tile's columns; four groups at 256 columns, whose single
     // accumulator buffer makes the drain time part of the tile time.
@@ -103,6 +110,7 @@ struct Cfg {
     static_assert(BN % BOX_ROWS == 0 && BN <= 256, "token tile = whole boxes, at most the MMA's N limit");
     static_assert(STAGES >= 2, "at least two pipeline stages");
     static_assert(!(INT4 && FP8), "INT4 weights take bf16 activations");
+    static_assert(!INT4 || BN <= 64, "INT4 keeps its A tiles next to the accumulators in TMEM");
     static_assert(COLS % 8 == 0, "split-K merges columns in chunks of 8");
     // Split-K of GEMM1 is compiled in where it can be chosen (see gemm_split_factor):
     // every tile width except FP8 at 64 columns, whose promotion registers are full.
@@ -272,26 +280,22 @@ __device__ __forceinline__ uint32_t int4_pair_bf16(uint32_t lo, uint32_t hi, int
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-__device__ __forceinline__ void dequant_int4_row(const uint8_t* raw, uint32_t sc, uint8_t* dst, int r) {
+// out[j] = the bf16 pair (K 2j, 2j+1) of the row segment, j < 32, in TMEM column order.
+__device__ __forceinline__ void dequant_int4_row(const uint8_t* raw, uint32_t sc, uint32_t* out) {
     __nv_bfloat162 s[2];
     s[0] = __halves2bfloat162(__ushort_as_bfloat16((unsigned short)(sc & 0xFFFFu)),
                               __ushort_as_bfloat16((unsigned short)(sc & 0xFFFFu)));
     s[1] = __halves2bfloat162(__ushort_as_bfloat16((unsigned short)(sc >> 16)),
                               __ushort_as_bfloat16((unsigned short)(sc >> 16)));
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
+    for (int half = 0; half < 2; ++half) {  // K 0-31 (scale 0) and 32-63 (scale 1)
         const uint4 q = *reinterpret_cast<const uint4*>(raw + 16 * half);
         const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {  // 16-byte chunk (8 K elements) 4*half + c of the row
+        for (int c = 0; c < 4; ++c) {
             const uint32_t lo = qw[c] & 0x0F0F0F0Fu, hi = (qw[c] >> 4) & 0x0F0F0F0Fu;
-            uint4 o;
-            o.x = int4_pair_bf16(lo, hi, 0, s[half]);
-            o.y = int4_pair_bf16(lo, hi, 1, s[half]);
-            o.z = int4_pair_bf16(lo, hi, 2, s[half]);
-            o.w = int4_pair_bf16(lo, hi, 3, s[half]);
-            const int chunk = (4 * half + c) ^ (r & 7);  // 128-byte swizzle: chunk XOR row mod 8
-            *reinterpret_cast<uint4*>(dst + chunk * 16) = o;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) out[16 * half + 4 * c + b] = int4_pair_bf16(lo, hi, b, s[half]);
         }
     }
 }
@@ -429,7 +433,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const uint32_t tx = (tl.dual ? 2 : 1) * (C::INT4 ? C::RAW_BYTES : C::A_BYTES) + n_box * C::BOX_BYTES;
                 auto load_act = [&](uint8_t* st, uint64_t* bar, int kx) {
                     for (int r = 0; r < n_box; ++r)
-                        tma_load_2d(st + 2 * C::A_BYTES + r * C::BOX_BYTES, ta, bar, kx, tl.row0 + r * C::BOX_ROWS);
+                        tma_load_2d(st + C::B_OFF + r * C::BOX_BYTES, ta, bar, kx, tl.row0 + r * C::BOX_ROWS);
                 };
                 // GEMM2 after GEMM1 in the same launch: weights of the first stages go out
                 // before waiting for the block's h rows.
@@ -522,12 +526,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         }
                         tc_fence_after();
                         const uint32_t a0 = smem_u32(smem + (size_t)stage * C::STAGE_BYTES);
-                        const uint32_t b0 = a0 + 2 * C::A_BYTES;
+                        const uint32_t b0 = a0 + C::B_OFF;
+                        const uint32_t at = tmem_base + C::A_TMEM + stage * C::A_TMEM_COLS;  // INT4 A tiles
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             const uint64_t bd = smem_desc_sw128(b0 + kk * 32);
                             const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-                            if constexpr (C::FP8) {
+                            if constexpr (C::INT4) {
+                                mma_bf16_tmem_a(d0, at + kk * 8, bd, idesc, acc);
+                                if (tl.dual) mma_bf16_tmem_a(d0 + C::BN, at + 32 + kk * 8, bd, idesc, acc);
+                            } else if constexpr (C::FP8) {
                                 mma_fp8(d0, smem_desc_sw128(a0 + kk * 32), bd, idesc, acc);
                                 if (tl.dual)
                                     mma_fp8(d0 + C::BN, smem_desc_sw128(a0 + C::A_BYTES + kk * 32), bd, idesc, acc);
@@ -555,12 +563,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         __syncwarp();
     } else if (C::INT4 && warp >= 2 + C::EPI) {
         // ------------------------------------------------------------ INT4 dequantisation
-        // Thread dt converts weight row r = dt % 128 of tile dt / 128 (A0, A1; with 4 warps
-        // both tiles) of every stage, in the same tile order as the MMA, then the warp
-        // completes the stage's `full` barrier.
-        const int dt = (warp - 2 - C::EPI) * 32 + lane;
-        const int r = dt % 128;
+        // Each warp converts the 32 weight rows of its TMEM lane quarter (warp % 4) of one
+        // tile (A0 or A1; with 4 warps both tiles) of every stage, in the same tile order as
+        // the MMA, stores them into the stage's TMEM A columns and completes `full`.
+        const int r = (warp & 3) * 32 + lane;
+        const int dt = ((warp - 2 - C::EPI) / 4) * 128 + r;  // tile = dt / 128
         constexpr int kTileStep = C::DQ * 32 / 128;  // tiles apart that one thread converts
+        const uint32_t lane_sel = (uint32_t)((warp & 3) * 32) << 16;
         uint32_t stage = 0, phase = 0;
         bool ok = true;
         for (int i = 0; ok; ++i) {
@@ -594,9 +603,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     break;
                 }
                 uint8_t* st = smem + (size_t)stage * C::STAGE_BYTES;
-                if (has0) dequant_int4_row(st + C::RAW_OFF + t0 * C::RAW_BYTES + r * 32, s0, st + t0 * C::A_BYTES + r * 128, r);
-                if (has1) dequant_int4_row(st + C::RAW_OFF + C::RAW_BYTES + r * 32, s1, st + C::A_BYTES + r * 128, r);
-                fence_proxy_async_smem();  // these generic writes are read by the MMA (async proxy)
+                const uint32_t at = tmem_base + lane_sel + C::A_TMEM + stage * C::A_TMEM_COLS;
+                uint32_t w[32];
+                if (has0) {  // warp-uniform: every lane of the warp works on the same tile
+                    dequant_int4_row(st + C::RAW_OFF + t0 * C::RAW_BYTES + r * 32, s0, w);
+                    tmem_st32(at + t0 * 32, w);
+                }
+                if (has1) {
+                    dequant_int4_row(st + C::RAW_OFF + C::RAW_BYTES + r * 32, s1, w);
+                    tmem_st32(at + 32, w);
+                }
+                tc_fence_before();  // the tensor-memory stores happen before the MMA that reads them
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[stage]);
                 if (++stage == (uint32_t)C::STAGES) {
@@ -1115,7 +1132,7 @@ int gemm_pick_bn(int64_t A, int G, int wdtype) {
     int bn = 16;
     while (bn < 256 && bn < avg) bn <<= 1;  // smallest tile holding an average group
     if (wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128 && bn > 64) bn = 64;  // fp32 promotion registers for gate and up
-    if (wdtype == MOE_WDTYPE_INT4_G32 && bn > 128) bn = 128;  // the dequantisation warps need their threads
+    if (wdtype == MOE_WDTYPE_INT4_G32 && bn > 64) bn = 64;  // A tiles share TMEM with the accumulators
     return bn;
 }
 
@@ -1163,7 +1180,6 @@ cudaError_t launch_moe_gemm(const MoeGemmArgs& a, cudaStream_t stream) {
             case 16: return launch_cfg<Cfg<16, false, true>>(a, stream);
             case 32: return launch_cfg<Cfg<32, false, true>>(a, stream);
             case 64: return launch_cfg<Cfg<64, false, true>>(a, stream);
-            case 128: return launch_cfg<Cfg<128, false, true>>(a, stream);
             default: return cudaErrorInvalidValue;
         }
     }
