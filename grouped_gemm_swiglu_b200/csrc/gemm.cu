@@ -30,7 +30,9 @@
 //
 // Roles (320 threads): warp 0 lane 0 issues TMA loads into a STAGES-deep ring; warp 1
 // owns TMEM and lane 0 issues tcgen05.mma; warps 2..9 are the epilogue (warp w reads
-// TMEM lanes 32*(w%4).., and columns of half (w-2)/4 of the tile). Every wait is bounded
+// TMEM lanes 32*(w%4).., and columns of half (w-2)/4 of the tile). FP8 tiles of 128
+// token columns launch 384 threads: warps 2-3 are spares whose registers go to the
+// epilogue, warps 4..11 are the epilogue. Every wait is bounded
 // (ptx.cuh): on timeout the CTA sets MOE_ERR_TIMEOUT, drains its outstanding copies and
 // MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -96,17 +98,27 @@ struct Cfg {
     // an equal share of the tile's columns; four groups at 256 columns, whose single
     // accumulator buffer makes the drain time part of the tile time.
     static constexpr int EPI = BN >= 256 ? 16 : ((INT4 && BN <= 32) ? 4 : 8);
-    static constexpr int THREADS = 64 + 32 * EPI + 32 * DQ;
+    // FP8 at 128 token columns: the promoted gate and up sums of a 128 x 128 tile take 128
+    // registers per epilogue thread. Two spare warps make warps 0-3 (producer, MMA, spares)
+    // one warpgroup, which gives registers back (setmaxnreg) to the two epilogue warpgroups:
+    // 384 threads launch with 168 registers; 4 warps drop to REG_LOW, 8 rise to REG_HIGH.
+    static constexpr bool WIDE = FP8 && BN >= 128;
+    static constexpr int EPI0 = WIDE ? 4 : 2;  // first epilogue warp
+    static constexpr int REG_LOW = 56, REG_HIGH = 224;
+    static constexpr int THREADS = 32 * EPI0 + 32 * EPI + 32 * DQ;
     static constexpr int GROUPS = EPI / 4;
     static constexpr int COLS = BN / GROUPS;  // columns per epilogue warp
     static constexpr int CW = COLS < 16 ? COLS : 16;  // TMEM load width (columns)
     static constexpr int RED_FLOATS = FP8 ? EPI * COLS : 4;
     // FP8: per epilogue warp, the two rows of scale products (A0, A1) of its columns
-    static constexpr int SCT_FLOATS = FP8 ? EPI * 2 * COLS : 4;
+    static constexpr int SCT_FLOATS = (FP8 && !WIDE) ? EPI * 2 * COLS : 4;
     static_assert(STAGE_BYTES % 1024 == 0, "stage tiles must stay 1024-byte aligned");
     static_assert(TMEM_COLS <= 512, "TMEM holds 512 columns");
     static_assert(COLS % CW == 0 && CW >= 4, "column share must be a multiple of the load width");
-    static_assert(!FP8 || COLS <= 32, "FP8 loads a warp's whole column share at once");
+    static_assert(!FP8 || WIDE || COLS <= 32, "FP8 loads a warp's whole column share at once");
+    static_assert(!WIDE || (BN == 128 && EPI == 8 && THREADS == 384 &&
+                            128 * REG_LOW + 256 * REG_HIGH <= THREADS * 168),
+                  "register split of the wide FP8 tile");
     static_assert(BN % BOX_ROWS == 0 && BN <= 256, "token tile = whole boxes, at most the MMA's N limit");
     static_assert(STAGES >= 2, "at least two pipeline stages");
     static_assert(!(INT4 && FP8), "INT4 weights take bf16 activations");
@@ -399,175 +411,185 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int total = T1 + nblk * p.c2;
     const bool chained = p.done1 != nullptr && p.c1 > 0 && p.c2 > 0;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            tma_prefetch_desc(&tmW1);
-            tma_prefetch_desc(&tmX);
-            tma_prefetch_desc(&tmW2);
-            tma_prefetch_desc(&tmH);
-            uint32_t stage = 0, phase = 0, pend_mask = 0, pend_phase = 0;
-            bool ok = true;
-            // Tiles are claimed one ahead, so the atomic's latency overlaps the current tile.
-            auto claim = [&](int i) -> int {
-                return p.tile_ctr ? (int)atomicAdd(p.tile_ctr, 1u) : (int)blockIdx.x + i * (int)gridDim.x;
-            };
-            int next_L = claim(0);
-            for (int i = 0; ok; ++i) {
-                const int slot = i % kRing;
-                int L = next_L;
-                if (L >= total) L = -1;
-                else next_L = claim(i + 1);
-                if (!mbar_wait(&ring_empty[slot], ((i / kRing) & 1) ^ 1, ab, p.status)) break;
-                ring[slot] = L;
-                mbar_arrive(&ring_full[slot]);
-                if (L < 0) break;
-                const Tile tl = decode_tile<C::BN>(L, T1, blk_start, s_off, p);
-                const bool g1 = tl.phase == 1;
-                const CUtensorMap* tw = g1 ? &tmW1 : &tmW2;
-                const CUtensorMap* ta = g1 ? &tmX : &tmH;
-                const int all_kb = (g1 ? p.H : p.I) / C::BK;
-                const int kbase = g1 ? tl.ks * all_kb / p.s1 : 0;  // this tile's K blocks
-                const int num_kb = g1 ? (tl.ks + 1) * all_kb / p.s1 - kbase : all_kb;
-                const int n_box = (max(16, (tl.nrows + 15) & ~15) + C::BOX_ROWS - 1) / C::BOX_ROWS;
-                const uint32_t tx = (tl.dual ? 2 : 1) * (C::INT4 ? C::RAW_BYTES : C::A_BYTES) + n_box * C::BOX_BYTES;
-                auto load_act = [&](uint8_t* st, uint64_t* bar, int kx) {
-                    for (int r = 0; r < n_box; ++r)
-                        tma_load_2d(st + C::B_OFF + r * C::BOX_BYTES, ta, bar, kx, tl.row0 + r * C::BOX_ROWS);
+    // Register split of the wide FP8 tile (warpgroup-uniform, at the top of each role so
+    // the compiler allocates each role within its own limit): warps 0-3 (producer, MMA,
+    // spares) give, the epilogue warps take.
+    if (warp < C::EPI0) {
+        if constexpr (C::WIDE) setmaxnreg_dec<C::REG_LOW>();
+        if (warp == 0) {
+            // ------------------------------------------------------------ TMA producer
+            if (lane == 0) {
+                tma_prefetch_desc(&tmW1);
+                tma_prefetch_desc(&tmX);
+                tma_prefetch_desc(&tmW2);
+                tma_prefetch_desc(&tmH);
+                uint32_t stage = 0, phase = 0, pend_mask = 0, pend_phase = 0;
+                bool ok = true;
+                // Tiles are claimed one ahead, so the atomic's latency overlaps the current tile.
+                auto claim = [&](int i) -> int {
+                    return p.tile_ctr ? (int)atomicAdd(p.tile_ctr, 1u) : (int)blockIdx.x + i * (int)gridDim.x;
                 };
-                // GEMM2 after GEMM1 in the same launch: weights of the first stages go out
-                // before waiting for the block's h rows.
-                const bool dep = chained && !g1;
-                const int pre = dep ? min(num_kb, C::STAGES) : 0;
-                const uint32_t st0 = stage;
-                // Wait for the block's h rows, then load the activation rows of the
-                // prefetched stages. They are loaded even when the wait gave up (the rows
-                // are in bounds; the results are discarded), so every armed stage completes.
-                auto release_prefetched = [&]() -> bool {
-                    const bool dep_ok = wait_counter_geq(p.done1 + tl.blk, p.c1, ab, p.status);
-                    uint32_t s2 = st0;
-                    for (int k2 = 0; k2 < pre; ++k2) {
-                        load_act(smem + (size_t)s2 * C::STAGE_BYTES, C::INT4 ? &raw_full[s2] : &full[s2],
-                                 (kbase + k2) * C::BK);
-                        if (++s2 == (uint32_t)C::STAGES) s2 = 0;
-                    }
-                    return dep_ok;
-                };
-                for (int kb = 0; kb < num_kb && ok; ++kb) {
-                    if (kb == pre && dep && !release_prefetched()) {
-                        ok = false;
-                        break;
-                    }
-                    if (!mbar_wait(&empty[stage], phase ^ 1, ab, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t* st = smem + (size_t)stage * C::STAGE_BYTES;
-                    uint64_t* bar = C::INT4 ? &raw_full[stage] : &full[stage];
-                    mbar_arrive_expect_tx(bar, tx);
-                    const int kx = (kbase + kb) * C::BK;
-                    if constexpr (C::INT4) {  // packed weight bytes: x is a byte offset (2 K per byte)
-                        tma_load_2d(st + C::RAW_OFF, tw, bar, kx / 2, tl.a0row);
-                        if (tl.dual) tma_load_2d(st + C::RAW_OFF + C::RAW_BYTES, tw, bar, kx / 2, tl.a1row);
-                    } else {
-                        tma_load_2d(st, tw, bar, kx, tl.a0row);
-                        if (tl.dual) tma_load_2d(st + C::A_BYTES, tw, bar, kx, tl.a1row);
-                    }
-                    if (kb >= pre) load_act(st, bar, kx);
-                    pend_mask |= 1u << stage;
-                    pend_phase = (pend_phase & ~(1u << stage)) | (phase << stage);
-                    if (++stage == (uint32_t)C::STAGES) {
-                        stage = 0;
-                        phase ^= 1;
-                    }
-                }
-                if (ok && dep && pre == num_kb && !release_prefetched()) ok = false;  // whole K prefetched
-            }
-            // Never leave with a copy in flight: wait for the last fill of every stage.
-            for (int s = 0; s < C::STAGES; ++s)
-                if ((pend_mask >> s) & 1u)
-                    mbar_wait_drain(C::INT4 ? &raw_full[s] : &full[s], (pend_phase >> s) & 1u);
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            uint32_t stage = 0, phase = 0, it = 0;
-            bool ok = true;
-            for (int i = 0; ok; ++i) {
-                const int slot = i % kRing;
-                if (!mbar_wait(&ring_full[slot], (i / kRing) & 1, ab, p.status)) break;
-                const int L = ring[slot];
-                mbar_arrive(&ring_empty[slot]);
-                if (L < 0) break;
-                const Tile tl = decode_tile<C::BN>(L, T1, blk_start, s_off, p);
-                const bool g1 = tl.phase == 1;
-                const int all_kb = (g1 ? p.H : p.I) / C::BK;
-                const int kbase = g1 ? tl.ks * all_kb / p.s1 : 0;
-                const int num_kb = g1 ? (tl.ks + 1) * all_kb / p.s1 - kbase : all_kb;
-                const int n_mma = max(16, (tl.nrows + 15) & ~15);
-                const uint32_t idesc = idesc_m128(n_mma, C::FP8);
-                // bf16: one TMEM buffer per tile; FP8: one per 128-deep K block
-                const int units = C::FP8 ? num_kb : 1;
-                const int kb_per_unit = C::FP8 ? 1 : num_kb;
-                int kb = 0;
-                for (int u = 0; u < units && ok; ++u) {
-                    const uint32_t buf = it % C::NBUF, bph = (it / C::NBUF) & 1;
-                    if (!mbar_wait(&tempty[buf], bph ^ 1, ab, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t d0 = tmem_base + buf * C::ACC_COLS;
-                    for (int j = 0; j < kb_per_unit; ++j, ++kb) {
-                        if (!mbar_wait(&full[stage], phase, ab, p.status)) {
+                int next_L = claim(0);
+                for (int i = 0; ok; ++i) {
+                    const int slot = i % kRing;
+                    int L = next_L;
+                    if (L >= total) L = -1;
+                    else next_L = claim(i + 1);
+                    if (!mbar_wait(&ring_empty[slot], ((i / kRing) & 1) ^ 1, ab, p.status)) break;
+                    ring[slot] = L;
+                    mbar_arrive(&ring_full[slot]);
+                    if (L < 0) break;
+                    const Tile tl = decode_tile<C::BN>(L, T1, blk_start, s_off, p);
+                    const bool g1 = tl.phase == 1;
+                    const CUtensorMap* tw = g1 ? &tmW1 : &tmW2;
+                    const CUtensorMap* ta = g1 ? &tmX : &tmH;
+                    const int all_kb = (g1 ? p.H : p.I) / C::BK;
+                    const int kbase = g1 ? tl.ks * all_kb / p.s1 : 0;  // this tile's K blocks
+                    const int num_kb = g1 ? (tl.ks + 1) * all_kb / p.s1 - kbase : all_kb;
+                    const int n_box = (max(16, (tl.nrows + 15) & ~15) + C::BOX_ROWS - 1) / C::BOX_ROWS;
+                    const uint32_t tx = (tl.dual ? 2 : 1) * (C::INT4 ? C::RAW_BYTES : C::A_BYTES) + n_box * C::BOX_BYTES;
+                    auto load_act = [&](uint8_t* st, uint64_t* bar, int kx) {
+                        for (int r = 0; r < n_box; ++r)
+                            tma_load_2d(st + C::B_OFF + r * C::BOX_BYTES, ta, bar, kx, tl.row0 + r * C::BOX_ROWS);
+                    };
+                    // GEMM2 after GEMM1 in the same launch: weights of the first stages go out
+                    // before waiting for the block's h rows.
+                    const bool dep = chained && !g1;
+                    const int pre = dep ? min(num_kb, C::STAGES) : 0;
+                    const uint32_t st0 = stage;
+                    // Wait for the block's h rows, then load the activation rows of the
+                    // prefetched stages. They are loaded even when the wait gave up (the rows
+                    // are in bounds; the results are discarded), so every armed stage completes.
+                    auto release_prefetched = [&]() -> bool {
+                        const bool dep_ok = wait_counter_geq(p.done1 + tl.blk, p.c1, ab, p.status);
+                        uint32_t s2 = st0;
+                        for (int k2 = 0; k2 < pre; ++k2) {
+                            load_act(smem + (size_t)s2 * C::STAGE_BYTES, C::INT4 ? &raw_full[s2] : &full[s2],
+                                     (kbase + k2) * C::BK);
+                            if (++s2 == (uint32_t)C::STAGES) s2 = 0;
+                        }
+                        return dep_ok;
+                    };
+                    for (int kb = 0; kb < num_kb && ok; ++kb) {
+                        if (kb == pre && dep && !release_prefetched()) {
                             ok = false;
                             break;
                         }
-                        tc_fence_after();
-                        const uint32_t a0 = smem_u32(smem + (size_t)stage * C::STAGE_BYTES);
-                        const uint32_t b0 = a0 + C::B_OFF;
-                        const uint32_t at = tmem_base + C::A_TMEM + stage * C::A_TMEM_COLS;  // INT4 A tiles
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t bd = smem_desc_sw128(b0 + kk * 32);
-                            const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-                            if constexpr (C::INT4) {
-                                mma_bf16_tmem_a(d0, at + kk * 8, bd, idesc, acc);
-                                if (tl.dual) mma_bf16_tmem_a(d0 + C::BN, at + 32 + kk * 8, bd, idesc, acc);
-                            } else if constexpr (C::FP8) {
-                                mma_fp8(d0, smem_desc_sw128(a0 + kk * 32), bd, idesc, acc);
-                                if (tl.dual)
-                                    mma_fp8(d0 + C::BN, smem_desc_sw128(a0 + C::A_BYTES + kk * 32), bd, idesc, acc);
-                            } else {
-                                mma_bf16(d0, smem_desc_sw128(a0 + kk * 32), bd, idesc, acc);
-                                if (tl.dual)
-                                    mma_bf16(d0 + C::BN, smem_desc_sw128(a0 + C::A_BYTES + kk * 32), bd, idesc, acc);
-                            }
+                        if (!mbar_wait(&empty[stage], phase ^ 1, ab, p.status)) {
+                            ok = false;
+                            break;
                         }
-                        tc_commit(&empty[stage]);
+                        uint8_t* st = smem + (size_t)stage * C::STAGE_BYTES;
+                        uint64_t* bar = C::INT4 ? &raw_full[stage] : &full[stage];
+                        mbar_arrive_expect_tx(bar, tx);
+                        const int kx = (kbase + kb) * C::BK;
+                        if constexpr (C::INT4) {  // packed weight bytes: x is a byte offset (2 K per byte)
+                            tma_load_2d(st + C::RAW_OFF, tw, bar, kx / 2, tl.a0row);
+                            if (tl.dual) tma_load_2d(st + C::RAW_OFF + C::RAW_BYTES, tw, bar, kx / 2, tl.a1row);
+                        } else {
+                            tma_load_2d(st, tw, bar, kx, tl.a0row);
+                            if (tl.dual) tma_load_2d(st + C::A_BYTES, tw, bar, kx, tl.a1row);
+                        }
+                        if (kb >= pre) load_act(st, bar, kx);
+                        pend_mask |= 1u << stage;
+                        pend_phase = (pend_phase & ~(1u << stage)) | (phase << stage);
                         if (++stage == (uint32_t)C::STAGES) {
                             stage = 0;
                             phase ^= 1;
                         }
                     }
-                    if (!ok) break;
-                    tc_commit(&tfull[buf]);
-                    ++it;
+                    if (ok && dep && pre == num_kb && !release_prefetched()) ok = false;  // whole K prefetched
                 }
+                // Never leave with a copy in flight: wait for the last fill of every stage.
+                for (int s = 0; s < C::STAGES; ++s)
+                    if ((pend_mask >> s) & 1u)
+                        mbar_wait_drain(C::INT4 ? &raw_full[s] : &full[s], (pend_phase >> s) & 1u);
             }
-            // All MMAs issued by this thread complete before TMEM is released.
-            tc_commit(drain);
-            mbar_wait_drain(drain, 0);
+            __syncwarp();
+        } else if (warp == 1) {
+            // ------------------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                uint32_t stage = 0, phase = 0, it = 0;
+                bool ok = true;
+                for (int i = 0; ok; ++i) {
+                    const int slot = i % kRing;
+                    if (!mbar_wait(&ring_full[slot], (i / kRing) & 1, ab, p.status)) break;
+                    const int L = ring[slot];
+                    mbar_arrive(&ring_empty[slot]);
+                    if (L < 0) break;
+                    const Tile tl = decode_tile<C::BN>(L, T1, blk_start, s_off, p);
+                    const bool g1 = tl.phase == 1;
+                    const int all_kb = (g1 ? p.H : p.I) / C::BK;
+                    const int kbase = g1 ? tl.ks * all_kb / p.s1 : 0;
+                    const int num_kb = g1 ? (tl.ks + 1) * all_kb / p.s1 - kbase : all_kb;
+                    const int n_mma = max(16, (tl.nrows + 15) & ~15);
+                    // wide FP8: M = the 128 token rows, N = the 256 (or 128) weight rows
+                    const uint32_t idesc = C::WIDE ? idesc_m128(tl.dual ? 256 : 128, true) : idesc_m128(n_mma, C::FP8);
+                    // bf16: one TMEM buffer per tile; FP8: one per 128-deep K block
+                    const int units = C::FP8 ? num_kb : 1;
+                    const int kb_per_unit = C::FP8 ? 1 : num_kb;
+                    int kb = 0;
+                    for (int u = 0; u < units && ok; ++u) {
+                        const uint32_t buf = it % C::NBUF, bph = (it / C::NBUF) & 1;
+                        if (!mbar_wait(&tempty[buf], bph ^ 1, ab, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t d0 = tmem_base + buf * C::ACC_COLS;
+                        for (int j = 0; j < kb_per_unit; ++j, ++kb) {
+                            if (!mbar_wait(&full[stage], phase, ab, p.status)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint32_t a0 = smem_u32(smem + (size_t)stage * C::STAGE_BYTES);
+                            const uint32_t b0 = a0 + C::B_OFF;
+                            const uint32_t at = tmem_base + C::A_TMEM + stage * C::A_TMEM_COLS;  // INT4 A tiles
+    #pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint64_t bd = smem_desc_sw128(b0 + kk * 32);
+                                const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+                                if constexpr (C::INT4) {
+                                    mma_bf16_tmem_a(d0, at + kk * 8, bd, idesc, acc);
+                                    if (tl.dual) mma_bf16_tmem_a(d0 + C::BN, at + 32 + kk * 8, bd, idesc, acc);
+                                } else if constexpr (C::WIDE) {
+                                    // the token tile is the A operand; A0 | A1 (contiguous) the B operand
+                                    mma_fp8(d0, bd, smem_desc_sw128(a0 + kk * 32), idesc, acc);
+                                } else if constexpr (C::FP8) {
+                                    mma_fp8(d0, smem_desc_sw128(a0 + kk * 32), bd, idesc, acc);
+                                    if (tl.dual)
+                                        mma_fp8(d0 + C::BN, smem_desc_sw128(a0 + C::A_BYTES + kk * 32), bd, idesc, acc);
+                                } else {
+                                    mma_bf16(d0, smem_desc_sw128(a0 + kk * 32), bd, idesc, acc);
+                                    if (tl.dual)
+                                        mma_bf16(d0 + C::BN, smem_desc_sw128(a0 + C::A_BYTES + kk * 32), bd, idesc, acc);
+                                }
+                            }
+                            tc_commit(&empty[stage]);
+                            if (++stage == (uint32_t)C::STAGES) {
+                                stage = 0;
+                                phase ^= 1;
+                            }
+                        }
+                        if (!ok) break;
+                        tc_commit(&tfull[buf]);
+                        ++it;
+                    }
+                }
+                // All MMAs issued by this thread complete before TMEM is released.
+                tc_commit(drain);
+                mbar_wait_drain(drain, 0);
+            }
+            __syncwarp();
         }
-        __syncwarp();
-    } else if (C::INT4 && warp >= 2 + C::EPI) {
+    } else if (C::INT4 && warp >= C::EPI0 + C::EPI) {
         // ------------------------------------------------------------ INT4 dequantisation
         // Each warp converts the 32 weight rows of its TMEM lane quarter (warp % 4) of one
         // tile (A0 or A1; with 4 warps both tiles) of every stage, in the same tile order as
         // the MMA, stores them into the stage's TMEM A columns and completes `full`.
         const int r = (warp & 3) * 32 + lane;
-        const int dt = ((warp - 2 - C::EPI) / 4) * 128 + r;  // tile = dt / 128
+        const int dt = ((warp - C::EPI0 - C::EPI) / 4) * 128 + r;  // tile = dt / 128
         constexpr int kTileStep = C::DQ * 32 / 128;  // tiles apart that one thread converts
         const uint32_t lane_sel = (uint32_t)((warp & 3) * 32) << 16;
         uint32_t stage = 0, phase = 0;
@@ -626,7 +648,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int ew = warp - 2;
+        if constexpr (C::WIDE) setmaxnreg_inc<C::REG_HIGH>();
+        const int ew = warp - C::EPI0;
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const int cg = ew >> 2;  // which group of the tile's columns
         const int c0 = cg * C::COLS;
@@ -769,6 +792,157 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                 const float hv = swiglu_dev(sg * gs[j], su * us[j], p.alpha, p.beta, lim);
                                 out[(size_t)(tl.row0 + n) * out_ld + col] = __float2bfloat16_rn(hv);
                             }
+                        }
+                    }
+                }
+            } else if constexpr (C::WIDE) {
+                // Token-major FP8 tile: TMEM lane = token row of the block, columns = weight
+                // rows (gate | up, or two 128-row chunks of H). This warp takes columns
+                // cg*64 .. +64 of each half, so a thread holds gate and up of 64 intermediate
+                // indices of its own token, and a K block's scale product is one scalar per
+                // half: no per-column scale table, a thread-local amax for h's 1x128 block
+                // (plus the other column group's, through shared memory), and whole 16-byte
+                // stores of h and y rows.
+                const int tok = row_local;
+                const bool has_tok = tok < tl.nrows;
+                const bool quarter_live = q * 32 < tl.nrows;  // warp-uniform
+                const int num_kb = (g1 ? p.H : p.I) / C::BK;   // no split-K at this width
+                const float* act_scale = g1 ? p.x_scale : p.h_scale;
+                const float* wscale = static_cast<const float*>(g1 ? p.w1_scale : p.w2_scale);
+                const float* wsg = wscale + (size_t)(tl.a0row / 128) * num_kb;
+                const float* wsu = wscale + (size_t)(tl.a1row / 128) * num_kb;
+                if (!g1 && chained) {  // h_scale comes from GEMM1 tiles of this block (see below)
+                    bool dep_ok = true;
+                    if (lane == 0) dep_ok = wait_counter_geq(p.done1 + tl.blk, p.c1, ab, p.status);
+                    dep_ok = __shfl_sync(0xffffffffu, dep_ok ? 1 : 0, 0) != 0;
+                    __syncwarp();
+                    if (!dep_ok) {
+                        ok = false;
+                        break;
+                    }
+                }
+                float acc0[64], acc1[64];
+#pragma unroll
+                for (int j = 0; j < 64; ++j) acc0[j] = acc1[j] = 0.f;
+                constexpr int kPF = 4;  // K blocks of scales loaded ahead
+                const float* sb_ptr = act_scale + tl.row0 + tok;
+                float q_sb[kPF], q_s0[kPF], q_s1[kPF];
+#pragma unroll
+                for (int i = 0; i < kPF; ++i) {
+                    const bool in = i < num_kb;
+                    q_sb[i] = (in && has_tok) ? __ldcg(sb_ptr + (size_t)i * p.A) : 0.f;
+                    q_s0[i] = in ? __ldg(wsg + i) : 0.f;
+                    q_s1[i] = (in && tl.dual) ? __ldg(wsu + i) : 0.f;
+                }
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    const uint32_t buf = it % C::NBUF, bph = (it / C::NBUF) & 1;
+                    const float f0 = q_s0[0] * q_sb[0], f1 = q_s1[0] * q_sb[0];
+#pragma unroll
+                    for (int i = 0; i + 1 < kPF; ++i) {
+                        q_sb[i] = q_sb[i + 1];
+                        q_s0[i] = q_s0[i + 1];
+                        q_s1[i] = q_s1[i + 1];
+                    }
+                    {
+                        const int kn = kb + kPF;
+                        const bool in = kn < num_kb;
+                        q_sb[kPF - 1] = (in && has_tok) ? __ldcg(sb_ptr + (size_t)kn * p.A) : 0.f;
+                        q_s0[kPF - 1] = in ? __ldg(wsg + kn) : 0.f;
+                        q_s1[kPF - 1] = (in && tl.dual) ? __ldg(wsu + kn) : 0.f;
+                    }
+                    if (!warp_wait(&tfull[buf], bph, ab, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t tb = tmem_base + lane_off + buf * C::ACC_COLS + cg * 64;
+                    if (!quarter_live) {  // no token of this lane quarter in the tile
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tempty[buf]);
+                    }
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        if (!quarter_live) break;
+                        float p0[16], p1[16];
+                        if (tl.dual) tmem_ld_x2<16>(tb + ch * 16, tb + C::BN + ch * 16, p0, p1);
+                        else tmem_ld_x1<16>(tb + ch * 16, p0);
+                        if (ch == 3) {  // the buffer goes back to the MMA before the arithmetic
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&tempty[buf]);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 16; j += 2) {
+                            ffma2(acc0[ch * 16 + j], acc0[ch * 16 + j + 1], p0[j], p0[j + 1], f0, f0);
+                            if (tl.dual) ffma2(acc1[ch * 16 + j], acc1[ch * 16 + j + 1], p1[j], p1[j + 1], f1, f1);
+                        }
+                    }
+                    ++it;
+                }
+                if (!ok) break;
+                if (g1) {
+                    float amax = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) {
+                        acc0[j] = swiglu_dev(sg * acc0[j], su * acc1[j], p.alpha, p.beta, lim);
+                        amax = fmaxf(amax, fabsf(acc0[j]));
+                    }
+                    red[cg * 128 + tok] = amax;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(epibar);
+                    if (!warp_wait(epibar, ephase, ab, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    ephase ^= 1;
+                    amax = fmaxf(red[tok], red[128 + tok]);  // the token's 1x128 block: both column groups
+                    const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+                    const float inv_s = amax == 0.f ? 1.f : __fdividef(448.f, amax);
+                    if (has_tok) {
+                        // h rows and the chunk offset are multiples of 16 bytes (I % 128 == 0,
+                        // h 16-byte aligned), so each 16 codes go out as one vector store
+                        uint8_t* dst = static_cast<uint8_t*>(p.h) + (size_t)(tl.row0 + tok) * p.I + tl.col0 + cg * 64;
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                const int j = v * 16 + t * 4;
+                                const uint32_t lo = __nv_cvt_float2_to_fp8x2(
+                                    make_float2(acc0[j] * inv_s, acc0[j + 1] * inv_s), __NV_SATFINITE, __NV_E4M3);
+                                const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+                                    make_float2(acc0[j + 2] * inv_s, acc0[j + 3] * inv_s), __NV_SATFINITE, __NV_E4M3);
+                                w[t] = lo | (hi << 16);
+                            }
+                            *reinterpret_cast<uint4*>(dst + 16 * v) = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                        if (cg == 0) p.h_scale[(size_t)tl.c * p.A + tl.row0 + tok] = s;
+                    }
+                } else if (has_tok) {
+                    // y rows (H % 128 == 0, y 16-byte aligned): 8 bf16 per vector store
+                    __nv_bfloat16* row = static_cast<__nv_bfloat16*>(p.y) + (size_t)(tl.row0 + tok) * p.H;
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const __nv_bfloat162 b = __floats2bfloat162_rn(acc0[v * 8 + 2 * t], acc0[v * 8 + 2 * t + 1]);
+                            w[t] = *reinterpret_cast<const uint32_t*>(&b);
+                        }
+                        *reinterpret_cast<uint4*>(row + tl.col0 + cg * 64 + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                    if (tl.dual) {
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                const __nv_bfloat162 b =
+                                    __floats2bfloat162_rn(acc1[v * 8 + 2 * t], acc1[v * 8 + 2 * t + 1]);
+                                w[t] = *reinterpret_cast<const uint32_t*>(&b);
+                            }
+                            *reinterpret_cast<uint4*>(row + tl.col1 + cg * 64 + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
                         }
                     }
                 }
@@ -1115,6 +1289,10 @@ static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
             cudaFuncAttributes fa;
             cudaError_t e = cudaFuncGetAttributes(&fa, moe_gemm_kernel<C>);
             if (e != cudaSuccess) return e;
+            // The register split must fit what the launch brings, else setmaxnreg.inc would
+            // wait for registers that never come: refuse to launch instead.
+            if (C::WIDE && fa.numRegs * C::THREADS < 128 * C::REG_LOW + (C::THREADS - 128) * C::REG_HIGH)
+                return cudaErrorInvalidConfiguration;
             limit = kSmemLimit - (int)fa.sharedSizeBytes;
             e = cudaFuncSetAttribute(moe_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, limit);
             if (e != cudaSuccess) return e;
@@ -1131,7 +1309,7 @@ int gemm_pick_bn(int64_t A, int G, int wdtype) {
     const double avg = G > 0 ? (double)A / (double)G : 0.0;
     int bn = 16;
     while (bn < 256 && bn < avg) bn <<= 1;  // smallest tile holding an average group
-    if (wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128 && bn > 64) bn = 64;  // fp32 promotion registers for gate and up
+    if (wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128 && bn > 128) bn = 128;  // fp32 promotion registers for gate and up
     if (wdtype == MOE_WDTYPE_INT4_G32 && bn > 64) bn = 64;  // A tiles share TMEM with the accumulators
     return bn;
 }
@@ -1188,6 +1366,7 @@ cudaError_t launch_moe_gemm(const MoeGemmArgs& a, cudaStream_t stream) {
             case 16: return launch_cfg<Cfg<16, true>>(a, stream);
             case 32: return launch_cfg<Cfg<32, true>>(a, stream);
             case 64: return launch_cfg<Cfg<64, true>>(a, stream);
+            case 128: return launch_cfg<Cfg<128, true>>(a, stream);
             default: return cudaErrorInvalidValue;
         }
     }

@@ -389,6 +389,18 @@ __device__ __forceinline__ void tmem_ld_x1(uint32_t ta, float* a) {
     else tmem_ld4(ta, a);
 }
 
+// Register reallocation between warpgroups: every warp of a warpgroup executes the same
+// instruction. dec returns registers to the CTA's pool, inc blocks until the pool holds
+// enough; the launch's threads x registers must cover the largest split.
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

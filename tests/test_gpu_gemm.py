@@ -92,7 +92,9 @@ GEMM1_CASES = [
     (1024, 8, 2, 0, 512, 256, False, {"skew": 2.0}),            # tile 256, several blocks, ragged tails
     (600, 4, 2, 1, 512, 384, False, {"scales": True}),          # tile 256, shared group of 600 rows
     (96, 32, 4, 0, 2048, 768, False, {"oai": True}),            # OAI-SwiGLU shape and parameters
-    (512, 8, 2, 0, 512, 256, True, {}),                         # FP8, tile 64
+    (512, 8, 2, 0, 512, 256, True, {}),                         # FP8, tile 128 (register split)
+    (256, 8, 2, 0, 512, 256, True, {}),                         # FP8, tile 64
+    (1024, 8, 2, 1, 512, 384, True, {"skew": 2.0, "scales": True, "limits": True}),  # FP8 tile 128, ragged, shared
     (40, 32, 4, 1, 512, 256, True, {"glm": True}),              # FP8, tile 16, shared group, L = 10
     (200, 8, 2, 0, 1024, 512, True, {"oai": True, "scales": True}),
     (128, 8, 2, 1, 512, 384, False, {"limits": True}),          # a clamp per expert (shared group too)
@@ -145,7 +147,9 @@ GEMM2_CASES = [
     (300, 16, 4, 1, 512, 256, False, False),    # one shared group with weight 1
     (1024, 8, 2, 0, 512, 256, False, False),    # tile 256
     (600, 4, 2, 1, 384, 256, False, True),      # tile 256, odd number of 128-row chunks of H
-    (512, 8, 2, 0, 512, 256, True, False),
+    (512, 8, 2, 0, 512, 256, True, False),      # FP8, tile 128
+    (256, 8, 2, 0, 512, 256, True, False),      # FP8, tile 64
+    (600, 4, 2, 1, 384, 256, True, True),       # FP8, tile 128, odd chunk count of H, sink-gated shared
     (40, 32, 4, 1, 512, 256, True, False),
     (8, 64, 4, 0, 256, 256, "int4", False),     # INT4 weights, tile 16
     (300, 16, 4, 2, 512, 256, "int4", True),    # INT4, sink-gated shared groups
