@@ -31,8 +31,9 @@
 // Roles (320 threads): warp 0 lane 0 issues TMA loads into a STAGES-deep ring; warp 1
 // owns TMEM and lane 0 issues tcgen05.mma; warps 2..9 are the epilogue (warp w reads
 // TMEM lanes 32*(w%4).., and columns of half (w-2)/4 of the tile). FP8 tiles of 128
-// token columns launch 384 threads: warps 2-3 are spares whose registers go to the
-// epilogue, warps 4..11 are the epilogue. Every wait is bounded
+// tokens are token-major (tokens = M = TMEM lanes) and launch 384 threads: warp 2
+// releases GEMM1 tiles' h to GEMM2, warp 3 only lends its registers, and warps 4..11 are
+// the epilogue. Every wait is bounded
 // (ptx.cuh): on timeout the CTA sets MOE_ERR_TIMEOUT, drains its outstanding copies and
 // MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -97,28 +98,33 @@ struct Cfg {
     // Epilogue warps: groups of four (one warp per TMEM lane quarter), each group owning
     // an equal share of the tile's columns; four groups at 256 columns, whose single
     // accumulator buffer makes the drain time part of the tile time.
-    static constexpr int EPI = BN >= 256 ? 16 : ((INT4 && BN <= 32) ? 4 : 8);
-    // FP8 at 128 token columns: the promoted gate and up sums of a 128 x 128 tile take 128
-    // registers per epilogue thread. Two spare warps make warps 0-3 (producer, MMA, spares)
-    // one warpgroup, which gives registers back (setmaxnreg) to the two epilogue warpgroups:
-    // 384 threads launch with 168 registers; 4 warps drop to REG_LOW, 8 rise to REG_HIGH.
+    // FP8 at 128 token columns: the promoted gate and up sums of a 128 x 128 tile fill half
+    // the register file. Two more warps make warps 0-3 (producer, MMA, the publisher of
+    // GEMM1 tiles, an idle warp) one warpgroup, which gives registers back (setmaxnreg) to
+    // the epilogue warpgroups: the launch's threads x registers cover 4 warps at REG_LOW
+    // and WEPI epilogue warps at REG_HIGH.
     static constexpr bool WIDE = FP8 && BN >= 128;
+    static constexpr int WEPI = 8;  // wide FP8 epilogue warps: 8 (128 sums each) or 16 (64)
+    static constexpr int EPI = WIDE ? WEPI : (BN >= 256 ? 16 : ((INT4 && BN <= 32) ? 4 : 8));
     static constexpr int EPI0 = WIDE ? 4 : 2;  // first epilogue warp
-    static constexpr int REG_LOW = 56, REG_HIGH = 224;
+    static constexpr int REG_LAUNCH = WIDE ? (65536 / (32 * (4 + WEPI))) / 8 * 8 : 0;
+    static constexpr int REG_LOW = 56, REG_HIGH = WEPI == 8 ? 224 : 104;
+    static constexpr int WCH = 16;  // wide FP8: TMEM columns per load of each half
     static constexpr int THREADS = 32 * EPI0 + 32 * EPI + 32 * DQ;
     static constexpr int GROUPS = EPI / 4;
     static constexpr int COLS = BN / GROUPS;  // columns per epilogue warp
     static constexpr int CW = COLS < 16 ? COLS : 16;  // TMEM load width (columns)
-    static constexpr int RED_FLOATS = FP8 ? EPI * COLS : 4;
+    static constexpr int RED_FLOATS = WIDE ? 2 * GROUPS * 128 : (FP8 ? EPI * COLS : 4);
     // FP8: per epilogue warp, the two rows of scale products (A0, A1) of its columns
     static constexpr int SCT_FLOATS = (FP8 && !WIDE) ? EPI * 2 * COLS : 4;
     static_assert(STAGE_BYTES % 1024 == 0, "stage tiles must stay 1024-byte aligned");
     static_assert(TMEM_COLS <= 512, "TMEM holds 512 columns");
     static_assert(COLS % CW == 0 && CW >= 4, "column share must be a multiple of the load width");
     static_assert(!FP8 || WIDE || COLS <= 32, "FP8 loads a warp's whole column share at once");
-    static_assert(!WIDE || (BN == 128 && EPI == 8 && THREADS == 384 &&
-                            128 * REG_LOW + 256 * REG_HIGH <= THREADS * 168),
-                  "register split of the wide FP8 tile");
+    static_assert(!WIDE || (BN == 128 && (EPI == 8 || EPI == 16) && COLS % 16 == 0 &&
+                            128 * REG_LOW + 32 * EPI * REG_HIGH <= THREADS * REG_LAUNCH &&
+                            REG_LOW + (EPI / 4) * REG_HIGH <= 512),
+                  "register split of the wide FP8 tile (whole CTA and per SM sub-partition)");
     static_assert(BN % BOX_ROWS == 0 && BN <= 256, "token tile = whole boxes, at most the MMA's N limit");
     static_assert(STAGES >= 2, "at least two pipeline stages");
     static_assert(!(INT4 && FP8), "INT4 weights take bf16 activations");
@@ -130,7 +136,7 @@ struct Cfg {
 
     // full/empty per stage, tfull/tempty per TMEM buffer, ring_full/ring_empty x kRing, drain,
     // epibar, and for INT4 raw_full per stage (packed bytes and token rows landed)
-    static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 2 * kRing + 2 + (INT4 ? STAGES : 0);
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 2 * kRing + 2 + (INT4 ? STAGES : 0) + (WIDE ? 1 : 0);
     static constexpr size_t ctrl_bytes() {
         return 8 * NUM_BARS + 16 + 4 * kRing + 16 + 4 * RED_FLOATS + 16 + 4 * SCT_FLOATS;
     }
@@ -337,7 +343,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint64_t* drain = ring_empty + kRing;
     uint64_t* epibar = drain + 1;
     uint64_t* raw_full = epibar + 1;  // INT4 only: [STAGES]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(raw_full + (C::INT4 ? C::STAGES : 0));
+    uint64_t* pubbar = raw_full + (C::INT4 ? C::STAGES : 0);  // wide FP8 only: a GEMM1 tile's h is stored
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pubbar + (C::WIDE ? 1 : 0));
     PipeAbort* ab = reinterpret_cast<PipeAbort*>(tmem_slot + 1);
     int* ring = reinterpret_cast<int*>(tmem_slot + 4);
     float* red = reinterpret_cast<float*>(ring + kRing + 4);
@@ -360,10 +367,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         for (int r = 0; r < kRing; ++r) {
             mbar_init(&ring_full[r], 1);
-            mbar_init(&ring_empty[r], 1 + C::EPI + C::DQ);
+            mbar_init(&ring_empty[r], 1 + C::EPI + C::DQ + (C::WIDE ? 1 : 0));
         }
         mbar_init(drain, 1);
         mbar_init(epibar, C::EPI);
+        if (C::WIDE) mbar_init(pubbar, C::EPI);
         ab->flag = 0;
         fence_barrier_init();
     }
@@ -582,6 +590,29 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 mbar_wait_drain(drain, 0);
             }
             __syncwarp();
+        } else if (C::WIDE && warp == 2) {
+            // -------------------------------------------------------- publisher (wide FP8)
+            // Releases each GEMM1 tile's h rows to the GEMM2 tiles of its block once every
+            // epilogue warp has stored its share (pubbar: arrive = release, wait = acquire at
+            // CTA scope, then a GPU-scope fence and a release add), so that fence, which can
+            // take microseconds under a saturated memory system, stays off the epilogue.
+            if (lane == 0) {
+                uint32_t pph = 0;
+                for (int i = 0;; ++i) {
+                    const int slot = i % kRing;
+                    if (!mbar_wait(&ring_full[slot], (i / kRing) & 1, ab, p.status)) break;
+                    const int L = ring[slot];
+                    mbar_arrive(&ring_empty[slot]);
+                    if (L < 0) break;
+                    if (!chained || L >= T1) continue;  // GEMM1 tiles of a two-phase launch only
+                    if (!mbar_wait(pubbar, pph, ab, p.status)) break;
+                    pph ^= 1;
+                    __threadfence();
+                    fence_proxy_async_global();
+                    red_release_add_gpu(p.done1 + (L / p.s1) / p.c1, 1);
+                }
+            }
+            __syncwarp();
         }
     } else if (C::INT4 && warp >= C::EPI0 + C::EPI) {
         // ------------------------------------------------------------ INT4 dequantisation
@@ -656,6 +687,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const int row_local = q * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         uint32_t it = 0, ephase = 0;
+        uint32_t g1_tiles = 0;  // wide FP8: GEMM1 tiles done (parity picks the amax buffer)
         bool ok = true;
         int* merge_flag = ring + kRing + 1;
         // Split-K of GEMM1: this split's partials are in memory. Returns 1 when this CTA
@@ -798,11 +830,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             } else if constexpr (C::WIDE) {
                 // Token-major FP8 tile: TMEM lane = token row of the block, columns = weight
                 // rows (gate | up, or two 128-row chunks of H). This warp takes columns
-                // cg*64 .. +64 of each half, so a thread holds gate and up of 64 intermediate
+                // cg*CC .. +CC of each half, so a thread holds gate and up of CC intermediate
                 // indices of its own token, and a K block's scale product is one scalar per
                 // half: no per-column scale table, a thread-local amax for h's 1x128 block
                 // (plus the other column group's, through shared memory), and whole 16-byte
                 // stores of h and y rows.
+                constexpr int CC = C::COLS;  // columns of each half per warp
                 const int tok = row_local;
                 const bool has_tok = tok < tl.nrows;
                 const bool quarter_live = q * 32 < tl.nrows;  // warp-uniform
@@ -821,9 +854,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         break;
                     }
                 }
-                float acc0[64], acc1[64];
+                float acc0[CC], acc1[CC];
 #pragma unroll
-                for (int j = 0; j < 64; ++j) acc0[j] = acc1[j] = 0.f;
+                for (int j = 0; j < CC; ++j) acc0[j] = acc1[j] = 0.f;
                 constexpr int kPF = 4;  // K blocks of scales loaded ahead
                 const float* sb_ptr = act_scale + tl.row0 + tok;
                 float q_sb[kPF], q_s0[kPF], q_s1[kPF];
@@ -855,27 +888,28 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t tb = tmem_base + lane_off + buf * C::ACC_COLS + cg * 64;
+                    const uint32_t tb = tmem_base + lane_off + buf * C::ACC_COLS + cg * CC;
                     if (!quarter_live) {  // no token of this lane quarter in the tile
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&tempty[buf]);
                     }
+                    constexpr int W = C::WCH;
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
+                    for (int ch = 0; ch < CC / W; ++ch) {
                         if (!quarter_live) break;
-                        float p0[16], p1[16];
-                        if (tl.dual) tmem_ld_x2<16>(tb + ch * 16, tb + C::BN + ch * 16, p0, p1);
-                        else tmem_ld_x1<16>(tb + ch * 16, p0);
-                        if (ch == 3) {  // the buffer goes back to the MMA before the arithmetic
+                        float p0[W], p1[W];
+                        if (tl.dual) tmem_ld_x2<W>(tb + ch * W, tb + C::BN + ch * W, p0, p1);
+                        else tmem_ld_x1<W>(tb + ch * W, p0);
+                        if (ch == CC / W - 1) {  // the buffer goes back to the MMA before the arithmetic
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) mbar_arrive(&tempty[buf]);
                         }
 #pragma unroll
-                        for (int j = 0; j < 16; j += 2) {
-                            ffma2(acc0[ch * 16 + j], acc0[ch * 16 + j + 1], p0[j], p0[j + 1], f0, f0);
-                            if (tl.dual) ffma2(acc1[ch * 16 + j], acc1[ch * 16 + j + 1], p1[j], p1[j + 1], f1, f1);
+                        for (int j = 0; j < W; j += 2) {
+                            ffma2(acc0[ch * W + j], acc0[ch * W + j + 1], p0[j], p0[j + 1], f0, f0);
+                            if (tl.dual) ffma2(acc1[ch * W + j], acc1[ch * W + j + 1], p1[j], p1[j + 1], f1, f1);
                         }
                     }
                     ++it;
@@ -884,11 +918,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 if (g1) {
                     float amax = 0.f;
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) {
+                    for (int j = 0; j < CC; ++j) {
                         acc0[j] = swiglu_dev(sg * acc0[j], su * acc1[j], p.alpha, p.beta, lim);
                         amax = fmaxf(amax, fabsf(acc0[j]));
                     }
-                    red[cg * 128 + tok] = amax;
+                    float* rb = red + (g1_tiles++ & 1) * (C::GROUPS * 128);  // two tiles' worth: no second meeting
+                    rb[cg * 128 + tok] = amax;
                     __syncwarp();
                     if (lane == 0) mbar_arrive(epibar);
                     if (!warp_wait(epibar, ephase, ab, p.status)) {
@@ -896,15 +931,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         break;
                     }
                     ephase ^= 1;
-                    amax = fmaxf(red[tok], red[128 + tok]);  // the token's 1x128 block: both column groups
+#pragma unroll
+                    for (int g = 0; g < C::GROUPS; ++g) amax = fmaxf(amax, rb[g * 128 + tok]);  // the 1x128 block
                     const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
                     const float inv_s = amax == 0.f ? 1.f : __fdividef(448.f, amax);
                     if (has_tok) {
                         // h rows and the chunk offset are multiples of 16 bytes (I % 128 == 0,
                         // h 16-byte aligned), so each 16 codes go out as one vector store
-                        uint8_t* dst = static_cast<uint8_t*>(p.h) + (size_t)(tl.row0 + tok) * p.I + tl.col0 + cg * 64;
+                        uint8_t* dst = static_cast<uint8_t*>(p.h) + (size_t)(tl.row0 + tok) * p.I + tl.col0 + cg * CC;
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
+                        for (int v = 0; v < CC / 16; ++v) {
                             uint32_t w[4];
 #pragma unroll
                             for (int t = 0; t < 4; ++t) {
@@ -923,18 +959,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     // y rows (H % 128 == 0, y 16-byte aligned): 8 bf16 per vector store
                     __nv_bfloat16* row = static_cast<__nv_bfloat16*>(p.y) + (size_t)(tl.row0 + tok) * p.H;
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) {
+                    for (int v = 0; v < CC / 8; ++v) {
                         uint32_t w[4];
 #pragma unroll
                         for (int t = 0; t < 4; ++t) {
                             const __nv_bfloat162 b = __floats2bfloat162_rn(acc0[v * 8 + 2 * t], acc0[v * 8 + 2 * t + 1]);
                             w[t] = *reinterpret_cast<const uint32_t*>(&b);
                         }
-                        *reinterpret_cast<uint4*>(row + tl.col0 + cg * 64 + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
+                        *reinterpret_cast<uint4*>(row + tl.col0 + cg * CC + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                     if (tl.dual) {
 #pragma unroll
-                        for (int v = 0; v < 8; ++v) {
+                        for (int v = 0; v < CC / 8; ++v) {
                             uint32_t w[4];
 #pragma unroll
                             for (int t = 0; t < 4; ++t) {
@@ -942,7 +978,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                     __floats2bfloat162_rn(acc1[v * 8 + 2 * t], acc1[v * 8 + 2 * t + 1]);
                                 w[t] = *reinterpret_cast<const uint32_t*>(&b);
                             }
-                            *reinterpret_cast<uint4*>(row + tl.col1 + cg * 64 + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
+                            *reinterpret_cast<uint4*>(row + tl.col1 + cg * CC + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
                         }
                     }
                 }
@@ -1125,7 +1161,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             // fencing thread instead of every thread: under a saturated memory system each
             // fence waits microseconds for its stores to be acknowledged. In FP8 mode the
             // meeting also keeps `red` from being rewritten while read.
-            if (g1 && (chained || C::FP8)) {
+            if constexpr (C::WIDE) {
+                if (g1 && chained) {  // the publisher warp releases the block counter
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(pubbar);
+                }
+            } else if (g1 && (chained || C::FP8)) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(epibar);
                 if (!warp_wait(epibar, ephase, ab, p.status)) {
@@ -1291,7 +1332,7 @@ static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
             if (e != cudaSuccess) return e;
             // The register split must fit what the launch brings, else setmaxnreg.inc would
             // wait for registers that never come: refuse to launch instead.
-            if (C::WIDE && fa.numRegs * C::THREADS < 128 * C::REG_LOW + (C::THREADS - 128) * C::REG_HIGH)
+            if (C::WIDE && fa.numRegs * C::THREADS < 128 * C::REG_LOW + 32 * C::EPI * C::REG_HIGH)
                 return cudaErrorInvalidConfiguration;
             limit = kSmemLimit - (int)fa.sharedSizeBytes;
             e = cudaFuncSetAttribute(moe_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, limit);
