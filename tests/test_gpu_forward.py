@@ -81,7 +81,7 @@ def test_forward_skewed_routing_one_hot_expert():
     assert_bf16_close(out.float().cpu().numpy(), ref, "skewed")
 
 
-@pytest.mark.parametrize("name", ["oai_swiglu", "decode_t8", "glm_fp8"])
+@pytest.mark.parametrize("name", ["oai_swiglu", "decode_t8", "glm_fp8", "decode_t1", "decode_t1_int4"])
 def test_public_stage_calls_reproduce_forward(name):
     """moe_route_topk -> moe_permute -> moe_experts -> moe_combine gives moe_forward's
     output bit for bit (same kernels, deterministic order), and matches the oracle."""

@@ -103,6 +103,12 @@ GEMM1_CASES = [
     (64, 16, 4, 0, 512, 256, False, {"int4": True}),           # INT4, tile 32
     (300, 16, 4, 1, 512, 384, False, {"int4": True, "oai": True, "scales": True}),  # INT4, shared group
     (512, 8, 2, 0, 512, 256, False, {"int4": True, "skew": 3.0, "limits": True}),   # INT4, tile 128
+    # decode-sized batches (at most 16 routed rows): one-row groups, split-K of GEMM1
+    (2, 64, 4, 1, 512, 256, False, {}),                         # 10 rows, a shared group of 2
+    (1, 32, 4, 0, 512, 384, False, {"scales": True, "limits": True}),  # one token, scales, clamp per expert
+    (8, 2, 2, 0, 512, 256, False, {"oai": True}),               # 2 groups of 8 rows
+    (2, 64, 4, 1, 512, 256, False, {"int4": True}),            # INT4, 10 rows
+    (3, 4, 2, 1, 512, 384, False, {"int4": True, "scales": True}),  # INT4, groups of several rows
 ]
 
 
@@ -154,6 +160,9 @@ GEMM2_CASES = [
     (8, 64, 4, 0, 256, 256, "int4", False),     # INT4 weights, tile 16
     (300, 16, 4, 2, 512, 256, "int4", True),    # INT4, sink-gated shared groups
     (512, 8, 2, 0, 384, 256, "int4", False),    # INT4, tile 128, odd chunk count of H
+    (2, 64, 4, 1, 512, 256, False, False),      # decode-sized: 10 routed rows
+    (2, 16, 4, 2, 512, 256, False, True),       # decode-sized, sink-gated shared groups
+    (8, 2, 2, 0, 384, 256, "int4", False),      # INT4, 2 groups of 8 rows
 ]
 
 
