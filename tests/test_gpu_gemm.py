@@ -163,6 +163,9 @@ GEMM2_CASES = [
     (2, 64, 4, 1, 512, 256, False, False),      # decode-sized: 10 routed rows
     (2, 16, 4, 2, 512, 256, False, True),       # decode-sized, sink-gated shared groups
     (8, 2, 2, 0, 384, 256, "int4", False),      # INT4, 2 groups of 8 rows
+    # many token blocks, an odd count of 128-row chunks of H (the last GEMM2 tile has one)
+    (4096, 128, 2, 0, 384, 256, False, False),
+    (4096, 128, 2, 0, 384, 256, True, False),   # FP8, tile 64
 ]
 
 
