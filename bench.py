@@ -198,33 +198,67 @@ def config_of(wl):
             "seed": wl.seed, "l2": "flushed between timed steps (512 MiB write, outside the timed events)"}
 
 
+# ------------------------------------------------------------------ ranks
+class Ranks:
+    """One process per GPU as torchrun starts them (RANK, LOCAL_RANK, WORLD_SIZE, MASTER_*).
+
+    The layer is token-parallel: every rank runs its own batch with replicated weights and
+    there is no data-path collective; the only collectives are the barriers around the
+    timed region and a MAX all-reduce of each timing, so the reported time is the slowest
+    rank's and the whole-job rate counts every rank's tokens. `backend` is "nccl" on GPUs;
+    the tests drive the same logic with "gloo" on CPU."""
+
+    def __init__(self, backend: str = "nccl", device=None, timeout_s: float = 180.0):
+        import torch
+        import torch.distributed as dist
+        self.dist = dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.device = device if device is not None else torch.device("cpu")
+        self.backend = backend
+        if self.world > 1:
+            from datetime import timedelta
+            kw = {"device_id": self.device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=timedelta(seconds=timeout_s), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            if self.backend == "nccl":
+                self.dist.barrier(device_ids=[self.local])
+            else:
+                self.dist.barrier()
+
+    def max_over_ranks(self, v: float) -> float:
+        if self.world == 1:
+            return v
+        import torch
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def rate(self, tokens_per_rank: int, ms_per_step: float) -> float:
+        """Whole-job tokens/s: every rank's tokens over the slowest rank's step time."""
+        return self.world * tokens_per_rank / (ms_per_step / 1e3)
+
+    def close(self):
+        if self.world > 1:
+            self.dist.destroy_process_group()
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args):
     import numpy as np
     import torch
-    import torch.distributed as dist
     import grouped_gemm_swiglu_b200 as moe
     from grouped_gemm_swiglu_b200 import workloads as W
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local])
-
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    barrier, max_over_ranks = ranks.barrier, ranks.max_over_ranks
 
     wl = workload_of(args)
     inp = W.make_inputs(wl, dev)
@@ -331,7 +365,7 @@ def run_ours(args):
             acc[k] += ev[2 + i].elapsed_time(ev[3 + i])
     st = {k: max_over_ranks(v / K) for k, v in acc.items()}
     ms = max_over_ranks(fwd_sum / K)
-    value = world * T / (ms / 1e3)
+    value = ranks.rate(T, ms)
     fwd_ms = ms
     for ws in (ws_p, ws_e, ws_c, layer.ws):
         assert moe.moe_read_status(ws) == 0, moe.status_string(moe.moe_read_status(ws))
@@ -421,7 +455,7 @@ def run_ours(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": Wm,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp8_e4m3" if fp8 else "bf16", "data": "synthetic", "config": config_of(wl),
-            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "e2e": {"value": ranks.rate(T, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "roofline": roof, "clocks": clocks, "gpu_launches": 2 * launches_per_step * K,
             "stages_ms": st, "forward_ms_per_step": fwd_ms, "experts_touched": used, "gate_route": gate,
@@ -437,8 +471,7 @@ def run_ours(args):
                                 "sample": f"first {n} of {wl.T} tokens of {wl.name} ({dt:.1f} s, fp64)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
     return 0
 
 
