@@ -17,7 +17,9 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
-_LIB = os.path.join(_HERE, "liboracle.so")
+# ORACLE_LIB selects another build of oracle.c (the mutation tests load planted-mistake
+# builds this way); it is used as given, never rebuilt.
+_LIB = os.environ.get("ORACLE_LIB") or os.path.join(_HERE, "liboracle.so")
 
 WDTYPE_BF16 = 0
 WDTYPE_FP8 = 1
@@ -26,12 +28,21 @@ SCORE_SOFTMAX = 0
 SCORE_SIGMOID = 1
 
 
+def compile_library(out: str, defines=()) -> str:
+    """gcc (OpenMP, IEEE float: no fast-math, no FMA contraction) of oracle.c into `out`;
+    `defines` are extra -D flags (the mutation tests plant mistakes with ORACLE_MUTANT)."""
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall", "-fno-fast-math",
+           "-ffp-contract=off", *[f"-D{d}" for d in defines], "-o", out, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
 def build(force: bool = False) -> str:
-    """Compile oracle.c into liboracle.so next to it (gcc, OpenMP, IEEE float)."""
+    """Compile oracle.c into liboracle.so next to it."""
+    if os.environ.get("ORACLE_LIB"):
+        return _LIB
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall",
-               "-fno-fast-math", "-ffp-contract=off", "-o", _LIB, _SRC, "-lm"]
-        subprocess.run(cmd, check=True)
+        compile_library(_LIB)
     return _LIB
 
 

@@ -40,6 +40,14 @@
 #include <omp.h>
 #endif
 
+/* Mutation hooks for the oracle's own tests: a build with -DORACLE_MUTANT=n plants one
+ * plausible mistake (numbered below) so the tests can show that a pin catches it. The
+ * normal build (ORACLE_MUTANT = 0) plants none. */
+#ifndef ORACLE_MUTANT
+#define ORACLE_MUTANT 0
+#endif
+#define MUTANT(n) (ORACLE_MUTANT == (n))
+
 /* ------------------------------------------------------------------------- */
 /* Number formats                                                             */
 /* ------------------------------------------------------------------------- */
@@ -76,7 +84,7 @@ uint8_t oracle_e4m3_encode(float v) {
     double best_err = a; /* distance to code 0 (value 0) */
     for (int c = 1; c <= 0x7E; ++c) {
         double err = fabs(a - oracle_e4m3_decode((uint8_t)c));
-        if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
+        if (err < best_err || (err == best_err && (MUTANT(10) || ((c & 1) == 0 && (best & 1) == 1)))) {
             best = c;
             best_err = err;
         }
@@ -100,7 +108,7 @@ void oracle_quant_1x128(const float* v, int64_t rows, int64_t cols, uint8_t* q, 
                 float a = fabsf(blk[j]);
                 if (a > amax) amax = a;
             }
-            float sc = (amax == 0.0f) ? 1.0f : amax / 448.0f;
+            float sc = (amax == 0.0f) ? 1.0f : amax / (MUTANT(11) ? 240.0f : 448.0f);
             s[r * nb + b] = sc;
             for (int j = 0; j < 128; ++j) {
                 float t = blk[j] / sc;
@@ -119,12 +127,12 @@ void oracle_quant_1x128(const float* v, int64_t rows, int64_t cols, uint8_t* q, 
  * The gate is clamped from above only. No clamp is L = +inf. alpha = 1, beta = 0 and
  * L = +inf is the standard silu(gate) * up ([P4] "Compatibility"). */
 double oracle_swiglu(double gate, double up, double alpha, double beta, double limit) {
-    double g = gate < limit ? gate : limit;
+    double g = (gate < limit || MUTANT(3)) ? gate : limit;
     double u = up;
     if (u > limit) u = limit;
-    if (u < -limit) u = -limit;
-    double sig = 1.0 / (1.0 + exp(-alpha * g));
-    return g * sig * (u + beta);
+    if (u < -limit && !MUTANT(4)) u = -limit;
+    double sig = 1.0 / (1.0 + exp((MUTANT(5) ? 1.0 : -1.0) * alpha * g));
+    return g * sig * (u + (MUTANT(6) ? 0.0 : beta));
 }
 
 /* ------------------------------------------------------------------------- */
@@ -167,25 +175,36 @@ static void route_row(const float* row, const float* bias, int N, int S, int k, 
         for (int e = 0; e < N; ++e) {
             if (taken[e]) continue;
             /* strictly greater keeps the lower id on ties, since e increases */
-            if (best < 0 || route_key(row, bias, e) > route_key(row, bias, best)) best = e;
+            if (best < 0 || route_key(row, bias, e) > route_key(row, bias, best) ||
+                (MUTANT(1) && route_key(row, bias, e) == route_key(row, bias, best)))
+                best = e;
         }
         taken[best] = 1;
         ids[j] = best;
-        lsel[j] = (double)row[best];
+        lsel[j] = MUTANT(2) ? 1.0 / (1.0 + exp(-(double)row[best])) : (double)row[best];
+        if (MUTANT(20) && bias) lsel[j] += (double)bias[best];
     }
     int n = k;
     if (score == 1) {
         for (int j = 0; j < k; ++j) lsel[j] = logsigmoid(lsel[j]);
         for (int s = 0; s < S; ++s) lsel[n++] = logsigmoid((double)row[N + s]);
     }
+    const int n_lse = MUTANT(7) ? k : n;
     double m = lsel[0];
-    for (int j = 1; j < n; ++j) if (lsel[j] > m) m = lsel[j];
+    for (int j = 1; j < n_lse; ++j) if (lsel[j] > m) m = lsel[j];
     double acc = 0.0;
-    for (int j = 0; j < n; ++j) acc += exp(lsel[j] - m);
+    for (int j = 0; j < n_lse; ++j) acc += exp(lsel[j] - m);
+    if (MUTANT(8) && score == 0)
+        for (int e = 0; e < N; ++e) {
+            int sel = 0;
+            for (int j = 0; j < k; ++j) sel |= ids[j] == e;
+            if (!sel) acc += exp((double)row[e] - m);
+        }
     double lse = m + log(acc);
-    for (int j = 0; j < k; ++j) w[j] = exp(lsel[j] - lse) * route_scale;
+    const double rs = MUTANT(15) ? 1.0 : route_scale;
+    for (int j = 0; j < k; ++j) w[j] = exp(lsel[j] - lse) * rs;
     if (score == 1)
-        for (int s = 0; s < S; ++s) shared_w[s] = exp(lsel[k + s] - lse) * route_scale;
+        for (int s = 0; s < S; ++s) shared_w[s] = exp(lsel[k + s] - lse) * rs;
     free(taken);
     free(lsel);
 }
@@ -243,7 +262,8 @@ int oracle_permute(const int32_t* ids, int T, int k, int E, int n_shared,
     for (int g = 0; g < G; ++g) offsets[g + 1] = offsets[g] + (int32_t)count[g];
     int32_t* cursor = (int32_t*)malloc(sizeof(int32_t) * (size_t)G);
     for (int g = 0; g < G; ++g) cursor[g] = offsets[g];
-    for (int t = 0; t < T; ++t) {
+    for (int tt = 0; tt < T; ++tt) {
+        const int t = MUTANT(9) ? T - 1 - tt : tt;
         for (int j = 0; j < k; ++j) {
             int e = ids[(int64_t)t * k + j];
             int32_t r = cursor[e]++;
@@ -300,7 +320,7 @@ static double round_bf16(double v) {
  * product has at most 12 significant bits, so it is exact before that rounding). */
 double oracle_int4_at(const uint8_t* packed, const uint16_t* scale, int64_t K, int64_t row, int64_t col) {
     uint8_t b = packed[row * (K / 2) + col / 2];
-    int n = (col & 1) ? (b >> 4) : (b & 0xF);
+    int n = ((col & 1) != MUTANT(13)) ? (b >> 4) : (b & 0xF);
     double s = oracle_bf16_to_double(scale[row * (K / 32) + col / 32]);
     return round_bf16((double)(n - 8) * s);
 }
@@ -314,11 +334,11 @@ static double w1_at(const oracle_layer* L, int e, int64_t row, int64_t col) {
                               col);
     int64_t nbr = 2 * L->I / 128, nbc = L->H / 128;
     double s = ((const float*)L->w1_scale)[((int64_t)e * nbr + row / 128) * nbc + col / 128];
-    return oracle_e4m3_decode(((const uint8_t*)L->w1)[idx]) * s;
+    return oracle_e4m3_decode(((const uint8_t*)L->w1)[idx]) * (MUTANT(12) ? 1.0 : s);
 }
 
 static double w2_at(const oracle_layer* L, int e, int64_t row, int64_t col) {
-    int64_t idx = ((int64_t)e * L->H + row) * L->I + col;
+    int64_t idx = MUTANT(18) ? ((int64_t)e * L->I + col) * L->H + row : ((int64_t)e * L->H + row) * L->I + col;
     if (L->wdtype == 0) return oracle_bf16_to_double(((const uint16_t*)L->w2)[idx]);
     if (L->wdtype == 2)
         return oracle_int4_at((const uint8_t*)L->w2, (const uint16_t*)L->w2_scale, L->I, (int64_t)e * L->H + row, col);
@@ -333,14 +353,20 @@ static double w2_at(const oracle_layer* L, int e, int64_t row, int64_t col) {
 static void expert_gemm1(const oracle_layer* L, int e, const double* xv, double* h) {
     double sg = L->gate_scale ? (double)L->gate_scale[e] : 1.0;
     double su = L->up_scale ? (double)L->up_scale[e] : 1.0;
+    if (MUTANT(17)) {
+        const double t = sg;
+        sg = su;
+        su = t;
+    }
     /* the clamp limit may be one fp32 value per expert (sglang PR #39920, "Speed Tests
      * and Profiling": a per-expert fp32 tensor materialised at weight-load time) */
-    double lim = L->limits ? (double)L->limits[e] : L->limit;
+    double lim = (L->limits && !MUTANT(16)) ? (double)L->limits[e] : L->limit;
+    const int64_t gr = MUTANT(19) ? L->I : 0, ur = MUTANT(19) ? 0 : L->I;  /* gate / up row offsets */
     for (int64_t i = 0; i < L->I; ++i) {
         double gate = 0.0, up = 0.0;
         for (int64_t c = 0; c < L->H; ++c) {
-            gate += xv[c] * w1_at(L, e, i, c);
-            up += xv[c] * w1_at(L, e, L->I + i, c);
+            gate += xv[c] * w1_at(L, e, gr + i, c);
+            up += xv[c] * w1_at(L, e, ur + i, c);
         }
         h[i] = oracle_swiglu(sg * gate, su * up, L->alpha, L->beta, lim);
     }
@@ -408,7 +434,7 @@ int oracle_moe_rows(const oracle_layer* L, const int32_t* tokens, int n_tok, dou
             for (int64_t c = 0; c < L->H; ++c) o[c] += w[j] * y[c];
         }
         for (int s = 0; s < L->n_shared; ++s) {
-            double gamma = (S > 0) ? sw[s] : 1.0;
+            double gamma = (S > 0 && !MUTANT(14)) ? sw[s] : 1.0;
             expert_mlp(L, L->E + s, xv, y);
             for (int64_t c = 0; c < L->H; ++c) o[c] += gamma * y[c];
         }
