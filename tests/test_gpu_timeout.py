@@ -1,0 +1,70 @@
+"""Failure detection on the GPU without a fault: a wait that can never complete runs out,
+the kernel records MOE_ERR_TIMEOUT in the workspace's status word and returns, and the
+context stays usable.
+
+The planted failure is a flag that nothing sets: the experts workspace's per-block GEMM1
+completion counters (the first words after the 256-byte header) start a million below
+zero, so the GEMM1 tiles' release-adds never bring them to the count the GEMM2 tiles wait
+for. Each GEMM2 tile's bounded wait (about a second) gives up, its CTA drains its copies
+and MMAs, frees tensor memory and leaves. No trap, no invalid address: the same workspace
+then runs the layer normally."""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import grouped_gemm_swiglu_b200 as moe
+from grouped_gemm_swiglu_b200 import workloads as W
+from helpers import assert_bf16_close, oracle_layer
+
+pytestmark = pytest.mark.gpu
+
+HEADER = 256        # workspace header bytes (status word and counters)
+MOE_ERR_TIMEOUT = -6
+
+
+def test_a_wait_that_never_completes_reports_timeout_and_the_context_survives():
+    wl = W.WORKLOADS["tiny"]
+    inp = W.make_inputs(wl, "cuda")
+    d = moe.MoeDims.of(wl)
+    T, k, A, G, H, I = wl.T, wl.k, d.A, d.G, wl.H, wl.I
+    dev = "cuda"
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    tw = torch.empty((T, k), dtype=torch.float32, device=dev)
+    offsets = torch.empty((G + 1,), dtype=torch.int32, device=dev)
+    perm = torch.empty((A,), dtype=torch.int32, device=dev)
+    inv = torch.empty((T, k), dtype=torch.int32, device=dev)
+    xp = torch.empty((A, H), dtype=torch.bfloat16, device=dev)
+    h = torch.empty((A, I), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((A, H), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    ws_p = moe.alloc_workspace(d, moe.MOE_WS_PERMUTE)
+    ws_e = moe.alloc_workspace(d, moe.MOE_WS_EXPERTS)
+    ws_c = moe.alloc_workspace(d, moe.MOE_WS_COMBINE)
+    moe.moe_route_topk(inp["logits"], d, None, ids, tw)
+    moe.moe_permute(ids, inp["x"], d, offsets, perm, inv, xp, None, ws_p)
+    torch.cuda.synchronize()
+    assert moe.moe_read_status(ws_p) == 0
+
+    nblk_max = min(A, G) + A // 16 + 1  # block counters the workspace holds for these sizes
+    counters = ws_e[HEADER:HEADER + 4 * nblk_max].view(torch.int32)
+    counters.fill_(-1_000_000)
+    args = (inp["w1"], None, None, None, None, inp["w2"], None)
+    t0 = time.perf_counter()
+    moe.moe_experts(xp, None, offsets, *args, d, h, None, y, ws_e)  # the launch itself succeeds
+    torch.cuda.synchronize()
+    waited = time.perf_counter() - t0
+    assert moe.moe_read_status(ws_e) == MOE_ERR_TIMEOUT
+    assert waited < 60.0
+
+    # the context and the workspace are usable again (the test undoes its own planting:
+    # counters past the launch's token blocks are not the kernel's to reset)
+    counters.zero_()
+    moe.moe_clear_status(ws_e)
+    moe.moe_experts(xp, None, offsets, *args, d, h, None, y, ws_e)
+    moe.moe_combine(y, offsets, inv, tw, None, d, out, ws_c)
+    torch.cuda.synchronize()
+    assert moe.moe_read_status(ws_e) == 0 and moe.moe_read_status(ws_c) == 0
+    ref = oracle_layer(wl, inp).moe_rows(np.arange(T, dtype=np.int32))
+    assert_bf16_close(out.float().cpu().numpy(), ref, "after a timed-out launch")
