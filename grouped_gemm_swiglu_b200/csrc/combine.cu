@@ -3,9 +3,10 @@
 // to bf16 (slot-specific routing-weight reduction with fp32 accumulation, batchgen
 // PR #239 commit notes; shared-sink weights gamma from sglang PR #36385 item 3).
 //
-// One thread per 8 output columns (16 bytes) of one token; blockIdx.x is the token, so
-// every thread issues its k + n_shared row loads back to back and the kernel runs at
-// the memory system's rate instead of one dependent load chain per warp.
+// One CTA per token, one thread per 8 output columns (16 bytes) at a time: the token's
+// source rows and weights are looked up once, and each thread issues the loads of eight
+// rows back to back (predicated, no branch) before it accumulates them in slot order, so
+// the kernel runs at the memory system's rate instead of one dependent chain per row.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -13,7 +14,8 @@
 
 namespace moe {
 
-constexpr int kCombineThreads = 128;
+constexpr int kCombineThreads = 256;
+constexpr int kCombineBatch = 8;  // row loads in flight per thread
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const uint16_t* __restrict__ y, const int32_t* __restrict__ offsets, const int32_t* __restrict__ inv,
@@ -44,39 +46,45 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
         s_w[d] = wt;
     }
     __syncthreads();
-    const int v = blockIdx.y * blockDim.x + threadIdx.x;
-    if (v >= H / 8) return;
-    float acc[8];
+    for (int v = threadIdx.x; v < H / 8; v += blockDim.x) {
+        float acc[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll 4
-    for (int d = 0; d < nd; ++d) {
-        const int R = s_row[d];
-        if (R < 0) continue;
-        const float W = s_w[d];
-        const uint4 yv = __ldg(reinterpret_cast<const uint4*>(y + (size_t)R * H) + v);
-        const uint32_t wv[4] = {yv.x, yv.y, yv.z, yv.w};
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        for (int d0 = 0; d0 < nd; d0 += kCombineBatch) {
+            uint4 yv[kCombineBatch];
+#pragma unroll
+            for (int b = 0; b < kCombineBatch; ++b) {  // all loads first; missing rows read as zero
+                const int d = d0 + b;
+                const int R = d < nd ? s_row[d] : -1;
+                yv[b] = R >= 0 ? __ldg(reinterpret_cast<const uint4*>(y + (size_t)R * H) + v) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int b = 0; b < kCombineBatch; ++b) {  // then the sums, in slot order
+                const int d = d0 + b;
+                const float W = (d < nd && s_row[d] >= 0) ? s_w[d] : 0.f;
+                const uint32_t wv[4] = {yv[b].x, yv[b].y, yv[b].z, yv[b].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    acc[2 * i] = fmaf(W, __uint_as_float(wv[i] << 16), acc[2 * i]);
+                    acc[2 * i + 1] = fmaf(W, __uint_as_float(wv[i] & 0xFFFF0000u), acc[2 * i + 1]);
+                }
+            }
+        }
+        uint32_t o[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            acc[2 * i] = fmaf(W, __uint_as_float(wv[i] << 16), acc[2 * i]);
-            acc[2 * i + 1] = fmaf(W, __uint_as_float(wv[i] & 0xFFFF0000u), acc[2 * i + 1]);
+            const __nv_bfloat162 p = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+            o[i] = *reinterpret_cast<const uint32_t*>(&p);
         }
+        reinterpret_cast<uint4*>(out + (size_t)t * H)[v] = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    uint32_t o[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 p = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-        o[i] = *reinterpret_cast<const uint32_t*>(&p);
-    }
-    reinterpret_cast<uint4*>(out + (size_t)t * H)[v] = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 cudaError_t launch_combine(const void* y, const int32_t* offsets, const int32_t* inv, const float* topk_w,
                            const float* shared_w, int T, int H, int k, int E, int n_shared, int n_sink, int64_t A,
                            void* out, int* status, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    dim3 grid(T, (H / 8 + kCombineThreads - 1) / kCombineThreads);
-    return launch_pdl(combine_kernel, grid, dim3(kCombineThreads), 0, stream, static_cast<const uint16_t*>(y), offsets,
+    return launch_pdl(combine_kernel, dim3(T), dim3(kCombineThreads), 0, stream, static_cast<const uint16_t*>(y), offsets,
                       inv, topk_w, shared_w, T, H, k, E, n_shared, n_sink, A, static_cast<uint16_t*>(out), status);
 }
 

@@ -17,7 +17,7 @@ namespace moe {
 
 constexpr int kChunk = 256;          // tokens per counting chunk (8 warps x 32 lanes)
 constexpr int kMaxGroups = 1024 + 32;
-constexpr int kScatterThreads = 128;
+constexpr int kScatterThreads = 256;
 
 size_t permute_scratch_bytes(int T, int k, int E) {
     const size_t nchunk = (size_t)(T + kChunk - 1) / kChunk;
@@ -133,9 +133,9 @@ __global__ void __launch_bounds__(256) permute_count_kernel(const int32_t* __res
     if (threadIdx.x == 0) *counter = 0u;
 }
 
-// blockIdx.x = token, blockIdx.y = 128 16-byte vectors of its row. Destinations of the
-// token's k routed slots and n_shared shared rows, perm / inv_perm (first column block),
-// and the copy (bf16) or quantised copy (E4M3 + scales) of x[t].
+// blockIdx.x = token: the destinations of its k routed slots and n_shared shared rows
+// are looked up once, perm / inv_perm written, then the CTA streams the row in 16-byte
+// vectors (kScatterThreads at a time): a copy (bf16) or a quantised copy (E4M3 + scales).
 template <bool FP8>
 __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
     const int32_t* __restrict__ ids, const int32_t* __restrict__ rank, const int32_t* __restrict__ base,
@@ -162,52 +162,52 @@ __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
             dst = -1;
         }
         s_dst[d] = (int)dst;
-        if (blockIdx.y == 0) {
-            if (d < k) inv[(size_t)t * k + d] = (int)dst;
-            if (dst >= 0) perm[dst] = t;
-        }
+        if (d < k) inv[(size_t)t * k + d] = (int)dst;
+        if (dst >= 0) perm[dst] = t;
     }
     __syncthreads();
     const int nvec = H / 8;
-    const int v = blockIdx.y * blockDim.x + threadIdx.x;
-    const bool act = v < nvec;  // nvec is a multiple of 16: a 128-wide block is all in or all out
-    const uint4 xv = act ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H) + v) : make_uint4(0, 0, 0, 0);
-    if constexpr (!FP8) {
-        if (!act) return;
-        for (int d = 0; d < nd; ++d) {
-            const int D = s_dst[d];
-            if (D >= 0) reinterpret_cast<uint4*>(static_cast<uint16_t*>(x_perm) + (size_t)D * H)[v] = xv;
-        }
-    } else {
-        // 16 threads x 8 values = one 128-wide block: amax, s = amax/448 (1 if 0),
-        // code = E4M3(x/s) with round-to-nearest-even and saturation, all in fp32.
-        float f[8];
-        const uint32_t wv[4] = {xv.x, xv.y, xv.z, xv.w};
+    for (int v0 = 0; v0 < nvec; v0 += blockDim.x) {
+        const int v = v0 + threadIdx.x;
+        const bool act = v < nvec;  // nvec is a multiple of 16: a 128-wide block is all in or all out
+        const uint4 xv = act ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H) + v) : make_uint4(0, 0, 0, 0);
+        if constexpr (!FP8) {
+            if (!act) break;
+            for (int d = 0; d < nd; ++d) {
+                const int D = s_dst[d];
+                if (D >= 0) reinterpret_cast<uint4*>(static_cast<uint16_t*>(x_perm) + (size_t)D * H)[v] = xv;
+            }
+        } else {
+            // 16 threads x 8 values = one 128-wide block: amax, s = amax/448 (1 if 0),
+            // code = E4M3(x/s) with round-to-nearest-even and saturation, all in fp32.
+            float f[8];
+            const uint32_t wv[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            f[2 * i] = __uint_as_float(wv[i] << 16);
-            f[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
-        }
-        float amax = 0.f;
+            for (int i = 0; i < 4; ++i) {
+                f[2 * i] = __uint_as_float(wv[i] << 16);
+                f[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+            }
+            float amax = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
 #pragma unroll
-        for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        if (!act) return;
-        const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
-        uint32_t lo = 0, hi = 0;
+            for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            if (!act) break;
+            const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+            uint32_t lo = 0, hi = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t q = (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(f[i], s), __NV_SATFINITE, __NV_E4M3);
-            if (i < 4) lo |= q << (8 * i);
-            else hi |= q << (8 * (i - 4));
-        }
-        const int blk = v / 16;
-        for (int d = 0; d < nd; ++d) {
-            const int D = s_dst[d];
-            if (D >= 0) {
-                reinterpret_cast<uint2*>(static_cast<uint8_t*>(x_perm) + (size_t)D * H)[v] = make_uint2(lo, hi);
-                if ((threadIdx.x & 15) == 0) x_scale[(size_t)blk * A + D] = s;
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t q = (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(f[i], s), __NV_SATFINITE, __NV_E4M3);
+                if (i < 4) lo |= q << (8 * i);
+                else hi |= q << (8 * (i - 4));
+            }
+            const int blk = v / 16;
+            for (int d = 0; d < nd; ++d) {
+                const int D = s_dst[d];
+                if (D >= 0) {
+                    reinterpret_cast<uint2*>(static_cast<uint8_t*>(x_perm) + (size_t)D * H)[v] = make_uint2(lo, hi);
+                    if ((threadIdx.x & 15) == 0) x_scale[(size_t)blk * A + D] = s;
+                }
             }
         }
     }
@@ -234,8 +234,7 @@ cudaError_t launch_permute(const int32_t* ids, const void* x, int T, int H, int 
                      offsets, counter, status, zero, zero ? zero_words : (size_t)0);
     if (err != cudaSuccess) return err;
     const int64_t A = (int64_t)T * (k + n_shared);
-    dim3 grid(T, (H / 8 + kScatterThreads - 1) / kScatterThreads);
-    return launch_pdl(fp8 ? permute_scatter_kernel<true> : permute_scatter_kernel<false>, grid, dim3(kScatterThreads),
+    return launch_pdl(fp8 ? permute_scatter_kernel<true> : permute_scatter_kernel<false>, dim3(T), dim3(kScatterThreads),
                       0, stream, ids, static_cast<const int32_t*>(rank), static_cast<const int32_t*>(cnt), offsets,
                       static_cast<const uint16_t*>(x), T, H, k, E, n_shared, A, perm, inv, x_perm, x_scale, status);
 }
