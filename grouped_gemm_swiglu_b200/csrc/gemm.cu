@@ -82,7 +82,11 @@ struct Cfg {
     static constexpr int BOX_ROWS = BN < 64 ? BN : 64;
     static constexpr int BOX_BYTES = BOX_ROWS * 128;
     // as many stages as fit next to the control block and the largest group table
-    static constexpr int STAGE_BUDGET = kSmemLimit - 1024 - 8 * (kMaxGroupsGemm + 1) - 1024 - 4 * 16 * 16 * 3;
+    // wide FP8 tile (FP8 at 128 tokens): 2 KB per epilogue warp to turn its token rows into
+    // row-contiguous stores (16 rows x 128 bytes at a time)
+    static constexpr int XPOSE_BYTES = (FP8_ && BN_ >= 128) ? 8 * 2048 : 0;
+    static constexpr int STAGE_BUDGET =
+        kSmemLimit - 1024 - 8 * (kMaxGroupsGemm + 1) - 1024 - 4 * 16 * 16 * 3 - XPOSE_BYTES;
     static constexpr int ACC_COLS = 2 * BN;  // one TMEM buffer: gate | up (GEMM2 uses the first BN)
     // bf16 hands one buffer per tile to the epilogue, FP8 one per 128-deep K block, so
     // FP8 keeps up to four partial buffers in flight.
@@ -121,6 +125,7 @@ struct Cfg {
     static_assert(TMEM_COLS <= 512, "TMEM holds 512 columns");
     static_assert(COLS % CW == 0 && CW >= 4, "column share must be a multiple of the load width");
     static_assert(!FP8 || WIDE || COLS <= 32, "FP8 loads a warp's whole column share at once");
+    static_assert(!WIDE || XPOSE_BYTES == EPI * 2048, "one 2 KB row-staging buffer per epilogue warp");
     static_assert(!WIDE || (BN == 128 && (EPI == 8 || EPI == 16) && COLS % 16 == 0 &&
                             128 * REG_LOW + 32 * EPI * REG_HIGH <= THREADS * REG_LAUNCH &&
                             REG_LOW + (EPI / 4) * REG_HIGH <= 512),
@@ -138,7 +143,7 @@ struct Cfg {
     // epibar, and for INT4 raw_full per stage (packed bytes and token rows landed)
     static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 2 * kRing + 2 + (INT4 ? STAGES : 0) + (WIDE ? 1 : 0);
     static constexpr size_t ctrl_bytes() {
-        return 8 * NUM_BARS + 16 + 4 * kRing + 16 + 4 * RED_FLOATS + 16 + 4 * SCT_FLOATS;
+        return 8 * NUM_BARS + 16 + 4 * kRing + 16 + 4 * RED_FLOATS + 16 + 4 * SCT_FLOATS + 16 + XPOSE_BYTES;
     }
     static size_t smem_bytes(int G) {  // + block table and clamped offsets, G+1 ints each
         return 1024 + (size_t)STAGES * STAGE_BYTES + ctrl_bytes() + 8 * (size_t)(G + 1) + 16;
@@ -318,6 +323,40 @@ __device__ __forceinline__ void dequant_int4_row(const uint8_t* raw, uint32_t sc
     }
 }
 
+// Row-contiguous stores of a warp's 32 token rows: lane i holds NV 16-byte pieces of row
+// i (its row = base + (row0 + i) * ld, pieces consecutive). Sixteen rows at a time go
+// through the warp's 2 KB buffer (16 rows x 128 bytes, the piece index XOR-swizzled by the
+// row so neither the writes nor the reads conflict), and come back out with 128 / (16 NV)
+// rows per store instruction and each row's bytes from consecutive lanes. Rows at or past
+// `nrows` (relative to row0) are not stored. NV is 4 or 8.
+template <int NV>
+__device__ __forceinline__ void store_rows(uint8_t* buf, const uint4 (&v)[NV], uint8_t* base, size_t ld, int row0,
+                                           int nrows, int lane) {
+    static_assert(NV == 4 || NV == 8, "a row is 64 or 128 bytes");
+    constexpr int RPI = 32 / NV;  // rows per store instruction
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+        __syncwarp();
+        if ((lane >> 4) == pass) {
+            const int r = lane & 15;
+#pragma unroll
+            for (int c = 0; c < NV; ++c)
+                *reinterpret_cast<uint4*>(buf + r * (NV * 16) + ((c ^ (r & (NV - 1))) * 16)) = v[c];
+        }
+        __syncwarp();
+#pragma unroll
+        for (int it = 0; it < 16 / RPI; ++it) {
+            const int r = it * RPI + lane / NV, c = lane % NV;
+            const int row = pass * 16 + r;
+            if (row < nrows) {
+                const uint4 val = *reinterpret_cast<const uint4*>(buf + r * (NV * 16) + ((c ^ (r & (NV - 1))) * 16));
+                *reinterpret_cast<uint4*>(base + (size_t)(row0 + row) * ld + c * 16) = val;
+            }
+        }
+    }
+    __syncwarp();
+}
+
 // Warp-collective bounded wait: lane 0 waits, the verdict is broadcast.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, PipeAbort* ab, int* status) {
     bool ok = true;
@@ -349,7 +388,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     int* ring = reinterpret_cast<int*>(tmem_slot + 4);
     float* red = reinterpret_cast<float*>(ring + kRing + 4);
     float* sct = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(red + C::RED_FLOATS) + 15) & ~uintptr_t(15));
-    int32_t* blk_start = reinterpret_cast<int32_t*>(sct + C::SCT_FLOATS);
+    uint8_t* xpose = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sct + C::SCT_FLOATS) + 15) & ~uintptr_t(15));
+    int32_t* blk_start = reinterpret_cast<int32_t*>(xpose + C::XPOSE_BYTES);
     int32_t* s_off = blk_start + (p.G + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -935,10 +975,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     for (int g = 0; g < C::GROUPS; ++g) amax = fmaxf(amax, rb[g * 128 + tok]);  // the 1x128 block
                     const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
                     const float inv_s = amax == 0.f ? 1.f : __fdividef(448.f, amax);
-                    if (has_tok) {
-                        // h rows and the chunk offset are multiples of 16 bytes (I % 128 == 0,
-                        // h 16-byte aligned), so each 16 codes go out as one vector store
-                        uint8_t* dst = static_cast<uint8_t*>(p.h) + (size_t)(tl.row0 + tok) * p.I + tl.col0 + cg * CC;
+                    {
+                        uint4 hv[CC / 16];  // this token's CC codes
 #pragma unroll
                         for (int v = 0; v < CC / 16; ++v) {
                             uint32_t w[4];
@@ -951,35 +989,33 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                     make_float2(acc0[j + 2] * inv_s, acc0[j + 3] * inv_s), __NV_SATFINITE, __NV_E4M3);
                                 w[t] = lo | (hi << 16);
                             }
-                            *reinterpret_cast<uint4*>(dst + 16 * v) = make_uint4(w[0], w[1], w[2], w[3]);
+                            hv[v] = make_uint4(w[0], w[1], w[2], w[3]);
                         }
-                        if (cg == 0) p.h_scale[(size_t)tl.c * p.A + tl.row0 + tok] = s;
+                        store_rows<CC / 16>(xpose + ew * 2048, hv, static_cast<uint8_t*>(p.h) + tl.col0 + cg * CC,
+                                            (size_t)p.I, tl.row0 + q * 32, tl.nrows - q * 32, lane);
+                        if (has_tok && cg == 0) p.h_scale[(size_t)tl.c * p.A + tl.row0 + tok] = s;
                     }
-                } else if (has_tok) {
-                    // y rows (H % 128 == 0, y 16-byte aligned): 8 bf16 per vector store
-                    __nv_bfloat16* row = static_cast<__nv_bfloat16*>(p.y) + (size_t)(tl.row0 + tok) * p.H;
+                } else {
+                    // y rows (H % 128 == 0, y 16-byte aligned): this token's CC bf16 of each half
+                    uint8_t* ybase = static_cast<uint8_t*>(p.y);
 #pragma unroll
-                    for (int v = 0; v < CC / 8; ++v) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int t = 0; t < 4; ++t) {
-                            const __nv_bfloat162 b = __floats2bfloat162_rn(acc0[v * 8 + 2 * t], acc0[v * 8 + 2 * t + 1]);
-                            w[t] = *reinterpret_cast<const uint32_t*>(&b);
-                        }
-                        *reinterpret_cast<uint4*>(row + tl.col0 + cg * CC + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
-                    }
-                    if (tl.dual) {
+                    for (int half = 0; half < 2; ++half) {
+                        if (half == 1 && !tl.dual) break;
+                        const float* a = half ? acc1 : acc0;
+                        uint4 yv[CC / 8];
 #pragma unroll
                         for (int v = 0; v < CC / 8; ++v) {
                             uint32_t w[4];
 #pragma unroll
                             for (int t = 0; t < 4; ++t) {
-                                const __nv_bfloat162 b =
-                                    __floats2bfloat162_rn(acc1[v * 8 + 2 * t], acc1[v * 8 + 2 * t + 1]);
+                                const __nv_bfloat162 b = __floats2bfloat162_rn(a[v * 8 + 2 * t], a[v * 8 + 2 * t + 1]);
                                 w[t] = *reinterpret_cast<const uint32_t*>(&b);
                             }
-                            *reinterpret_cast<uint4*>(row + tl.col1 + cg * CC + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
+                            yv[v] = make_uint4(w[0], w[1], w[2], w[3]);
                         }
+                        const int colb = (half ? tl.col1 : tl.col0) + cg * CC;  // first bf16 column
+                        store_rows<CC / 8>(xpose + ew * 2048, yv, ybase + 2 * (size_t)colb, 2 * (size_t)p.H,
+                                           tl.row0 + q * 32, tl.nrows - q * 32, lane);
                     }
                 }
             } else {
