@@ -24,6 +24,7 @@ _LIB = os.environ.get("ORACLE_LIB") or os.path.join(_HERE, "liboracle.so")
 WDTYPE_BF16 = 0
 WDTYPE_FP8 = 1
 WDTYPE_INT4 = 2
+WDTYPE_NVFP4 = 3
 SCORE_SOFTMAX = 0
 SCORE_SIGMOID = 1
 
@@ -73,6 +74,11 @@ def _load():
         lib.oracle_gate_logits.restype = ctypes.c_int
         lib.oracle_gate_logits.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, ctypes.c_void_p]
+        lib.oracle_e2m1_decode.restype = ctypes.c_double
+        lib.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_fp4_at.restype = ctypes.c_double
+        lib.oracle_fp4_at.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                      ctypes.c_int64]
         lib.oracle_int4_at.restype = ctypes.c_double
         lib.oracle_int4_at.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                                        ctypes.c_int64]
@@ -189,6 +195,23 @@ def int4_dequant(packed, scale_bits):
     return out
 
 
+def e2m1_decode(code: int) -> float:
+    return _load().oracle_e2m1_decode(int(code))
+
+
+def fp4_dequant(packed, scale_codes):
+    """NVFP4 weights: packed uint8 [rows, K/2], E4M3 scale codes uint8 [rows, K/16] -> fp64 [rows, K]."""
+    p = _c(packed, np.uint8)
+    s = _c(scale_codes, np.uint8)
+    rows, K = p.shape[0], p.shape[1] * 2
+    lib = _load()
+    out = np.empty((rows, K), dtype=np.float64)
+    for r in range(rows):
+        for c in range(K):
+            out[r, c] = lib.oracle_fp4_at(_ptr(p), _ptr(s), K, r, c)
+    return out
+
+
 def gate_logits(x_bits, w_bits):
     """Gate GEMV: x bf16 bits [T,H], w bf16 bits [C,H] -> fp64 logits [T,C]."""
     x = _c(x_bits, np.uint16)
@@ -229,7 +252,8 @@ class Layer:
                  route_scale, logits, x, w1, w2, w1_scale=None, w2_scale=None,
                  gate_scale=None, up_scale=None, limits=None, router_bias=None):
         wt = np.uint16 if wdtype == WDTYPE_BF16 else np.uint8
-        st = np.uint16 if wdtype == WDTYPE_INT4 else np.float32  # INT4 group scales are bf16 bits
+        # INT4 group scales are bf16 bits, NVFP4 block scales E4M3 codes
+        st = {WDTYPE_INT4: np.uint16, WDTYPE_NVFP4: np.uint8}.get(wdtype, np.float32)
         self._keep = dict(
             logits=_c(logits, np.float32), x=_c(x, np.uint16), w1=_c(w1, wt), w2=_c(w2, wt),
             w1_scale=_c(w1_scale, st), w2_scale=_c(w2_scale, st),

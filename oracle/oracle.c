@@ -285,7 +285,8 @@ int oracle_permute(const int32_t* ids, int T, int k, int E, int n_shared,
 typedef struct {
     int32_t T, H, I, E, k, n_sink, n_shared;
     int32_t wdtype;               /* 0: bf16 weights; 1: E4M3 with 128x128 fp32 block scales;
-                                     2: INT4 group-32 with bf16 scales (activations bf16) */
+                                     2: INT4 group-32 with bf16 scales (activations bf16);
+                                     3: NVFP4, E2M1 with one E4M3 scale per 16 (activations bf16) */
     int32_t score;                /* 0: softmax renorm; 1: sigmoid + logsigmoid-LSE renorm */
     int32_t pad_;
     double alpha, beta, limit, route_scale;
@@ -293,10 +294,12 @@ typedef struct {
     const uint16_t* x;            /* [T][H] bf16 bits */
     const void* w1;               /* [E+n_shared][2I][H]; rows [0,I) gate, [I,2I) up */
     const void* w1_scale;         /* wdtype 1: fp32 [E+n_shared][2I/128][H/128];
-                                     wdtype 2: bf16 bits [E+n_shared][2I][H/32] */
+                                     wdtype 2: bf16 bits [E+n_shared][2I][H/32];
+                                     wdtype 3: E4M3 codes [E+n_shared][2I][H/16] */
     const void* w2;               /* [E+n_shared][H][I] */
     const void* w2_scale;         /* wdtype 1: fp32 [E+n_shared][H/128][I/128];
-                                     wdtype 2: bf16 bits [E+n_shared][H][I/32] */
+                                     wdtype 2: bf16 bits [E+n_shared][H][I/32];
+                                     wdtype 3: E4M3 codes [E+n_shared][H][I/16] */
     const float* gate_scale;      /* [E+n_shared] or NULL (1.0) */
     const float* up_scale;        /* [E+n_shared] or NULL (1.0) */
     const float* limits;          /* [E+n_shared] clamp per expert, or NULL (limit) */
@@ -325,6 +328,29 @@ double oracle_int4_at(const uint8_t* packed, const uint16_t* scale, int64_t K, i
     return round_bf16((double)(n - 8) * s);
 }
 
+/* E2M1 (the 4-bit element of NVFP4, named on the xorl-wheels FlashInfer 0.6.18 page,
+ * "Changes": NVFP4 checkpoints): 1 sign bit, 2 exponent bits with bias 1, 1 mantissa bit,
+ * no infinities or NaN. Exponent field 0 is subnormal: m * 2^-1; otherwise
+ * (1 + m/2) * 2^(e - 1). */
+double oracle_e2m1_decode(uint8_t code) {
+    int sgn = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double mag = e == 0 ? 0.5 * m : (1.0 + 0.5 * m) * ldexp(1.0, e - (MUTANT(21) ? 2 : 1));
+    return sgn ? -mag : mag;
+}
+
+/* NVFP4 weight element: packed [rows][K/2] bytes (low nibble = even K index, as for INT4),
+ * one E4M3 scale per 16 consecutive K [rows][K/16]; value E2M1(nibble) * E4M3(scale). The
+ * product has at most 6 significant bits and lies in bf16's range, so it enters the MMA
+ * exactly (the rounding below is the identity). The per-expert global scales of NVFP4
+ * checkpoints (gate and up halves separately) are the layer's gate_scale / up_scale. */
+double oracle_fp4_at(const uint8_t* packed, const uint8_t* scale, int64_t K, int64_t row, int64_t col) {
+    uint8_t b = packed[row * (K / 2) + col / 2];
+    uint8_t n = (col & 1) ? (b >> 4) : (b & 0xF);
+    double s = MUTANT(22) ? oracle_e4m3_decode(scale[row * (K / 16) + col / 32])
+                          : oracle_e4m3_decode(scale[row * (K / 16) + col / 16]);
+    return round_bf16(oracle_e2m1_decode(n) * s);
+}
+
 /* Dequantised weight element. */
 static double w1_at(const oracle_layer* L, int e, int64_t row, int64_t col) {
     int64_t idx = ((int64_t)e * 2 * L->I + row) * L->H + col;
@@ -332,6 +358,9 @@ static double w1_at(const oracle_layer* L, int e, int64_t row, int64_t col) {
     if (L->wdtype == 2)
         return oracle_int4_at((const uint8_t*)L->w1, (const uint16_t*)L->w1_scale, L->H, (int64_t)e * 2 * L->I + row,
                               col);
+    if (L->wdtype == 3)
+        return oracle_fp4_at((const uint8_t*)L->w1, (const uint8_t*)L->w1_scale, L->H, (int64_t)e * 2 * L->I + row,
+                             col);
     int64_t nbr = 2 * L->I / 128, nbc = L->H / 128;
     double s = ((const float*)L->w1_scale)[((int64_t)e * nbr + row / 128) * nbc + col / 128];
     return oracle_e4m3_decode(((const uint8_t*)L->w1)[idx]) * (MUTANT(12) ? 1.0 : s);
@@ -342,6 +371,8 @@ static double w2_at(const oracle_layer* L, int e, int64_t row, int64_t col) {
     if (L->wdtype == 0) return oracle_bf16_to_double(((const uint16_t*)L->w2)[idx]);
     if (L->wdtype == 2)
         return oracle_int4_at((const uint8_t*)L->w2, (const uint16_t*)L->w2_scale, L->I, (int64_t)e * L->H + row, col);
+    if (L->wdtype == 3)
+        return oracle_fp4_at((const uint8_t*)L->w2, (const uint8_t*)L->w2_scale, L->I, (int64_t)e * L->H + row, col);
     int64_t nbr = L->H / 128, nbc = L->I / 128;
     double s = ((const float*)L->w2_scale)[((int64_t)e * nbr + row / 128) * nbc + col / 128];
     return oracle_e4m3_decode(((const uint8_t*)L->w2)[idx]) * s;

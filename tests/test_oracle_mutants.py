@@ -39,6 +39,8 @@ MUTANTS = [
     (19, "gate and up halves of W1 swapped", "test_layer_single_expert_is_dense_swiglu_mlp"),
     (20, "correction bias added to the weights, not only the ranking",
      "test_route_dominant_bias_forces_the_selection_and_not_the_weights"),
+    (21, "E2M1 exponent bias 2 instead of 1", "test_e2m1_decode_all_codes_match_ml_dtypes"),
+    (22, "NVFP4 block scale per 32 weights instead of 16", "test_fp4_dequant_follows_the_nibble_order_and_block_scale"),
 ]
 
 

@@ -562,3 +562,72 @@ def test_layer_int4_equals_bf16_layer_with_dequantised_weights():
     w2b = np.stack([_torch_int4_dequant(w2p[g], w2s[g]).view(torch.int16).numpy().view(np.uint16) for g in range(G)])
     b = oracle.Layer(**common, wdtype=oracle.WDTYPE_BF16, w1=w1b, w2=w2b)
     np.testing.assert_array_equal(q.moe_rows(np.arange(T)), b.moe_rows(np.arange(T)))
+
+
+# ------------------------------------------------------------------ NVFP4 weights
+# E2M1 elements with one E4M3 scale per 16 along K (the NVFP4 checkpoints of the
+# xorl-wheels FlashInfer 0.6.18 page, "Changes"); ml_dtypes implements both element
+# formats independently of the oracle.
+
+def _ml_fp4_dequant(packed, scale_codes):
+    """packed uint8 [rows, K/2] (low nibble = even K), E4M3 codes [rows, K/16] -> bf16 bits
+    of E2M1 * E4M3 (exact in bf16), computed with ml_dtypes and torch."""
+    import ml_dtypes
+    n = np.stack([packed & 0xF, packed >> 4], axis=-1).reshape(packed.shape[0], -1)
+    v = n.astype(np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    s = scale_codes.view(ml_dtypes.float8_e4m3fn).astype(np.float64).repeat(16, axis=1)
+    w = torch.from_numpy(v * s).to(torch.bfloat16)
+    assert torch.equal(w.double(), torch.from_numpy(v * s))  # exact: at most 6 significant bits
+    return w.view(torch.int16).numpy().view(np.uint16)
+
+
+def test_e2m1_decode_all_codes_match_ml_dtypes():
+    import ml_dtypes
+    ref = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    got = np.array([oracle.e2m1_decode(c) for c in range(16)])
+    np.testing.assert_array_equal(got, ref)
+    assert np.array_equal(np.signbit(got), np.signbit(ref))
+
+
+def _finite_e4m3_codes(rng, shape, lo=0x20, hi=0x48):
+    """positive finite E4M3 codes (no NaN pattern), exponents around 2^-4 .. 2^1"""
+    return rng.integers(lo, hi, shape, dtype=np.uint8)
+
+
+def test_fp4_dequant_follows_the_nibble_order_and_block_scale():
+    rng = np.random.default_rng(51)
+    packed = rng.integers(0, 256, (6, 64), dtype=np.uint8)  # K = 128: 8 blocks of 16
+    scales = _finite_e4m3_codes(rng, (6, 8))
+    packed[0, 0] = 0x2F  # K 0: low nibble 0xF = -6, K 1: high nibble 0x2 = +1
+    got = oracle.fp4_dequant(packed, scales)
+    ref = _bf16_val(_ml_fp4_dequant(packed, scales))
+    np.testing.assert_array_equal(got, ref)
+    import ml_dtypes
+    s0 = float(np.array([scales[0, 0]], np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)[0])
+    assert got[0, 0] == -6 * s0 and got[0, 1] == 1 * s0
+    # the scale of K 16..31 is the second code of the row
+    s1 = float(np.array([scales[2, 1]], np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)[0])
+    b = packed[2, 8]
+    assert got[2, 16] == float(np.array([b & 0xF], np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)[0]) * s1
+
+
+def test_layer_nvfp4_equals_bf16_layer_with_dequantised_weights():
+    # with per-expert gate/up global scales (the NVFP4 checkpoints' g1_alphas / g1_alphas_up)
+    rng = np.random.default_rng(52)
+    T, H, I, E, k, S = 6, 128, 64, 4, 2, 1
+    G = E + S
+    w1p = rng.integers(0, 256, (G, 2 * I, H // 2), dtype=np.uint8)
+    w2p = rng.integers(0, 256, (G, H, I // 2), dtype=np.uint8)
+    w1s = _finite_e4m3_codes(rng, (G, 2 * I, H // 16), 0x10, 0x30)
+    w2s = _finite_e4m3_codes(rng, (G, H, I // 16), 0x10, 0x30)
+    gs = rng.uniform(0.5, 1.3, G).astype(np.float32)
+    us = rng.uniform(0.5, 1.3, G).astype(np.float32)
+    x = _bf16_bits(rng.normal(0, 1, (T, H)))
+    logits = rng.normal(0, 1, (T, E)).astype(np.float32)
+    common = dict(T=T, H=H, I=I, E=E, k=k, n_sink=0, n_shared=S, score=oracle.SCORE_SOFTMAX, alpha=1.702, beta=1.0,
+                  limit=7.0, route_scale=1.0, logits=logits, x=x, gate_scale=gs, up_scale=us)
+    q = oracle.Layer(**common, wdtype=oracle.WDTYPE_NVFP4, w1=w1p, w2=w2p, w1_scale=w1s, w2_scale=w2s)
+    w1b = np.stack([_ml_fp4_dequant(w1p[g], w1s[g]) for g in range(G)])
+    w2b = np.stack([_ml_fp4_dequant(w2p[g], w2s[g]) for g in range(G)])
+    b = oracle.Layer(**common, wdtype=oracle.WDTYPE_BF16, w1=w1b, w2=w2b)
+    np.testing.assert_array_equal(q.moe_rows(np.arange(T)), b.moe_rows(np.arange(T)))
