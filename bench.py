@@ -197,7 +197,8 @@ def workload_of(args):
 def config_of(wl):
     return {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "top_k": wl.k,
             "n_sink": wl.n_sink, "n_shared": wl.n_shared,
-            "weights": {1: "fp8_e4m3_block128", 2: "int4_group32_bf16_scales"}.get(wl.wdtype, "bf16"),
+            "weights": {1: "fp8_e4m3_block128", 2: "int4_group32_bf16_scales",
+                        3: "nvfp4_e2m1_e4m3_scales_per16"}.get(wl.wdtype, "bf16"),
             "score": "sigmoid_logsigmoid_lse" if wl.score == 1 else "softmax_renorm",
             "alpha": wl.alpha, "beta": wl.beta, "limit": None if math.isinf(wl.limit) else wl.limit,
             "seed": wl.seed, "l2": "flushed between timed steps (512 MiB write, outside the timed events)"}
@@ -433,8 +434,8 @@ def run_ours(args):
     used = int(((off[1:] - off[:-1]) > 0).sum())
     hbm, bf16_tf, peak_src = peaks()
     elt = 1 if fp8 else 2  # activations (x_perm, h)
-    int4 = wl.wdtype == 2
-    welt = 0.5 + 2.0 / 32 if int4 else elt  # weight bytes per element (INT4: a nibble + a bf16 scale per 32)
+    # weight bytes per element: INT4 a nibble + a bf16 scale per 32; NVFP4 a nibble + an E4M3 scale per 16
+    welt = {2: 0.5 + 2.0 / 32, 3: 0.5 + 1.0 / 16}.get(wl.wdtype, elt)
     H_, I_ = wl.H, wl.I
     flops = 2.0 * A * H_ * 2 * I_ + 2.0 * A * I_ * H_
     nbytes = used * 3 * I_ * H_ * welt + A * H_ * elt + 2 * A * I_ * elt + A * H_ * 2

@@ -23,7 +23,7 @@ STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED
 MOE_WS_PERMUTE, MOE_WS_GEMM1, MOE_WS_GEMM2_COMBINE, MOE_WS_FORWARD, MOE_WS_EXPERTS, MOE_WS_COMBINE = 0, 1, 2, 3, 4, 5
 MOE_WS_GATE_ROUTE = 6
 MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
-MOE_WDTYPE_BF16, MOE_WDTYPE_FP8_E4M3_BLOCK128 = 0, 1
+MOE_WDTYPE_BF16, MOE_WDTYPE_FP8_E4M3_BLOCK128, MOE_WDTYPE_INT4_G32, MOE_WDTYPE_NVFP4 = 0, 1, 2, 3
 
 
 class MoeError(RuntimeError):

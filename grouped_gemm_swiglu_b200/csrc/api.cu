@@ -25,7 +25,8 @@ int check_dims(const moe_dims* d) {
     if (d->n_sink < 0 || d->k + d->n_sink > kMaxSlots) return MOE_ERR_INVALID_ARG;
     if (d->n_shared < 0 || d->k + d->n_shared > kMaxSlots) return MOE_ERR_INVALID_ARG;
     if (d->score != MOE_SCORE_SOFTMAX && d->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
-    if (d->wdtype != MOE_WDTYPE_BF16 && d->wdtype != MOE_WDTYPE_FP8_E4M3_BLOCK128 && d->wdtype != MOE_WDTYPE_INT4_G32)
+    if (d->wdtype != MOE_WDTYPE_BF16 && d->wdtype != MOE_WDTYPE_FP8_E4M3_BLOCK128 && d->wdtype != MOE_WDTYPE_INT4_G32 &&
+        d->wdtype != MOE_WDTYPE_NVFP4)
         return MOE_ERR_INVALID_ARG;
     if (d->n_sink > 0 && d->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
     if (d->n_sink > 0 && d->n_shared > 0 && d->n_shared != d->n_sink) return MOE_ERR_INVALID_ARG;
@@ -55,7 +56,9 @@ int64_t rows_A(const moe_dims* d) { return (int64_t)d->T * (d->k + d->n_shared);
 int groups(const moe_dims* d) { return d->E + d->n_shared; }
 size_t act_elt(const moe_dims* d) { return d->wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128 ? 1 : 2; }
 bool is_fp8(const moe_dims* d) { return d->wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128; }
-bool is_int4(const moe_dims* d) { return d->wdtype == MOE_WDTYPE_INT4_G32; }
+// 4-bit weights (INT4 group-32 or NVFP4): packed bytes, per-row scales read one 32-bit
+// word per 64-deep K step, bf16 activations
+bool is_int4(const moe_dims* d) { return d->wdtype == MOE_WDTYPE_INT4_G32 || d->wdtype == MOE_WDTYPE_NVFP4; }
 
 // Sub-buffers of a workspace, as byte offsets from its start.
 struct Layout {
@@ -138,7 +141,8 @@ MoeGemmArgs gemm_args(const moe_dims* d, const int32_t* offsets, int* status) {
     a.H = d->H;
     a.I = d->I;
     a.fp8 = is_fp8(d);
-    a.int4 = d->wdtype == MOE_WDTYPE_INT4_G32;
+    a.int4 = is_int4(d);
+    a.fp4 = d->wdtype == MOE_WDTYPE_NVFP4;
     a.alpha = d->alpha;
     a.beta = d->beta;
     a.limit = d->limit;

@@ -156,8 +156,9 @@ struct DevArgs {
     int c1;      // GEMM1 tiles per token block: I/128 (0 = phase absent)
     int c2;      // GEMM2 tiles per token block: ceil(H/256), each two 128-row chunks of H (0 = absent)
     const float* x_scale;   // FP8: [H/128][A]
-    const void* w1_scale;   // FP8: fp32 [G][2I/128][H/128]; INT4: bf16 [G][2I][H/32]
-    const void* w2_scale;   // FP8: fp32 [G][H/128][I/128]; INT4: bf16 [G][H][I/32]
+    const void* w1_scale;   // FP8: fp32 [G][2I/128][H/128]; INT4: bf16 [G][2I][H/32]; NVFP4: E4M3 [G][2I][H/16]
+    const void* w2_scale;   // FP8: fp32 [G][H/128][I/128]; INT4: bf16 [G][H][I/32]; NVFP4: E4M3 [G][H][I/16]
+    int fp4;                // 4-bit weights are NVFP4 (else INT4 group-32)
     const float* gate_scale;
     const float* up_scale;
     float alpha, beta, limit;
@@ -355,6 +356,59 @@ __device__ __forceinline__ void store_rows(uint8_t* buf, const uint4 (&v)[NV], u
         }
     }
     __syncwarp();
+}
+
+// NVFP4 dequantisation of one 64-deep weight row segment: 32 packed bytes (low nibble =
+// even K) of E2M1 values (1 sign, 2 exponent bits with bias 1, 1 mantissa bit), one E4M3
+// scale per 16 K (`sc` holds the segment's four scale bytes, K 0-15 in the low byte). The
+// E2M1 magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 are bf16 values whose high and low bytes are
+// two 8-entry byte tables: one byte permute looks up four values' high (or low) bytes at
+// once, two more interleave them into bf16 pairs, and a fourth gathers the pair's two sign
+// bits into bits 15 and 31. The product with the bf16 scale is exact (at most 6
+// significant bits), so the tile holds exactly E2M1 * E4M3.
+//   q: one packed word (K 8w .. 8w+7); out[b]: the bf16 pair of its byte b.
+__device__ __forceinline__ void fp4_word_bf16(uint32_t q, __nv_bfloat162 s, uint32_t* out) {
+    // bf16 bits of the magnitudes, split into high and low bytes (entries 0-3, 4-7)
+    constexpr uint32_t kHi03 = 0x3F3F3F00u, kHi47 = 0x40404040u;
+    constexpr uint32_t kLo03 = 0xC0800000u, kLo47 = 0xC0804000u;
+    const uint32_t m = q & 0x77777777u;  // magnitude codes, one per nibble
+    const uint32_t t = q << 4;           // bit 7 of byte b: the sign of byte b's even-K value
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {  // values 0-3, then 4-7 (the selector takes 4 nibbles)
+        const uint32_t sel = h ? (m >> 16) : m;
+        const uint32_t hi = byte_perm(kHi03, kHi47, sel);
+        const uint32_t lo = byte_perm(kLo03, kLo47, sel);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const uint32_t b = 2 * h + j;  // the packed byte this pair comes from
+            uint32_t u = byte_perm(lo, hi, j ? 0x7362u : 0x5140u);  // lo hi lo hi: two bf16
+            // bytes 1 and 3 of the sign word: byte b of t (even value), byte b of q (odd value)
+            const uint32_t sg = byte_perm(t, q, b * 0x111u | ((4u + b) << 12));
+            u |= sg & 0x80008000u;
+            __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&u);
+            v = __hmul2(v, s);
+            out[b] = *reinterpret_cast<const uint32_t*>(&v);
+        }
+    }
+}
+
+__device__ __forceinline__ void dequant_fp4_row(const uint8_t* raw, uint32_t sc, uint32_t* out) {
+    // the four E4M3 scales to bf16, two per conversion (every E4M3 value is exact in f16 and bf16)
+    __nv_bfloat162 sb[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const __half2 h2 = __half2(__nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)((sc >> (16 * i)) & 0xFFFFu),
+                                                              __NV_E4M3));
+        sb[i] = __float22bfloat162_rn(__half22float2(h2));
+    }
+    const uint4 q0 = *reinterpret_cast<const uint4*>(raw);
+    const uint4 q1 = *reinterpret_cast<const uint4*>(raw + 16);
+    const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {  // 16 K per scale: two words per scale
+        const __nv_bfloat16 s1 = (w & 2) ? sb[w >> 2].y : sb[w >> 2].x;
+        fp4_word_bf16(qw[w], __halves2bfloat162(s1, s1), out + 4 * w);
+    }
 }
 
 // Warp-collective bounded wait: lane 0 waits, the verdict is broadcast.
@@ -678,7 +732,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const int all_kb = K / C::BK;
             const int kbase = g1 ? tl.ks * all_kb / p.s1 : 0;
             const int num_kb = g1 ? (tl.ks + 1) * all_kb / p.s1 - kbase : all_kb;
-            // this row's bf16 group scales: [rows][K/32], two groups (one 32-bit word) per stage
+            // this row's scales, one 32-bit word per 64-deep stage: INT4 two bf16 group scales
+            // ([rows][K/32]), NVFP4 four E4M3 block scales ([rows][K/16])
             const uint32_t* sc = static_cast<const uint32_t*>(g1 ? p.w1_scale : p.w2_scale);
             const int t0 = dt / 128;  // first tile of this thread (0 = A0, 1 = A1)
             const bool has0 = t0 == 0 || tl.dual;
@@ -699,11 +754,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const uint32_t at = tmem_base + lane_sel + C::A_TMEM + stage * C::A_TMEM_COLS;
                 uint32_t w[32];
                 if (has0) {  // warp-uniform: every lane of the warp works on the same tile
-                    dequant_int4_row(st + C::RAW_OFF + t0 * C::RAW_BYTES + r * 32, s0, w);
+                    if (p.fp4) dequant_fp4_row(st + C::RAW_OFF + t0 * C::RAW_BYTES + r * 32, s0, w);
+                    else dequant_int4_row(st + C::RAW_OFF + t0 * C::RAW_BYTES + r * 32, s0, w);
                     tmem_st32(at + t0 * 32, w);
                 }
                 if (has1) {
-                    dequant_int4_row(st + C::RAW_OFF + C::RAW_BYTES + r * 32, s1, w);
+                    if (p.fp4) dequant_fp4_row(st + C::RAW_OFF + C::RAW_BYTES + r * 32, s1, w);
+                    else dequant_int4_row(st + C::RAW_OFF + C::RAW_BYTES + r * 32, s1, w);
                     tmem_st32(at + 32, w);
                 }
                 tc_fence_before();  // the tensor-memory stores happen before the MMA that reads them
@@ -1335,6 +1392,7 @@ static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
     p.x_scale = a.x_scale;
     p.w1_scale = a.w1_scale;
     p.w2_scale = a.w2_scale;
+    p.fp4 = a.fp4 ? 1 : 0;
     p.gate_scale = a.gate_scale;
     p.up_scale = a.up_scale;
     p.alpha = a.alpha;
@@ -1348,7 +1406,9 @@ static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
     p.exit_ctr = a.exit_ctr;
     p.done1 = (p1 && p2) ? a.done1 : nullptr;
     p.s1 = p1 ? gemm_split_factor(a.A, a.G, a.H, a.I,
-                                  C::INT4 ? MOE_WDTYPE_INT4_G32 : (C::FP8 ? MOE_WDTYPE_FP8_E4M3_BLOCK128 : MOE_WDTYPE_BF16))
+                                  a.fp4 ? MOE_WDTYPE_NVFP4
+                                        : (C::INT4 ? MOE_WDTYPE_INT4_G32
+                                                   : (C::FP8 ? MOE_WDTYPE_FP8_E4M3_BLOCK128 : MOE_WDTYPE_BF16)))
               : 1;
     p.part = a.part;
     p.split_cnt = a.split_cnt;
@@ -1387,7 +1447,8 @@ int gemm_pick_bn(int64_t A, int G, int wdtype) {
     int bn = 16;
     while (bn < 256 && bn < avg) bn <<= 1;  // smallest tile holding an average group
     if (wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128 && bn > 128) bn = 128;  // fp32 promotion registers for gate and up
-    if (wdtype == MOE_WDTYPE_INT4_G32 && bn > 64) bn = 64;  // A tiles share TMEM with the accumulators
+    if ((wdtype == MOE_WDTYPE_INT4_G32 || wdtype == MOE_WDTYPE_NVFP4) && bn > 64)
+        bn = 64;  // 4-bit weights: A tiles share TMEM with the accumulators
     return bn;
 }
 
@@ -1428,7 +1489,8 @@ size_t gemm_split_counter_bytes(int64_t A, int G, int H, int I, int wdtype) {
 
 cudaError_t launch_moe_gemm(const MoeGemmArgs& a, cudaStream_t stream) {
     if (a.A == 0 || a.G == 0 || (!a.run_gemm1 && !a.run_gemm2)) return cudaSuccess;
-    const int wdtype = a.int4 ? MOE_WDTYPE_INT4_G32 : (a.fp8 ? MOE_WDTYPE_FP8_E4M3_BLOCK128 : MOE_WDTYPE_BF16);
+    const int wdtype = a.fp4 ? MOE_WDTYPE_NVFP4
+                             : (a.int4 ? MOE_WDTYPE_INT4_G32 : (a.fp8 ? MOE_WDTYPE_FP8_E4M3_BLOCK128 : MOE_WDTYPE_BF16));
     const int bn = gemm_pick_bn(a.A, a.G, wdtype);
     if (a.int4) {
         switch (bn) {

@@ -77,12 +77,13 @@ struct MoeGemmArgs {
     int64_t A;               // rows of x_perm / h / y
     int H, I;
     bool fp8;
-    bool int4;               // INT4 group-32 weights (bf16 activations)
+    bool int4;               // 4-bit weights, INT4 group-32 or NVFP4 (bf16 activations)
+    bool fp4;                // the 4-bit weights are NVFP4 (E2M1, E4M3 scale per 16 K)
     bool run_gemm1, run_gemm2;
     const void* x_perm;      // [A][H]
     const float* x_scale;    // FP8: [H/128][A]
     const void* w1;          // [G][2I][H]
-    const void* w1_scale;    // FP8: fp32 [G][2I/128][H/128]; INT4: bf16 [G][2I][H/32]
+    const void* w1_scale;    // FP8: fp32 [G][2I/128][H/128]; INT4: bf16 [G][2I][H/32]; NVFP4: E4M3 [G][2I][H/16]
     const float* gate_scale; // [G] or NULL
     const float* up_scale;   // [G] or NULL
     float alpha, beta, limit;
@@ -90,7 +91,7 @@ struct MoeGemmArgs {
     void* h;                 // [A][I]
     float* h_scale;          // FP8: [I/128][A]
     const void* w2;          // [G][H][I]
-    const void* w2_scale;    // FP8: fp32 [G][H/128][I/128]; INT4: bf16 [G][H][I/32]
+    const void* w2_scale;    // FP8: fp32 [G][H/128][I/128]; INT4: bf16 [G][H][I/32]; NVFP4: E4M3 [G][H][I/16]
     void* y;                 // [A][H] bf16
     unsigned int* tile_ctr;  // zero when idle; left at zero
     unsigned int* exit_ctr;  // zero when idle; left at zero

@@ -20,6 +20,9 @@ Workloads (synthetic stand-ins; no checkpoint or evaluation data is used):
   decode_t{1,64}_int4  the decode shapes with INT4 group-32 weights (batchgen PR #239 commit
                 notes: packed nibbles, one bf16 scale per 32 K); uniform nibbles and scales
                 drawn so that the weights' spread matches the bf16 workloads (std ~0.02).
+  decode_t{1,64}_nvfp4  the decode shapes with NVFP4 weights (E2M1, one E4M3 scale per 16 K)
+                and per-expert gate/up global scales U[0.52, 1.22] (xorl-wheels release
+                notes, "Changes": NVFP4 checkpoints with distinct gate and up scales).
 """
 from __future__ import annotations
 
@@ -31,6 +34,7 @@ import torch
 WDTYPE_BF16 = 0
 WDTYPE_FP8 = 1
 WDTYPE_INT4 = 2
+WDTYPE_NVFP4 = 3
 SCORE_SOFTMAX = 0
 SCORE_SIGMOID = 1
 
@@ -100,6 +104,12 @@ WORKLOADS = {
                                wdtype=WDTYPE_INT4, score=SCORE_SIGMOID, zipf_s=1.2, special_row=True),
     "decode_t64_int4": Workload("decode_t64_int4", T=64, H=4096, I=1024, E=256, k=8, n_sink=2, n_shared=2,
                                 wdtype=WDTYPE_INT4, score=SCORE_SIGMOID, zipf_s=1.2, special_row=True),
+    "decode_t1_nvfp4": Workload("decode_t1_nvfp4", T=1, H=4096, I=1024, E=256, k=8, n_sink=2, n_shared=2,
+                                wdtype=WDTYPE_NVFP4, score=SCORE_SIGMOID, zipf_s=1.2, special_row=True,
+                                expert_scales=(0.52, 1.22)),
+    "decode_t64_nvfp4": Workload("decode_t64_nvfp4", T=64, H=4096, I=1024, E=256, k=8, n_sink=2, n_shared=2,
+                                 wdtype=WDTYPE_NVFP4, score=SCORE_SIGMOID, zipf_s=1.2, special_row=True,
+                                 expert_scales=(0.52, 1.22)),
 }
 
 
@@ -130,6 +140,18 @@ def random_int4_weights(gen, shape, device, std: float):
     return packed.to(torch.uint8).contiguous(), scale.to(torch.bfloat16).contiguous()
 
 
+def random_nvfp4_weights(gen, shape, device, std: float):
+    """Offline NVFP4 weight format (an input format, not a step of the layer): uniform random
+    bytes [.., R, C/2] (two E2M1 codes each, low nibble = even column) and one E4M3 scale per
+    row and 16 columns [.., R, C/16] (uint8 codes), drawn around std / 2.93 (the root mean
+    square of the 16 E2M1 values) so the weights have std close to `std`."""
+    *lead, R, C = shape
+    packed = torch.randint(0, 256, (*lead, R, C // 2), generator=gen, device=device, dtype=torch.int32)
+    scale = (std / 2.926) * (0.75 + 0.5 * torch.rand((*lead, R, C // 16), generator=gen, device=device))
+    codes = scale.to(torch.float8_e4m3fn).view(torch.uint8)
+    return packed.to(torch.uint8).contiguous(), codes.contiguous()
+
+
 def _special_row(gen, n_cols: int, k: int, device) -> torch.Tensor:
     """Every logit below -104 (where fp32 sigmoid flushes to zero), drawn from
     {-105, -110, -150, -200}, with an exact tie straddling the top-k boundary:
@@ -150,7 +172,8 @@ def make_inputs(wl: Workload, device="cpu", seed: int | None = None) -> dict:
 
     Returns torch tensors: x bf16 [T,H]; logits fp32 [T,E+n_sink]; w1 [G,2I,H] and
     w2 [G,H,I] (bf16, or uint8 E4M3 codes with w1_scale/w2_scale fp32 block scales, or
-    INT4 packed bytes [G,2I,H/2] / [G,H,I/2] with bf16 group scales [G,2I,H/32] / [G,H,I/32]);
+    INT4 packed bytes [G,2I,H/2] / [G,H,I/2] with bf16 group scales [G,2I,H/32] / [G,H,I/32],
+    or NVFP4 packed bytes with E4M3 scale codes [G,2I,H/16] / [G,H,I/16]);
     gate_scale/up_scale fp32 [G] or None. Gate logits are x.W_r in fp64 rounded to fp32.
     """
     seed = wl.seed if seed is None else seed
@@ -188,6 +211,10 @@ def make_inputs(wl: Workload, device="cpu", seed: int | None = None) -> dict:
         elif wl.wdtype == WDTYPE_INT4:
             q1, s1 = random_int4_weights(gen, (n, 2 * I, H), dev, wl.w_std * wl.gate_up_mult)
             q2, s2 = random_int4_weights(gen, (n, H, I), dev, wl.w_std)
+            w1_parts.append(q1); w2_parts.append(q2); s1_parts.append(s1); s2_parts.append(s2)
+        elif wl.wdtype == WDTYPE_NVFP4:
+            q1, s1 = random_nvfp4_weights(gen, (n, 2 * I, H), dev, wl.w_std * wl.gate_up_mult)
+            q2, s2 = random_nvfp4_weights(gen, (n, H, I), dev, wl.w_std)
             w1_parts.append(q1); w2_parts.append(q2); s1_parts.append(s1); s2_parts.append(s2)
         else:
             w1_parts.append(w1.to(torch.bfloat16)); w2_parts.append(w2.to(torch.bfloat16))

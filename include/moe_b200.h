@@ -56,7 +56,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 3
+#define MOE_ABI_VERSION 4
 
 typedef enum moe_status {
     MOE_OK = 0,
@@ -80,9 +80,15 @@ typedef enum moe_wdtype {
     MOE_WDTYPE_BF16 = 0,             /* bf16 weights and activations                       */
     MOE_WDTYPE_FP8_E4M3_BLOCK128 = 1, /* E4M3 weights with one fp32 scale per 128x128 block;
                                         E4M3 activations with one fp32 scale per 1x128 block */
-    MOE_WDTYPE_INT4_G32 = 2          /* [P5] INT4 weights, two per byte (low nibble = even K),
+    MOE_WDTYPE_INT4_G32 = 2,         /* [P5] INT4 weights, two per byte (low nibble = even K),
                                         one bf16 scale per 32 K per row, value
                                         bf16((nibble - 8) * scale); bf16 activations       */
+    MOE_WDTYPE_NVFP4 = 3             /* [P1] NVFP4 weights: E2M1 values (1 sign, 2 exponent
+                                        bits with bias 1, 1 mantissa bit), two per byte (low
+                                        nibble = even K), one E4M3 scale per 16 K per row,
+                                        value E2M1 * E4M3 (exact in bf16); the checkpoint's
+                                        per-expert gate / up global scales are gate_scale /
+                                        up_scale; bf16 activations                          */
 } moe_wdtype;
 
 /* Problem statement. All fields are read on every call.
@@ -231,10 +237,10 @@ int moe_permute_noalloc(const int32_t* topk_ids, const void* x, const moe_dims* 
  *   h[r][i] = min(gate, L) * sigmoid(alpha * min(gate, L)) * (clamp(up, -L, L) + beta)
  * accumulated in fp32 (FP8: per 128-deep K block, times x_scale * w1_scale).
  *   x_perm, x_scale, offsets   as written by moe_permute (A = offsets[G]).
- *   w1        [G][2I][H]: rows [0, I) gate, [I, 2I) up; bf16 or E4M3, or for INT4 [G][2I][H/2]
- *             packed bytes (16-byte aligned).
- *   w1_scale  FP8: fp32 [G][2I/128][H/128]; INT4: bf16 [G][2I][H/32] (4-byte aligned);
- *             else NULL.
+ *   w1        [G][2I][H]: rows [0, I) gate, [I, 2I) up; bf16 or E4M3, or for INT4 and NVFP4
+ *             [G][2I][H/2] packed bytes (16-byte aligned).
+ *   w1_scale  FP8: fp32 [G][2I/128][H/128]; INT4: bf16 [G][2I][H/32]; NVFP4: E4M3 codes
+ *             [G][2I][H/16] (both 4-byte aligned); else NULL.
  *   gate_scale, up_scale  [G] fp32 per-group scales, or NULL for 1.0.
  *   limits    [G] fp32 clamp L per group ([P2'] one value per expert), or NULL for
  *             dims->limit. Each value > 0; +INFINITY disables that group's clamp.
@@ -255,8 +261,9 @@ int moe_gemm1_swiglu(const void* x_perm, const float* x_scale, const int32_t* of
  * summed in fp32 in that fixed order and rounded once to bf16.
  *   h, h_scale, offsets  as written by moe_gemm1_swiglu / moe_permute.
  *   inv_perm [T][k], topk_w [T][k], shared_w [T][n_sink] (NULL iff n_sink == 0).
- *   w2       [G][H][I] bf16 or E4M3, or INT4 [G][H][I/2] packed bytes; w2_scale FP8: fp32
- *            [G][H/128][I/128], INT4: bf16 [G][H][I/32]; else NULL.
+ *   w2       [G][H][I] bf16 or E4M3, or INT4 / NVFP4 [G][H][I/2] packed bytes; w2_scale FP8:
+ *            fp32 [G][H/128][I/128], INT4: bf16 [G][H][I/32], NVFP4: E4M3 codes [G][H][I/16];
+ *            else NULL.
  *   out      [T][H] bf16 out.
  * Errors: INVALID_ARG, WORKSPACE, ARCH, CUDA; TIMEOUT in the status word. */
 int moe_gemm2_combine(const void* h, const float* h_scale, const int32_t* offsets,

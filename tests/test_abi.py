@@ -26,7 +26,7 @@ def test_every_header_function_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert moe.moe_abi_version() == 3
+    assert moe.moe_abi_version() == 4
     for code in range(-7, 1):
         assert moe.status_string(code)
     assert "unknown" in moe.status_string(-99)
@@ -43,7 +43,8 @@ def _dims(**kw):
                                  dict(k=33, E=64), dict(n_sink=1, score=moe.MOE_SCORE_SOFTMAX),
                                  dict(n_sink=2, n_shared=1, score=moe.MOE_SCORE_SIGMOID), dict(T=-1),
                                  dict(limit=0.0), dict(limit=float("nan")), dict(alpha=float("inf")),
-                                 dict(wdtype=5), dict(score=3), dict(k=8, n_sink=25, score=moe.MOE_SCORE_SIGMOID)])
+                                 dict(wdtype=4), dict(wdtype=5), dict(score=3),
+                                 dict(k=8, n_sink=25, score=moe.MOE_SCORE_SIGMOID)])
 def test_invalid_dims_rejected(L, bad):
     d = _dims(**bad)
     with pytest.raises(moe.MoeError) as ei:
@@ -113,3 +114,18 @@ def test_gate_route_checks(L):
     d = _dims(T=4)
     assert L.moe_gate_route(fake, fake + 8, ctypes.byref(d), None, None, fake, fake, None, None, fake, n,
                             None) == -1  # w_gate not 16-byte aligned
+
+
+@pytest.mark.parametrize("wdtype", [moe.MOE_WDTYPE_INT4_G32, moe.MOE_WDTYPE_NVFP4])
+def test_4bit_weights_need_aligned_scales(L, wdtype):
+    """INT4 and NVFP4 layers size their workspaces like bf16 ones (bf16 activations) and
+    reject a missing or misaligned scale array before any CUDA call."""
+    d = _dims(wdtype=wdtype)
+    assert moe.moe_workspace_size(d, moe.MOE_WS_GEMM1) == moe.moe_workspace_size(_dims(), moe.MOE_WS_GEMM1)
+    fake = 1 << 20
+    n = moe.moe_workspace_size(d, moe.MOE_WS_GEMM1)
+    # x_perm, x_scale, offsets, w1, w1_scale, gate_scale, up_scale, limits, dims, h, h_scale, ws, ws_bytes, stream
+    assert L.moe_gemm1_swiglu(fake, None, fake, fake, None, None, None, None, ctypes.byref(d), fake, None, fake, n,
+                              None) == -1
+    assert L.moe_gemm1_swiglu(fake, None, fake, fake, fake + 2, None, None, None, ctypes.byref(d), fake, None, fake,
+                              n, None) == -1

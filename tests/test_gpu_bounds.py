@@ -29,6 +29,8 @@ SHAPES = [
                score=W.SCORE_SIGMOID, limit=10.0),
     W.Workload("t3_int4", T=3, H=512, I=256, E=8, k=2, n_sink=2, n_shared=2, wdtype=W.WDTYPE_INT4,
                score=W.SCORE_SIGMOID),
+    W.Workload("t37_nvfp4_scales", T=37, H=512, I=256, E=8, k=2, n_shared=1, wdtype=W.WDTYPE_NVFP4,
+               score=W.SCORE_SIGMOID, expert_scales=(0.52, 1.22)),
     # about 150 rows per group: the token-major 128-token FP8 tile, with ragged tails
     W.Workload("t300_fp8_wide", T=300, H=512, I=384, E=4, k=2, n_shared=1, wdtype=W.WDTYPE_FP8,
                score=W.SCORE_SIGMOID, limit=10.0),

@@ -12,7 +12,8 @@ from helpers import assert_bf16_close, assert_fp8_close, f32, oracle_layer, samp
 
 pytestmark = pytest.mark.gpu
 
-FULL = ["tiny", "oai_swiglu", "decode_t1", "decode_t8", "decode_t64", "decode_t1_int4", "decode_t64_int4"]
+FULL = ["tiny", "oai_swiglu", "decode_t1", "decode_t8", "decode_t64", "decode_t1_int4", "decode_t64_int4",
+        "decode_t1_nvfp4", "decode_t64_nvfp4"]
 SAMPLED = {"qwen3_30b_a3b": 48, "glm_fp8": 24}
 
 
@@ -81,7 +82,8 @@ def test_forward_skewed_routing_one_hot_expert():
     assert_bf16_close(out.float().cpu().numpy(), ref, "skewed")
 
 
-@pytest.mark.parametrize("name", ["oai_swiglu", "decode_t8", "glm_fp8", "decode_t1", "decode_t1_int4"])
+@pytest.mark.parametrize("name", ["oai_swiglu", "decode_t8", "glm_fp8", "decode_t1", "decode_t1_int4",
+                                  "decode_t1_nvfp4"])
 def test_public_stage_calls_reproduce_forward(name):
     """moe_route_topk -> moe_permute -> moe_experts -> moe_combine gives moe_forward's
     output bit for bit (same kernels, deterministic order), and matches the oracle."""

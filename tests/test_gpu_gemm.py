@@ -16,7 +16,7 @@ pytestmark = pytest.mark.gpu
 
 
 def make_case(T, E, k, S, H, I, fp8, seed, gate_up_mult=1.0, scales=False, sinks=False, skew=0.0, limits=False,
-              int4=False):
+              int4=False, fp4=False):
     ids = W.random_topk_ids(T, E, k, seed=seed, skew=skew)
     offsets, perm, inv = oracle.permute(ids.numpy(), E, S)
     A = T * (k + S)
@@ -26,11 +26,12 @@ def make_case(T, E, k, S, H, I, fp8, seed, gate_up_mult=1.0, scales=False, sinks
     w2f = torch.randn((G, H, I), generator=g, device="cuda") * 0.02
     xf = torch.randn((A, H), generator=g, device="cuda")
     hf = torch.randn((A, I), generator=g, device="cuda")
-    c = dict(T=T, E=E, k=k, S=S, H=H, I=I, A=A, G=G, fp8=fp8, int4=int4, ids=ids, offsets=offsets, perm=perm,
-             inv=inv)
-    if int4:  # INT4 group-32 weights, bf16 activations
-        c["w1"], c["w1_scale"] = W.random_int4_weights(g, (G, 2 * I, H), "cuda", 0.02 * gate_up_mult)
-        c["w2"], c["w2_scale"] = W.random_int4_weights(g, (G, H, I), "cuda", 0.02)
+    c = dict(T=T, E=E, k=k, S=S, H=H, I=I, A=A, G=G, fp8=fp8, int4=int4, fp4=fp4, ids=ids, offsets=offsets,
+             perm=perm, inv=inv)
+    if int4 or fp4:  # INT4 group-32 or NVFP4 weights, bf16 activations
+        make = W.random_nvfp4_weights if fp4 else W.random_int4_weights
+        c["w1"], c["w1_scale"] = make(g, (G, 2 * I, H), "cuda", 0.02 * gate_up_mult)
+        c["w2"], c["w2_scale"] = make(g, (G, H, I), "cuda", 0.02)
         c["xs"] = c["hs"] = None
         c["xp"], c["hp"] = xf.to(torch.bfloat16), hf.to(torch.bfloat16)
     elif fp8:
@@ -59,19 +60,22 @@ def make_case(T, E, k, S, H, I, fp8, seed, gate_up_mult=1.0, scales=False, sinks
 
 def dims_of(c, alpha=1.0, beta=0.0, limit=math.inf):
     return moe.MoeDims(T=c["T"], H=c["H"], I=c["I"], E=c["E"], k=c["k"], n_sink=c["S"] if c["shared_w"] is not None else 0,
-                       n_shared=c["S"], wdtype=2 if c.get("int4") else (1 if c["fp8"] else 0), score=1, alpha=alpha,
+                       n_shared=c["S"], wdtype=3 if c.get("fp4") else (2 if c.get("int4") else (1 if c["fp8"] else 0)),
+                       score=1, alpha=alpha,
                        beta=beta,
                        limit=limit, route_scale=1.0)
 
 
 def oracle_of(c, d):
     fp8 = c["fp8"]
-    if c.get("int4"):
+    if c.get("int4") or c.get("fp4"):
+        scl = u8 if c.get("fp4") else bits16  # NVFP4: E4M3 scale codes; INT4: bf16 scale bits
         return oracle.Layer(T=c["T"], H=c["H"], I=c["I"], E=c["E"], k=c["k"], n_sink=d.n_sink, n_shared=c["S"],
-                            wdtype=oracle.WDTYPE_INT4, score=1, alpha=d.alpha, beta=d.beta, limit=d.limit,
+                            wdtype=oracle.WDTYPE_NVFP4 if c.get("fp4") else oracle.WDTYPE_INT4, score=1,
+                            alpha=d.alpha, beta=d.beta, limit=d.limit,
                             route_scale=1.0, logits=np.zeros((c["T"], c["E"] + d.n_sink), np.float32),
                             x=np.zeros((c["T"], c["H"]), np.uint16), w1=u8(c["w1"]), w2=u8(c["w2"]),
-                            w1_scale=bits16(c["w1_scale"]), w2_scale=bits16(c["w2_scale"]),
+                            w1_scale=scl(c["w1_scale"]), w2_scale=scl(c["w2_scale"]),
                             gate_scale=f32(c["gate_scale"]), up_scale=f32(c["up_scale"]), limits=f32(c.get("limits")))
     return oracle.Layer(T=c["T"], H=c["H"], I=c["I"], E=c["E"], k=c["k"], n_sink=d.n_sink, n_shared=c["S"],
                         wdtype=1 if fp8 else 0, score=1, alpha=d.alpha, beta=d.beta, limit=d.limit,
@@ -103,6 +107,11 @@ GEMM1_CASES = [
     (64, 16, 4, 0, 512, 256, False, {"int4": True}),           # INT4, tile 32
     (300, 16, 4, 1, 512, 384, False, {"int4": True, "oai": True, "scales": True}),  # INT4, shared group
     (512, 8, 2, 0, 512, 256, False, {"int4": True, "skew": 3.0, "limits": True}),   # INT4, tile 128
+    # NVFP4 weights (E2M1, E4M3 scale per 16 K), per-group global scales on gate and up
+    (8, 64, 4, 0, 256, 256, False, {"fp4": True}),                           # tile 16, split-K
+    (64, 16, 4, 0, 512, 256, False, {"fp4": True, "scales": True}),          # tile 32, global scales
+    (300, 16, 4, 1, 512, 384, False, {"fp4": True, "oai": True, "scales": True}),  # shared group, OAI params
+    (512, 8, 2, 0, 512, 256, False, {"fp4": True, "skew": 3.0, "limits": True}),   # tile 64, ragged, clamps
     # decode-sized batches (at most 16 routed rows): one-row groups, split-K of GEMM1
     (2, 64, 4, 1, 512, 256, False, {}),                         # 10 rows, a shared group of 2
     (1, 32, 4, 0, 512, 384, False, {"scales": True, "limits": True}),  # one token, scales, clamp per expert
@@ -117,7 +126,7 @@ def test_gemm1_swiglu(T, E, k, S, H, I, fp8, extra):
     oai, glm = extra.get("oai", False), extra.get("glm", False)
     c = make_case(T, E, k, S, H, I, fp8, seed=T + E + H, gate_up_mult=4.0 if oai else 1.0,
                   scales=extra.get("scales", False), skew=extra.get("skew", 0.0), limits=extra.get("limits", False),
-                  int4=extra.get("int4", False))
+                  int4=extra.get("int4", False), fp4=extra.get("fp4", False))
     d = dims_of(c, alpha=1.702 if oai else 1.0, beta=1.0 if oai else 0.0,
                 limit=7.0 if oai else (10.0 if glm else math.inf))
     A = c["A"]
@@ -163,6 +172,9 @@ GEMM2_CASES = [
     (2, 64, 4, 1, 512, 256, False, False),      # decode-sized: 10 routed rows
     (2, 16, 4, 2, 512, 256, False, True),       # decode-sized, sink-gated shared groups
     (8, 2, 2, 0, 384, 256, "int4", False),      # INT4, 2 groups of 8 rows
+    (8, 64, 4, 0, 256, 256, "fp4", False),      # NVFP4, tile 16
+    (300, 16, 4, 2, 512, 256, "fp4", True),     # NVFP4, sink-gated shared groups
+    (512, 8, 2, 0, 384, 256, "fp4", False),     # NVFP4, tile 64, odd chunk count of H
     # many token blocks, an odd count of 128-row chunks of H (the last GEMM2 tile has one)
     (4096, 128, 2, 0, 384, 256, False, False),
     (4096, 128, 2, 0, 384, 256, True, False),   # FP8, tile 64
@@ -171,9 +183,9 @@ GEMM2_CASES = [
 
 @pytest.mark.parametrize("T,E,k,S,H,I,fp8,sinks", GEMM2_CASES)
 def test_gemm2_combine(T, E, k, S, H, I, fp8, sinks):
-    int4 = fp8 == "int4"
+    int4, fp4 = fp8 == "int4", fp8 == "fp4"
     fp8 = fp8 is True
-    c = make_case(T, E, k, S, H, I, fp8, seed=3 * T + E, sinks=sinks, int4=int4)
+    c = make_case(T, E, k, S, H, I, fp8, seed=3 * T + E, sinks=sinks, int4=int4, fp4=fp4)
     d = dims_of(c)
     out = torch.zeros((T, H), dtype=torch.bfloat16, device="cuda")
     ws = moe.alloc_workspace(d, moe.MOE_WS_GEMM2_COMBINE)
