@@ -74,12 +74,16 @@ struct Cfg {
     static constexpr int STAGE_BYTES = INT4 ? B_BYTES + 2 * RAW_BYTES : 2 * A_BYTES + B_BYTES;  // GEMM1-sized
     static constexpr int A_TMEM_COLS = 64;  // INT4: one stage's bf16 A0 | A1 (128 x 64 K, two K per column)
     // Dequantisation warps, in sets of four (a warp may only touch its TMEM lane quarter,
-    // warp % 4, so a set covers the 128 rows of a tile): the NS sets split each stage's
-    // 64 K of the one or two tiles evenly (single tile: a K range each; two tiles: one tile
-    // or a K range of one tile each). 8 warps for decode-sized tiles (the epilogue then has
-    // 4 warps), else 4. (16 warps at decode sizes measured no faster.)
+    // warp % 4, so a set covers the 128 rows of a tile). For decode-sized tiles (the
+    // epilogue then has 4 warps) 8 warps in two stage groups of one set each: a group
+    // converts every other stage, so one stage's fixed latency (barrier wait, shared-memory
+    // load, tensor-memory store and its wait, fence, arrive) overlaps the other's work.
+    // Otherwise one group of 4. A thread converts its row of both tiles of a stage.
+    // (Measured at decode sizes: one group of 8 and of 16 warps splitting each stage's
+    // tiles or K range, two groups of 8, four of 4 were all slower.)
     static constexpr int DQ = INT4 ? (BN <= 32 ? 8 : 4) : 0;
-    static constexpr int NS = DQ / 4;
+    static constexpr int NGRP = (INT4 && BN <= 32) ? 2 : 1;  // stage groups (alternate stages)
+    static constexpr int DQG = DQ / NGRP;                    // warps per stage: one set of 4
     // Token rows arrive in boxes of up to 64 rows, and only the boxes a tile's rows reach
     // are loaded, so a short token block does not pull a full BN-row tile through L2.
     static constexpr int BOX_ROWS = BN < 64 ? BN : 64;
@@ -137,7 +141,7 @@ struct Cfg {
     static_assert(STAGES >= 2, "at least two pipeline stages");
     static_assert(!(INT4 && FP8), "INT4 weights take bf16 activations");
     static_assert(!INT4 || BN <= 64, "INT4 keeps its A tiles next to the accumulators in TMEM");
-    static_assert(!INT4 || NS == 1 || NS == 2 || NS == 4, "4, 8 or 16 dequantisation warps");
+    static_assert(!INT4 || (DQG == 4 && DQG * NGRP == DQ), "dequantisation warps: stage groups of 4");
     static_assert(COLS % 8 == 0, "split-K merges columns in chunks of 8");
     // Split-K of GEMM1 is compiled in where it can be chosen (see gemm_split_factor):
     // every tile width except FP8 at 64 columns, whose promotion registers are full.
@@ -285,23 +289,15 @@ __device__ __forceinline__ void sum_split_partials(const float* part_tile, int s
     }
 }
 
-// Packed 4-bit weights: NW words (8 K each) of one row, 16-byte aligned for NW >= 4.
-template <int NW>
+// Packed 4-bit weights: the 8 words (8 K each) of a row's 64-deep stage segment (16-byte aligned).
 __device__ __forceinline__ void load_words(const uint8_t* raw, uint32_t* qw) {
-    static_assert(NW == 2 || NW == 4 || NW == 8, "16, 32 or 64 K");
-    if constexpr (NW == 2) {
-        const uint2 q = *reinterpret_cast<const uint2*>(raw);
-        qw[0] = q.x;
-        qw[1] = q.y;
-    } else {
 #pragma unroll
-        for (int i = 0; i < NW / 4; ++i) {
-            const uint4 q = *reinterpret_cast<const uint4*>(raw + 16 * i);
-            qw[4 * i] = q.x;
-            qw[4 * i + 1] = q.y;
-            qw[4 * i + 2] = q.z;
-            qw[4 * i + 3] = q.w;
-        }
+    for (int i = 0; i < 2; ++i) {
+        const uint4 q = *reinterpret_cast<const uint4*>(raw + 16 * i);
+        qw[4 * i] = q.x;
+        qw[4 * i + 1] = q.y;
+        qw[4 * i + 2] = q.z;
+        qw[4 * i + 3] = q.w;
     }
 }
 
@@ -326,15 +322,13 @@ __device__ __forceinline__ uint32_t int4_pair_bf16(uint32_t lo, uint32_t hi, int
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// out[j] = the bf16 pair (K 2j, 2j+1) of a segment of NW words (8 NW K) that starts on a
-// 32-K group boundary or inside the group of its first word; `sc` holds the scales from
-// that group on (bf16 bits, the first in the low half).
-template <int NW>
-__device__ __forceinline__ void dequant_int4_seg(const uint8_t* raw, uint32_t sc, uint32_t* out) {
-    uint32_t qw[NW];
-    load_words<NW>(raw, qw);
+// out[j] = the bf16 pair (K 2j, 2j+1) of a row's 64-deep segment, j < 32; `sc` holds its
+// two group scales (bf16 bits, K 0-31 in the low half).
+__device__ __forceinline__ void dequant_int4_row(const uint8_t* raw, uint32_t sc, uint32_t* out) {
+    uint32_t qw[8];
+    load_words(raw, qw);
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {
+    for (int w = 0; w < 8; ++w) {
         const unsigned short sb = (unsigned short)((sc >> (16 * (w >> 2))) & 0xFFFFu);  // 4 words per group
         const __nv_bfloat162 s = __halves2bfloat162(__ushort_as_bfloat16(sb), __ushort_as_bfloat16(sb));
         const uint32_t lo = qw[w] & 0x0F0F0F0Fu, hi = (qw[w] >> 4) & 0x0F0F0F0Fu;
@@ -411,38 +405,32 @@ __device__ __forceinline__ void fp4_word_bf16(uint32_t q, __nv_bfloat162 s, uint
     }
 }
 
-// out[j] = the bf16 pair (K 2j, 2j+1) of a segment of NW words (8 NW K) starting on a
-// 16-K block boundary; `sc` holds the E4M3 scale bytes from that block on (low byte first).
-template <int NW>
-__device__ __forceinline__ void dequant_fp4_seg(const uint8_t* raw, uint32_t sc, uint32_t* out) {
-    // the segment's NW / 2 scales to bf16, two per conversion (every E4M3 value is exact in
-    // f16 and in bf16)
-    constexpr int NS2 = NW >= 4 ? NW / 4 : 1;
-    __nv_bfloat162 sb[NS2];
+// out[j] = the bf16 pair (K 2j, 2j+1) of a row's 64-deep segment, j < 32; `sc` holds its
+// four E4M3 scale bytes (K 0-15 in the low byte).
+__device__ __forceinline__ void dequant_fp4_row(const uint8_t* raw, uint32_t sc, uint32_t* out) {
+    // the four scales to bf16, two per conversion (every E4M3 value is exact in f16 and in bf16)
+    __nv_bfloat162 sb[2];
 #pragma unroll
-    for (int i = 0; i < NS2; ++i) {
+    for (int i = 0; i < 2; ++i) {
         const __half2 h2 = __half2(__nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)((sc >> (16 * i)) & 0xFFFFu),
                                                               __NV_E4M3));
         sb[i] = __float22bfloat162_rn(__half22float2(h2));
     }
-    uint32_t qw[NW];
-    load_words<NW>(raw, qw);
+    uint32_t qw[8];
+    load_words(raw, qw);
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {  // two words per scale
+    for (int w = 0; w < 8; ++w) {  // two words per scale
         const __nv_bfloat16 s1 = (w & 2) ? sb[w >> 2].y : sb[w >> 2].x;
         fp4_word_bf16(qw[w], __halves2bfloat162(s1, s1), out + 4 * w);
     }
 }
 
-// One thread's share of a stage: NW words of one tile row into TMEM columns from `at`.
-template <int NW>
+// One tile row of a stage into the 32 TMEM columns from `at`.
 __device__ __forceinline__ void dequant_store(bool fp4, const uint8_t* raw, uint32_t sc, uint32_t at) {
-    uint32_t w[4 * NW];
-    if (fp4) dequant_fp4_seg<NW>(raw, sc, w);
-    else dequant_int4_seg<NW>(raw, sc, w);
-    if constexpr (NW == 8) tmem_st32(at, w);
-    else if constexpr (NW == 4) tmem_st16(at, w);
-    else tmem_st8(at, w);
+    uint32_t w[32];
+    if (fp4) dequant_fp4_row(raw, sc, w);
+    else dequant_int4_row(raw, sc, w);
+    tmem_st32(at, w);
 }
 
 // Warp-collective bounded wait: lane 0 waits, the verdict is broadcast.
@@ -485,7 +473,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&full[s], C::INT4 ? C::DQ : 1);  // INT4: the dequantisation warps complete it
+            mbar_init(&full[s], C::INT4 ? C::DQG : 1);  // INT4: the dequantisation warps complete it
             if (C::INT4) mbar_init(&raw_full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -744,14 +732,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
     } else if (C::INT4 && warp >= C::EPI0 + C::EPI) {
         // ------------------------------------------------------------ INT4 dequantisation
-        // Each warp converts the 32 weight rows of its TMEM lane quarter (warp % 4): its set
-        // (of NS) takes a fixed share of every stage's 64 K of the tile pair (or the single
-        // tile), in the same order as the MMA, stores it into the stage's TMEM A columns and
-        // completes `full`.
+        // Each warp converts the 32 weight rows of its TMEM lane quarter (warp % 4) of both
+        // tiles (A0, A1) of every stage of its stage group, in the same order as the MMA,
+        // stores them into the stage's TMEM A columns and completes `full`.
         const int r = (warp & 3) * 32 + lane;
-        const int set = (warp - C::EPI0 - C::EPI) / 4;
+        const int grp = (warp - C::EPI0 - C::EPI) / C::DQG;  // this warp's stage group
         const uint32_t lane_sel = (uint32_t)((warp & 3) * 32) << 16;
-        uint32_t stage = 0, phase = 0;
+        uint32_t stage = 0, phase = 0, n_run = 0;  // n_run: stages of earlier tiles
         bool ok = true;
         for (int i = 0; ok; ++i) {
             const int slot = i % kRing;
@@ -766,38 +753,37 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const int all_kb = K / C::BK;
             const int kbase = g1 ? tl.ks * all_kb / p.s1 : 0;
             const int num_kb = g1 ? (tl.ks + 1) * all_kb / p.s1 - kbase : all_kb;
-            // This thread's share: K values [k0, k0 + nk) of tile t0 (and, for one set over a
-            // tile pair, all of tile 1 too). nk is 64, 32 or 16.
-            const int per = (tl.dual ? 128 : 64) / C::NS;
-            const bool both = per == 128;
-            const int nk = both ? 64 : per;
-            const int t0 = both ? 0 : (set * per) / 64;
-            const int k0 = both ? 0 : (set * per) % 64;
-            // the row's scales, one 32-bit word per 64-deep stage: INT4 two bf16 group scales
-            // ([rows][K/32]), NVFP4 four E4M3 block scales ([rows][K/16]); shifted to k0
-            const int sshift = p.fp4 ? 8 * (k0 / 16) : 16 * (k0 / 32);
+            // this thread's row of tile A0 and, for a tile pair, of A1; the row's scales are
+            // one 32-bit word per 64-deep stage: INT4 two bf16 group scales ([rows][K/32]),
+            // NVFP4 four E4M3 block scales ([rows][K/16])
+            const bool both = tl.dual;
             const uint32_t* sc = static_cast<const uint32_t*>(g1 ? p.w1_scale : p.w2_scale);
-            const uint32_t* sc0 = sc + (size_t)((t0 == 0 ? tl.a0row : tl.a1row) + r) * (K / 64) + kbase;
+            const uint32_t* sc0 = sc + (size_t)(tl.a0row + r) * (K / 64) + kbase;
             const uint32_t* sc1 = sc + (size_t)(tl.a1row + r) * (K / 64) + kbase;
-            uint32_t s0 = __ldg(sc0), s1 = both ? __ldg(sc1) : 0u;
+            // this group's stages of the tile: kb = kb_first, kb_first + NGRP, ...
+            const int kb_first = (int)((uint32_t)(grp - (int)(n_run % C::NGRP) + C::NGRP) % C::NGRP);
+            const bool any = kb_first < num_kb;
+            uint32_t s0 = any ? __ldg(sc0 + kb_first) : 0u, s1 = (any && both) ? __ldg(sc1 + kb_first) : 0u;
             for (int kb = 0; kb < num_kb; ++kb) {
+                if ((int)((n_run + kb) % C::NGRP) != grp) {  // another group's stage
+                    if (++stage == (uint32_t)C::STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                    continue;
+                }
                 // the next stage's scales are loaded before this stage's bytes are awaited
-                const bool more = kb + 1 < num_kb;
-                const uint32_t n0 = more ? __ldg(sc0 + kb + 1) : 0u;
-                const uint32_t n1 = (more && both) ? __ldg(sc1 + kb + 1) : 0u;
+                const bool more = kb + C::NGRP < num_kb;
+                const uint32_t n0 = more ? __ldg(sc0 + kb + C::NGRP) : 0u;
+                const uint32_t n1 = (more && both) ? __ldg(sc1 + kb + C::NGRP) : 0u;
                 if (!warp_wait(&raw_full[stage], phase, ab, p.status)) {
                     ok = false;
                     break;
                 }
                 const uint8_t* raw = smem + (size_t)stage * C::STAGE_BYTES + C::RAW_OFF + r * 32;
                 const uint32_t at = tmem_base + lane_sel + C::A_TMEM + stage * C::A_TMEM_COLS;
-                // warp-uniform branches: every lane of the warp takes the same share
-                const uint8_t* raw0 = raw + t0 * C::RAW_BYTES + k0 / 2;
-                const uint32_t at0 = at + t0 * 32 + k0 / 2;
-                if (nk == 64) dequant_store<8>(p.fp4, raw0, s0 >> sshift, at0);
-                else if (nk == 32) dequant_store<4>(p.fp4, raw0, s0 >> sshift, at0);
-                else dequant_store<2>(p.fp4, raw0, s0 >> sshift, at0);
-                if (both) dequant_store<8>(p.fp4, raw + C::RAW_BYTES, s1, at + 32);
+                dequant_store(p.fp4, raw, s0, at);
+                if (both) dequant_store(p.fp4, raw + C::RAW_BYTES, s1, at + 32);  // warp-uniform
                 tc_fence_before();  // the tensor-memory stores happen before the MMA that reads them
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[stage]);
@@ -808,6 +794,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 s0 = n0;
                 s1 = n1;
             }
+            n_run += (uint32_t)num_kb;
         }
     } else {
         // ------------------------------------------------------------ epilogue
