@@ -85,6 +85,9 @@ def lib() -> ctypes.CDLL:
                              ctypes.c_size_t, _VP], ctypes.c_int),
             "moe_combine": ([_VP, _VP, _VP, _VP, _VP, P, _VP, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
             "moe_gate_route": ([_VP, _VP, P, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP], ctypes.c_int),
+            "moe_ep_row_ids": ([_VP, P, _VP, _VP], ctypes.c_int),
+            "moe_ep_rebase": ([_VP, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                               _VP, _VP], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -200,6 +203,15 @@ def moe_experts(x_perm, x_scale, offsets, w1, w1_scale, gate_scale, up_scale, li
 def moe_combine(y, offsets, inv_perm, topk_w, shared_w, dims: MoeDims, out, ws, stream=None) -> None:
     _check("moe_combine", lib().moe_combine(_p(y), _p(offsets), _p(inv_perm), _p(topk_w), _p(shared_w),
                                             ctypes.byref(dims), _p(out), _p(ws), _nbytes(ws), _s(stream)))
+
+
+def moe_ep_row_ids(offsets, dims: MoeDims, row_ids, stream=None) -> None:
+    _check("moe_ep_row_ids", lib().moe_ep_row_ids(_p(offsets), ctypes.byref(dims), _p(row_ids), _s(stream)))
+
+
+def moe_ep_rebase(ids, n: int, E: int, n_shared: int, local_offset: int, n_local: int, out, stream=None) -> None:
+    _check("moe_ep_rebase", lib().moe_ep_rebase(_p(ids), int(n), int(E), int(n_shared), int(local_offset),
+                                                int(n_local), _p(out), _s(stream)))
 
 
 def _nbytes(t) -> int:

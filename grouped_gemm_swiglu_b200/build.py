@@ -22,7 +22,7 @@ BUILD = os.path.join(PKG, "_build")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libmoe_b200.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc" if os.path.exists("/usr/local/cuda/bin/nvcc") else "nvcc")
-SOURCES = ["api.cu", "router.cu", "permute.cu", "combine.cu", "gemm.cu", "permute_noalloc.cu"]
+SOURCES = ["api.cu", "router.cu", "permute.cu", "combine.cu", "gemm.cu", "permute_noalloc.cu", "ep.cu"]
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include"), "-I", CSRC]

@@ -436,4 +436,25 @@ int moe_forward(const float* logits, const float* bias, const void* x, const voi
     return do_combine(at<void>(ws, L.y), offsets, at<int32_t>(ws, L.inv), w, sw, d, out, status, s);
 }
 
+int moe_ep_row_ids(const int32_t* offsets, const moe_dims* d, int32_t* row_ids, void* stream) {
+    int rc = check_dims(d);
+    if (rc != MOE_OK) return rc;
+    if (d->T > 0 && (!offsets || !row_ids)) return MOE_ERR_INVALID_ARG;
+    if ((rc = check_arch()) != MOE_OK) return rc;
+    if (d->T == 0) return MOE_OK;
+    return cuda_status(launch_ep_row_ids(offsets, groups(d), (int)rows_A(d), row_ids, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_ep_rebase(const int32_t* ids, int64_t n, int32_t E, int32_t n_shared, int32_t local_offset, int32_t n_local,
+                  int32_t* out, void* stream) {
+    if (n < 0 || n > INT32_MAX || E < 1 || E > kMaxE || n_shared < 0 || n_shared > kMaxSlots || n_local < 1 ||
+        local_offset < 0 || (int64_t)local_offset + n_local > E)
+        return MOE_ERR_INVALID_ARG;
+    if (n > 0 && (!ids || !out)) return MOE_ERR_INVALID_ARG;
+    int rc = check_arch();
+    if (rc != MOE_OK) return rc;
+    return cuda_status(
+        launch_ep_rebase(ids, n, E, n_shared, local_offset, n_local, out, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

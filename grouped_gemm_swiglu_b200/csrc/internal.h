@@ -111,6 +111,9 @@ int gemm_split_factor(int64_t A, int G, int H, int I, int wdtype);
 size_t gemm_split_scratch_bytes(int64_t A, int G, int H, int I, int wdtype);
 size_t gemm_split_counter_bytes(int64_t A, int G, int H, int I, int wdtype);
 cudaError_t launch_moe_gemm(const MoeGemmArgs& a, cudaStream_t stream);
+cudaError_t launch_ep_row_ids(const int32_t* offsets, int G, int A, int32_t* row_ids, cudaStream_t stream);
+cudaError_t launch_ep_rebase(const int32_t* ids, int64_t n, int E, int n_shared, int local_offset, int n_local,
+                             int32_t* out, cudaStream_t stream);
 
 int num_sms();
 

@@ -28,6 +28,10 @@
  *        the expert range are an error.
  *   [P5] batchgen PR #239 "sm100: Fused INT4 grouped + SiLU Triton kernel": per-expert
  *        sorted-token dispatch, fp32 accumulation, slot-specific weighted reduction.
+ *   [P1'] the same xorl-wheels release, "Changes": expert-parallel lookups are rank-local;
+ *        routing ids stay global, each rank rebases them by its local expert offset and
+ *        bounds-checks them against its local expert count, and ids outside that range
+ *        are an error.
  *
  * Conventions shared by every entry point
  *   - Every pointer argument is a DEVICE pointer on the current CUDA device unless
@@ -56,7 +60,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 4
+#define MOE_ABI_VERSION 5
 
 typedef enum moe_status {
     MOE_OK = 0,
@@ -313,6 +317,35 @@ int moe_forward(const float* logits, const float* bias, const void* x, const voi
                 const float* limits, const void* w2, const void* w2_scale, const moe_dims* dims,
                 void* out, int32_t* topk_ids, float* topk_w, float* shared_w, uint32_t* packed,
                 void* ws, size_t ws_bytes, void* stream);
+
+/* ---- Expert parallelism [P1']: experts partitioned over ranks ----------------------
+ * Rank r of R holds routed experts [r*E/R, (r+1)*E/R) and every shared expert. A rank
+ * permutes its own tokens as usual (the routed rows are then already in order of the
+ * rank that owns their expert), sends each routed row with its global group id to that
+ * rank, rebases the ids it receives (moe_ep_rebase), runs moe_permute / moe_experts /
+ * moe_combine (k = 1, unit weights) over its local groups, sends the rows back and
+ * combines them as in the one-rank layer. The exchange itself is the caller's (NCCL). */
+
+/* moe_ep_row_ids -- the weight group of every permuted row.
+ *   offsets [G+1] as written by moe_permute (G = E + n_shared; entries are clamped into
+ *   [0, A] before use), A = T*(k + n_shared) from dims.
+ *   row_ids [A] int32 out: row_ids[r] = g with offsets[g] <= r < offsets[g+1], i.e. the
+ *   global routed expert id (< E) or E + s for shared expert s.
+ * Errors: INVALID_ARG (dims, NULL pointers), ARCH, CUDA. */
+int moe_ep_row_ids(const int32_t* offsets, const moe_dims* dims, int32_t* row_ids, void* stream);
+
+/* moe_ep_rebase -- global group ids to this rank's local group ids.
+ *   ids [n] int32: global ids as written by moe_ep_row_ids on any rank.
+ *   E, n_shared: the global routed expert count and shared expert count;
+ *   local_offset, n_local: this rank's routed experts are [local_offset,
+ *   local_offset + n_local) (0 <= local_offset, local_offset + n_local <= E).
+ *   out [n] int32: id - local_offset for a local routed expert, n_local + s for shared
+ *   expert s (replicated on every rank), -1 for anything else: an id of another rank or
+ *   out of range. moe_permute over these local ids (E = n_local + n_shared, k = 1)
+ *   records MOE_ERR_EXPERT_ID for a -1 and drops that row. out may alias ids.
+ * Errors: INVALID_ARG (sizes, NULL pointers), ARCH, CUDA. */
+int moe_ep_rebase(const int32_t* ids, int64_t n, int32_t E, int32_t n_shared, int32_t local_offset,
+                  int32_t n_local, int32_t* out, void* stream);
 
 #ifdef __cplusplus
 }

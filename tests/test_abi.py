@@ -26,7 +26,7 @@ def test_every_header_function_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert moe.moe_abi_version() == 4
+    assert moe.moe_abi_version() == 5
     for code in range(-7, 1):
         assert moe.status_string(code)
     assert "unknown" in moe.status_string(-99)
@@ -69,6 +69,29 @@ def test_null_pointers_and_small_workspace_rejected(L):
     # sink weights pointer must match n_sink
     rc = L.moe_route_topk(fake, ctypes.byref(d), None, fake, fake, fake, None, None)
     assert rc == -1
+
+
+@pytest.mark.parametrize("args", [
+    (-1, 8, 0, 0, 4),     # negative row count
+    (16, 0, 0, 0, 1),     # no routed experts
+    (16, 8, -1, 0, 4),    # negative shared count
+    (16, 8, 0, -1, 4),    # negative local offset
+    (16, 8, 0, 4, 5),     # local range past E
+    (16, 8, 0, 0, 0),     # no local experts
+    (16, 2000, 0, 0, 4),  # E beyond the library's limit
+])
+def test_ep_rebase_rejects_bad_ranges(L, args):
+    n, E, n_shared, off, n_local = args
+    fake = 1 << 20  # never dereferenced: the checks fail first
+    assert L.moe_ep_rebase(fake, n, E, n_shared, off, n_local, fake, None) == -1
+
+
+def test_ep_calls_reject_null_pointers(L):
+    d = _dims()
+    assert L.moe_ep_rebase(None, 16, 8, 0, 0, 4, None, None) == -1
+    assert L.moe_ep_row_ids(None, ctypes.byref(d), None, None) == -1
+    bad = _dims(k=0)
+    assert L.moe_ep_row_ids(1 << 20, ctypes.byref(bad), 1 << 20, None) == -1
 
 
 @pytest.mark.parametrize("name", list(W.WORKLOADS))
