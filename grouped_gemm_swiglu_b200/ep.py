@@ -49,11 +49,15 @@ class TorchExchange:
     def all_to_all(self, out: torch.Tensor, inp: torch.Tensor, out_splits: list[int], in_splits: list[int]) -> None:
         self.dist.all_to_all_single(out, inp, out_splits, in_splits, group=self.group)
 
+    def all_reduce(self, t: torch.Tensor) -> None:
+        """In-place sum over the ranks."""
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.SUM, group=self.group)
+
 
 class LocalExchange:
-    """R ranks as threads of one process on one device: all_to_all by device copies
-    between the ranks' buffers, after every rank's work so far has finished (the ranks'
-    kernels never wait on one another; the threads meet on the host)."""
+    """R ranks as threads of one process on one device: all_to_all (and all_reduce) by
+    device copies between the ranks' buffers, after every rank's work so far has finished
+    (the ranks' kernels never wait on one another; the threads meet on the host)."""
 
     def __init__(self, world: int):
         self.world = world
@@ -86,6 +90,21 @@ class _LocalRankExchange:
         if out.is_cuda:
             torch.cuda.synchronize(out.device)
         hub._barrier.wait()  # every rank has read the posted buffers
+
+    def all_reduce(self, t: torch.Tensor) -> None:
+        """In-place sum over the ranks, in fp32 and rank order (the same bits on every rank)."""
+        hub = self.hub
+        if t.is_cuda:
+            torch.cuda.synchronize(t.device)
+        hub._posted[self.rank] = (t, [])
+        hub._barrier.wait()
+        acc = torch.zeros(t.shape, dtype=torch.float32, device=t.device)
+        for src in range(self.world):
+            acc += hub._posted[src][0].float()
+        hub._barrier.wait()  # every rank has read every tensor before any is overwritten
+        t.copy_(acc.to(t.dtype))
+        if t.is_cuda:
+            torch.cuda.synchronize(t.device)
 
 
 def shard(t: torch.Tensor | None, rank: int, world: int, E: int, n_shared: int):
