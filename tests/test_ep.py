@@ -250,3 +250,49 @@ def test_an_id_outside_the_local_range_is_reported():
     # rows meant for rank 1 arrive with id 0 (rank 0's expert): rank 1's rebase turns them
     # into -1 and its local permutation records the error
     assert layers[1].status() == MOE_ERR_EXPERT_ID
+
+
+def _dying_rank(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:  # leaves between steps, before its first exchange
+        _put_and_exit(q, (rank, "left"))
+    d = _dims(0, 8, 2, 0, 0)
+    w1, w2 = _weights(8, 0)
+    logits, x = _inputs(rank, 6, 8, 0, d.H)
+    layer = ep.ExpertParallelMoE(d, rank, world, ep.shard(w1, rank, world, 8, 0), ep.shard(w2, rank, world, 8, 0),
+                                 exchange=ep.TorchExchange(), ops=CpuOps)
+    try:
+        layer.forward(logits, x)
+        msg = "finished"
+    except Exception as e:  # noqa: BLE001 (the expected outcome)
+        msg = "error: " + type(e).__name__
+    _put_and_exit(q, (rank, msg))
+
+
+def _put_and_exit(q, item):
+    """Report, then leave without the process group's orderly shutdown (which would wait
+    for the other rank)."""
+    q.put(item)
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
+def test_a_rank_that_leaves_ends_the_others_exchange_with_an_error():
+    """Failure detection on the host: one rank exits before the exchange; the other's
+    all_to_all ends with an error within the process group's short timeout, not a hang."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dying_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = dict(q.get(timeout=10) for _ in range(2))
+    assert res[1] == "left"
+    assert res[0].startswith("error"), res[0]
