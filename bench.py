@@ -44,17 +44,52 @@ def parse():
     return ap.parse_args()
 
 
+KERNEL_SOURCES = ("gemm.cu", "ptx.cuh", "internal.h")  # the grouped-GEMM kernel and what it includes
+
+
+def strip_comments(text: str) -> str:
+    """C/C++ source without comments and with whitespace runs collapsed (string and
+    character literals kept as they are)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
+def kernel_code_digest() -> str:
+    """sha1 of the grouped-GEMM kernel's sources without their comments: a comment edit
+    keeps a capture's counters, any code edit retires them."""
+    import hashlib
+    h = hashlib.sha1()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "grouped_gemm_swiglu_b200", "csrc", name)) as f:
+            h.update(strip_comments(f.read()).encode())
+    return h.hexdigest()
+
+
 def profiled_traffic(workload: str):
     """DRAM bytes per launch of the grouped-GEMM kernel from the committed ncu capture,
-    or None when the kernel source changed since that capture."""
-    import hashlib
+    or None when the kernel's code changed since that capture."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)
-        src = os.path.join(ROOT, "grouped_gemm_swiglu_b200", "csrc", "gemm.cu")
-        with open(src, "rb") as f:
-            digest = hashlib.sha1(f.read()).hexdigest()
-        if rec.get("gemm_cu_sha1") != digest:
+        if rec.get("kernel_code_sha1") != kernel_code_digest():
             return None
         return rec.get("workloads", {}).get(workload)
     except Exception:

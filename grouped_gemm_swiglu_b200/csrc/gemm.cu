@@ -12,7 +12,8 @@
 // #39920 "Modifications"; DeepGEMM PR #445 "Summary") runs in the epilogue, with the
 // per-group gate/up scales applied to the accumulators first (xorl-wheels FlashInfer
 // 0.6.18 release notes, "Changes"). The intermediate never leaves the SM unactivated.
-// Phase 2, GEMM2: one MMA per K step; the epilogue stores y in bf16.
+// Phase 2, GEMM2: a tile covers two 128-row chunks of H (the last one alone when H/128
+// is odd), two MMAs per K step; the epilogue stores y in bf16.
 //
 // FP8 (E4M3, 128x128 weight blocks, 1x128 activation blocks; GLM FP8 blockwise, sglang
 // PR #39920 "Motivation"): every 128-deep K block is one pipeline stage; its product
@@ -20,20 +21,25 @@
 // registers with the product of the two block scales, while the tensor core fills the
 // other buffer. GEMM1's epilogue then quantises h per 1x128 block (fused act-quant).
 //
-// Scheduling: tiles are numbered GEMM1 first -- (token block, 128-row chunk of I) --
-// then GEMM2 -- (token block, 128-row chunk of H). The producer warp claims the next
+// 4-bit weights (INT4 group-32, NVFP4): TMA brings the packed bytes and the token rows;
+// dequantisation warps convert each 64-deep stage of the weight rows to bf16 and store
+// it into tensor memory, which the MMA reads as its A operand.
+//
+// Scheduling: tiles are numbered GEMM1 first -- (token block, 128-row chunk of I, K
+// split) -- then GEMM2 -- (token block, pair of 128-row chunks of H). The producer warp claims the next
 // tile from a global counter and hands its number to the MMA and epilogue warps through
 // a two-slot ring in shared memory. When both phases run, a GEMM2 tile of token block b
 // first loads its weights, then waits until all GEMM1 tiles of b have published their h
 // rows (a per-block release counter); a tile only ever waits for tiles claimed before
 // it, which never wait themselves, so the schedule cannot deadlock.
 //
-// Roles (320 threads): warp 0 lane 0 issues TMA loads into a STAGES-deep ring; warp 1
-// owns TMEM and lane 0 issues tcgen05.mma; warps 2..9 are the epilogue (warp w reads
-// TMEM lanes 32*(w%4).., and columns of half (w-2)/4 of the tile). FP8 tiles of 128
-// tokens are token-major (tokens = M = TMEM lanes) and launch 384 threads: warp 2
-// releases GEMM1 tiles' h to GEMM2, warp 3 only lends its registers, and warps 4..11 are
-// the epilogue. Every wait is bounded
+// Roles: warp 0 lane 0 issues TMA loads into a STAGES-deep ring; warp 1 owns TMEM and
+// lane 0 issues tcgen05.mma; the next EPI warps are the epilogue (warp w reads TMEM lanes
+// 32*(w%4).., and its group's share of the tile's columns): 8 warps (320 threads), 16 at
+// 256 token columns, 4 for 4-bit decode tiles, which add their DQ dequantisation warps
+// after the epilogue. FP8 tiles of 128 tokens are token-major (tokens = M = TMEM lanes)
+// and launch 384 threads: warp 2 releases GEMM1 tiles' h to GEMM2, warp 3 only lends its
+// registers, and warps 4..11 are the epilogue. Every wait is bounded
 // (ptx.cuh): on timeout the CTA sets MOE_ERR_TIMEOUT, drains its outstanding copies and
 // MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
