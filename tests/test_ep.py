@@ -296,3 +296,30 @@ def test_a_rank_that_leaves_ends_the_others_exchange_with_an_error():
     res = dict(q.get(timeout=10) for _ in range(2))
     assert res[1] == "left"
     assert res[0].startswith("error"), res[0]
+
+
+def _random_configs(n, seed=5):
+    import random
+    rnd = random.Random(seed)
+    out = []
+    while len(out) < n:
+        world = rnd.choice([1, 2, 3, 4])
+        E = world * rnd.randint(1, 4)
+        k = rnd.randint(1, min(E, 4))
+        n_sink = rnd.choice([0, 0, 2])
+        n_shared = n_sink if n_sink and rnd.random() < 0.5 else (0 if n_sink else rnd.choice([0, 1, 2]))
+        Ts = [rnd.choice([0, 1, 3, 8]) for _ in range(world)]
+        out.append((world, tuple(Ts), E, k, n_sink, n_shared))
+    return out
+
+
+@pytest.mark.parametrize("cfg", _random_configs(16), ids=lambda c: "w{}-T{}-E{}-k{}-s{}-sh{}".format(
+    c[0], "_".join(map(str, c[1])), *c[2:]))
+def test_random_layouts_match_the_one_rank_pipeline(cfg):
+    world, Ts, E, k, n_sink, n_shared = cfg
+    outs, errs, layers = _run_threads(world, list(Ts), E, k, n_sink, n_shared)
+    assert not errs, errs
+    for r in range(world):
+        got, ref = outs[r]
+        assert torch.equal(got, ref), f"rank {r}"
+        assert layers[r].status() == 0
