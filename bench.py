@@ -21,6 +21,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -114,7 +115,7 @@ class ClockSampler:
     def __init__(self, uuid: str):
         self.uuid = uuid.lower().replace("gpu-", "")
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"moe_b200_clocks_{os.getpid()}.csv")
 
     def start(self):
         try:

@@ -65,7 +65,7 @@ extern "C" {
 typedef enum moe_status {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = -1,  /* a size, pointer or parameter outside the documented range */
-    MOE_ERR_UNSUPPORTED = -2,  /* a valid combination this build does not implement */
+    MOE_ERR_UNSUPPORTED = -2,  /* a valid combination this library does not implement */
     MOE_ERR_ARCH = -3,         /* the current device is not compute capability 10.x */
     MOE_ERR_WORKSPACE = -4,    /* ws is NULL, misaligned (256 B) or smaller than required */
     MOE_ERR_EXPERT_ID = -5,    /* (device) routing data out of range: an id outside [0, E) or
