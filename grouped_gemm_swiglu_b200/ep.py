@@ -118,10 +118,9 @@ def shard(t: torch.Tensor | None, rank: int, world: int, E: int, n_shared: int):
 
 @dataclass
 class _Sent:
+    """What a rank keeps from its dispatch to finish the layer for its own tokens."""
     T: int
     dims: MoeDims
-    send_dims: MoeDims
-    ids: torch.Tensor
     tw: torch.Tensor
     sw: torch.Tensor | None
     offsets: torch.Tensor
@@ -178,7 +177,7 @@ class ExpertParallelMoE:
         offs = offsets.cpu().tolist()  # host copy of the group bounds sizes the exchange
         nl = self.n_local
         send = [offs[(r + 1) * nl] - offs[r * nl] for r in range(self.world)]
-        return _Sent(T, d, sd, ids, tw, sw, offsets, inv, x_perm, row_ids, offs[d.E], send)
+        return _Sent(T, d, tw, sw, offsets, inv, x_perm, row_ids, offs[d.E], send)
 
     # ---------------------------------------------------------------- phase 3 (local)
     def _local_experts(self, rows: torch.Tensor, row_ids: torch.Tensor) -> torch.Tensor:
