@@ -150,8 +150,10 @@ struct Cfg {
     static_assert(!INT4 || (DQG == 4 && DQG * NGRP == DQ), "dequantisation warps: stage groups of 4");
     static_assert(COLS % 8 == 0, "split-K merges columns in chunks of 8");
     // Split-K of GEMM1 is compiled in where it can be chosen (see gemm_split_factor):
-    // every tile width except FP8 at 64 columns, whose promotion registers are full.
-    static constexpr bool SPLIT_OK = !(FP8 && BN >= 64);
+    // every tile width except FP8 from 64 columns, whose promotion registers are full,
+    // and 256 columns, whose merge path alone would push the kernel past its register
+    // cap (a 256-column tile means large groups, which never need a split).
+    static constexpr bool SPLIT_OK = !(FP8 && BN >= 64) && BN < 256;
 
     // full/empty per stage, tfull/tempty per TMEM buffer, ring_full/ring_empty x kRing, drain,
     // epibar, and for INT4 raw_full per stage (packed bytes and token rows landed)
@@ -873,7 +875,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const uint32_t tb = tmem_base + lane_off + buf * C::ACC_COLS;
                 __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g1 ? p.h : p.y);
                 const int tile1 = tl.blk * p.c1 + tl.c;
-                if (g1 && p.s1 > 1) {
+                if (C::SPLIT_OK && g1 && p.s1 > 1) {
                     // split-K: store this split's fp32 gate/up sums; the last split merges
 #pragma unroll 1
                     for (int cc = c0; cc < c0 + C::COLS && cc < n_mma; cc += C::CW) {
@@ -930,7 +932,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[buf]);
                 ++it;
-                if (g1 && p.s1 > 1) {
+                if (C::SPLIT_OK && g1 && p.s1 > 1) {
                     const int r = split_arrive(tile1);
                     if (r < 0) {
                         ok = false;
@@ -1496,7 +1498,7 @@ int gemm_split_factor(int64_t A, int G, int H, int I, int wdtype) {
     const int bn = gemm_pick_bn(A, G, wdtype);
     const int64_t tiles = gemm_max_blocks(A, G, bn) * (I / 128);
     const int kb = H / (fp8 ? 128 : 64);
-    if (fp8 && bn >= 64) return 1;  // the kernel variant has no split-K path
+    if ((fp8 && bn >= 64) || bn >= 256) return 1;  // the kernel variant has no split-K path
     int s = 1;
     while (s < 4 && tiles * s < kTarget && kb >= 4 * s) s *= 2;
     return s;

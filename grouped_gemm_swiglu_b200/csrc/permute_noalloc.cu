@@ -12,8 +12,11 @@
 // The array is a file-scope __device__ variable: every GPU that loads the library holds
 // kNoAllocScratchBytes of it until the process exits, and every call on that GPU shares
 // it. Host code must not pass the array's name to a kernel (on the host it is only a
-// stand-in symbol); the device address is fetched once per device with
-// cudaGetSymbolAddress, with that device current, on the first call.
+// stand-in symbol); the device address is fetched with cudaGetSymbolAddress, with the
+// device current: on every call that is not being captured into a CUDA graph (so a
+// context created after cudaDeviceReset, or another context current on the device, gets
+// its own address), and from the last such lookup on that device while the stream is
+// capturing.
 #include <mutex>
 
 #include "internal.h"
@@ -29,16 +32,22 @@ constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void* g_scratch_addr[kMaxDevices] = {nullptr};
 
-// Device address of the static scratch on the current device (set-up on first use).
-int scratch_address(void** out) {
+// Device address of the static scratch in the current context. Looked up on each call
+// (a cheap host call once the module is loaded), except while `stream` is capturing,
+// where the address of the last uncaptured call on this device is reused.
+int scratch_address(cudaStream_t stream, void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return MOE_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_addr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
         g_scratch_addr[dev] = p;
+    } else if (!g_scratch_addr[dev]) {
+        return MOE_ERR_UNSUPPORTED;  // the look-up itself may not run under capture
     }
     *out = g_scratch_addr[dev];
     return MOE_OK;
@@ -49,7 +58,9 @@ bool valid_dims(const moe_dims* d) {
     if (d->T < 0 || d->H <= 0 || d->I <= 0 || d->H % 128 || d->I % 128) return false;
     if (d->E < 1 || d->E > 1024 || d->k < 1 || d->k > d->E || d->k > 32) return false;
     if (d->n_shared < 0 || d->k + d->n_shared > 32) return false;
-    if (d->wdtype != MOE_WDTYPE_BF16 && d->wdtype != MOE_WDTYPE_FP8_E4M3_BLOCK128) return false;
+    if (d->wdtype != MOE_WDTYPE_BF16 && d->wdtype != MOE_WDTYPE_FP8_E4M3_BLOCK128 && d->wdtype != MOE_WDTYPE_INT4_G32 &&
+        d->wdtype != MOE_WDTYPE_NVFP4)
+        return false;  // 4-bit weights take bf16 activations: a bf16 permutation
     return (int64_t)d->T * (d->k + d->n_shared) <= INT32_MAX / 2;
 }
 
@@ -73,12 +84,16 @@ extern "C" int moe_permute_noalloc(const int32_t* topk_ids, const void* x, const
         return MOE_ERR_CUDA;
     if (major != 10) return MOE_ERR_ARCH;
     void* scratch = nullptr;
-    int rc = scratch_address(&scratch);
+    int rc = scratch_address(static_cast<cudaStream_t>(stream), &scratch);
     if (rc != MOE_OK) return rc;
-    // The first word of the array counts finished CTAs of the counting kernel; it must be
-    // zero when a call starts. It is zero at module load and every call leaves it at zero;
-    // the rest of the array is written before it is read. The status word is the caller's.
+    // The first word of the array counts finished CTAs of the counting kernel and must be
+    // zero when the counting kernel starts. A clean call leaves it at zero, but two calls
+    // that overlapped can leave it anywhere, so every call clears it on its stream first
+    // (a memset, no allocation): one race then corrupts only the calls that raced. The
+    // rest of the array is written before it is read. The status word is the caller's.
     unsigned int* counter = static_cast<unsigned int*>(scratch);
+    if (d->T > 0 && cudaMemsetAsync(counter, 0, sizeof(unsigned int), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return MOE_ERR_CUDA;
     cudaError_t e = moe::launch_permute(topk_ids, x, d->T, d->H, d->k, d->E, d->n_shared, fp8, offsets, perm,
                                         inv_perm, x_perm, x_scale, static_cast<char*>(scratch) + 256, counter, status,
                                         static_cast<cudaStream_t>(stream));

@@ -218,17 +218,23 @@ int moe_permute(const int32_t* topk_ids, const void* x, const moe_dims* dims,
  *   Arguments as moe_permute, except: no ws/ws_bytes; `status` is an optional device
  *   int32 (NULL = not reported) where a routing id outside [0, E) or repeated within a
  *   token is recorded (first error wins, the caller zeroes it).
+ *   Weight types: all four (BF16, FP8, INT4_G32, NVFP4), as moe_permute; only FP8
+ *   quantises x_perm, the others copy it in bf16.
  *   Scratch: a 1 MiB array compiled into the library, one per GPU that loads it, held
  *   until the process exits. Calls needing more -- 256-byte-rounded
- *   ceil(T/256)*E*4 + T*k*4 bytes above 1 MiB (about T > 16000 at k = 8, E = 288) --
- *   return MOE_ERR_WORKSPACE and enqueue nothing.
- *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   ceil(T/256)*E*4 + T*k*4 bytes above 1 MiB - 256 (at k = 8, E = 288: T >= 28689)
+ *   -- return MOE_ERR_WORKSPACE and enqueue nothing.
+ *   The array's device address is looked up (cudaGetSymbolAddress) in the current
+ *   context on every call made outside stream capture, so a context created after
+ *   cudaDeviceReset is served correctly. Under capture the address of the last
+ *   uncaptured call on the device is used: make one uncaptured call on each device
+ *   (and again after a reset) before capturing; a captured call with none before it
+ *   returns MOE_ERR_UNSUPPORTED.
  *   Every call shares the array: calls that overlap on the GPU (two streams, or two
  *   host threads) race and corrupt each other's results. Its first word counts the
- *   CTAs of a call that have finished counting and must be zero when a call starts: it
- *   is zero when the library loads and every call leaves it at zero; the rest of the
- *   array is written by each call before it is read.
+ *   CTAs of a call that have finished counting; every call first clears it on its own
+ *   stream (cudaMemsetAsync of 4 bytes), so a race damages only the calls that raced.
+ *   The rest of the array is written by each call before it is read.
  * Errors: INVALID_ARG, WORKSPACE (too large), ARCH, CUDA. */
 int moe_permute_noalloc(const int32_t* topk_ids, const void* x, const moe_dims* dims,
                         int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* x_perm,

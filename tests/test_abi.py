@@ -152,3 +152,25 @@ def test_4bit_weights_need_aligned_scales(L, wdtype):
                               None) == -1
     assert L.moe_gemm1_swiglu(fake, None, fake, fake, fake + 2, None, None, None, ctypes.byref(d), fake, None, fake,
                               n, None) == -1
+
+
+def _noalloc(L):
+    fn = L.moe_permute_noalloc
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(moe.MoeDims)] + [ctypes.c_void_p] * 7
+    fn.restype = ctypes.c_int
+    return fn
+
+
+def test_noalloc_size_limit_is_where_the_header_says(L):
+    """The static scratch holds 1 MiB - 256 bytes of counts and ranks; at k = 8, E = 288
+    the first size that does not fit is T = 28689. The refusal comes before any CUDA call,
+    so fake (never dereferenced) pointers are enough here; T = 28688 runs on the GPU."""
+    al = lambda b: (b + 255) & ~255
+    need = lambda T: al(((T + 255) // 256) * 288 * 4) + al(T * 8 * 4)
+    assert need(28688) <= (1 << 20) - 256 < need(28689)
+    fake = 1 << 20
+    for wd in (0, 1, 2, 3):  # the four weight types are accepted alike
+        d = _dims(T=28689, H=512, E=288, k=8, n_shared=1, n_sink=0, wdtype=wd, score=moe.MOE_SCORE_SIGMOID)
+        assert _noalloc(L)(fake, fake, ctypes.byref(d), fake, fake, fake, fake, fake, None, None) == -4
+    d = _dims(T=28689, H=512, E=288, k=8, n_shared=1, n_sink=0, wdtype=4)
+    assert _noalloc(L)(fake, fake, ctypes.byref(d), fake, fake, fake, fake, fake, None, None) == -1

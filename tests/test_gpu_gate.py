@@ -1,6 +1,7 @@
 """Fused gate GEMV + router (moe_gate_route) on the GPU: the logits against the fp64
 oracle GEMV within the fp32 summation bound, the routing against the oracle on the
-device's own fp32 logits (ids bit-exact, weights 1e-6), the packed form, and reuse."""
+device's own fp32 logits (ids bit-exact, weights 1e-6) and against the oracle's routing of
+its own fp64 logits wherever the top-k gaps exceed that bound, the packed form, and reuse."""
 import numpy as np
 import pytest
 import scipy.special
@@ -76,6 +77,25 @@ def test_gate_route_matches_oracle(T, H, N, S, k, score, bias_std):
         den = np.take_along_axis(sig, got_ids.astype(np.int64), 1).sum(1) + sig[:, N:].sum(1)
         want = np.take_along_axis(sig, got_ids.astype(np.int64), 1) / den[:, None]
         assert np.abs(got_w - want).max() <= TOL_WEIGHTS
+    # Routing of the oracle's own fp64 logits: wherever the fp64 gaps around the selection
+    # exceed twice the fp32 summation bound (plus the fp32 rounding of each side), the
+    # device's fp32 logits cannot reorder them, so its selection (and, where every gap in
+    # the top k + 1 is that wide, its slot order) must be the oracle's.
+    if bias is None:
+        r_ids, _, _ = oracle.route(ref.astype(np.float32), N, k, score)
+        n_set = n_order = 0
+        for t in range(T):
+            r = ref[t, :N]
+            tol = 2 * bound[t, :N].max() + 2 * float(np.spacing(np.float32(np.abs(r).max())))
+            order = np.lexsort((np.arange(N), -r))[:k + 1]
+            gaps = r[order[:-1]] - r[order[1:]]
+            if k == N or gaps[k - 1] > tol:
+                assert set(got_ids[t].tolist()) == set(r_ids[t].tolist()), t
+                n_set += 1
+            if k == N or gaps[:k].min() > tol:
+                assert np.array_equal(got_ids[t], r_ids[t]), t
+                n_order += 1
+        assert n_set >= 1, "no token's top-k gap exceeds the fp32 bound: the fp64 comparison checked nothing"
     pk = packed.cpu().numpy().view(np.uint32)
     wb = w.cpu().to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16).astype(np.uint32)
     assert np.array_equal(pk >> 16, got_ids.astype(np.uint32)) and np.array_equal(pk & 0xFFFF, wb)

@@ -19,8 +19,9 @@ from grouped_gemm_swiglu_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-def _dims(T, E, k, S, H, fp8):
-    return moe.MoeDims(T=T, H=H, I=128, E=E, k=k, n_sink=0, n_shared=S, wdtype=1 if fp8 else 0, score=0,
+def _dims(T, E, k, S, H, fp8, wdtype=None):
+    wd = (1 if fp8 else 0) if wdtype is None else wdtype
+    return moe.MoeDims(T=T, H=H, I=128, E=E, k=k, n_sink=0, n_shared=S, wdtype=wd, score=0,
                        alpha=1.0, beta=0.0, limit=float("inf"), route_scale=1.0)
 
 
@@ -33,10 +34,10 @@ def _outputs(d, fp8, dev="cuda"):
                 xs=torch.zeros((d.H // 128, A), dtype=torch.float32, device=dev) if fp8 else None)
 
 
-def _case(T, E, k, S, H, fp8, seed, skew=0.0):
+def _case(T, E, k, S, H, fp8, seed, skew=0.0, wdtype=None):
     ids = W.random_topk_ids(T, E, k, seed=seed, skew=skew).cuda()
     x = W.random_activations(T, H, seed=seed + 1, device="cuda").to(torch.bfloat16)
-    d = _dims(T, E, k, S, H, fp8)
+    d = _dims(T, E, k, S, H, fp8, wdtype)
     ref = _outputs(d, fp8)
     ws = moe.alloc_workspace(d, moe.MOE_WS_PERMUTE)
     moe.moe_permute(ids, x, d, ref["offsets"], ref["perm"], ref["inv"], ref["xp"], ref["xs"], ws)
@@ -98,3 +99,19 @@ def test_noalloc_refuses_sizes_beyond_its_scratch():
     fn.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(moe.MoeDims)] + [ctypes.c_void_p] * 7
     fn.restype = ctypes.c_int
     assert fn(fake, fake, ctypes.byref(d), fake, fake, fake, fake, None, None, None) == -4
+
+
+def test_noalloc_runs_at_its_largest_size_and_with_4bit_weight_types():
+    """T = 28688 at k = 8, E = 288 is the largest problem the static scratch holds (the
+    next size is refused: tests/test_abi.py); INT4 and NVFP4 layers permute bf16 rows
+    exactly as moe_permute does for them."""
+    cases = [(28688, 288, 8, 1, 128, False, 21, 0.0, None),
+             (500, 64, 4, 0, 256, False, 22, 0.0, 2),
+             (500, 64, 4, 2, 256, False, 23, 1.0, 3)]
+    for T, E, k, S, H, fp8, seed, skew, wd in cases:
+        ids, x, d, ref = _case(T, E, k, S, H, fp8, seed, skew, wd)
+        got = _outputs(d, fp8)
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        assert _call_noalloc(ids, x, d, got, status) == 0
+        _assert_same(got, ref, fp8)
+        assert int(status.item()) == 0
