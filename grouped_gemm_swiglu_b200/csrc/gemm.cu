@@ -46,6 +46,7 @@
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "internal.h"
@@ -63,10 +64,17 @@ constexpr int pow2_at_least(int v) {
     return p;
 }
 
-template <int BN_, bool FP8_, bool INT4_ = false>
+template <int BN_, bool FP8_, bool INT4_ = false, bool PAIR_ = false>
 struct Cfg {
     static constexpr int BN = BN_;
     static constexpr bool FP8 = FP8_;
+    // Two CTAs of a cluster share each MMA (cta_group::2, M = 256 token rows): each CTA
+    // loads its own 128 token rows and half of the 256 weight rows (the gate rows in the
+    // even CTA, the up rows in the odd one; GEMM2: one 128-row chunk of H each), so a CTA
+    // pulls 32 KB through L2 per 128-deep K block instead of 48 KB. A token block is then
+    // TB = 256 rows of a group.
+    static constexpr bool PAIR = PAIR_;
+    static constexpr int TB = PAIR ? 2 * BN : BN;  // token rows per block
     // INT4 group-32 weights: TMA brings the packed bytes (RAW_BYTES per 128x64 block) and
     // dequantisation warps write the bf16 weight tiles into tensor memory, where the MMA
     // takes its A operand; shared memory then holds only the token tile and packed bytes.
@@ -75,9 +83,10 @@ struct Cfg {
     static constexpr int A_BYTES = 128 * 128;
     static constexpr int B_BYTES = BN * 128;
     static constexpr int RAW_BYTES = INT4 ? 128 * 32 : 0;
-    static constexpr int B_OFF = INT4 ? 0 : 2 * A_BYTES;  // token tile within a stage
+    static constexpr int B_OFF = INT4 ? 0 : (PAIR ? A_BYTES : 2 * A_BYTES);  // token tile within a stage
     static constexpr int RAW_OFF = B_OFF + B_BYTES;        // INT4: packed A0, A1 after the token tile
-    static constexpr int STAGE_BYTES = INT4 ? B_BYTES + 2 * RAW_BYTES : 2 * A_BYTES + B_BYTES;  // GEMM1-sized
+    static constexpr int STAGE_BYTES =
+        INT4 ? B_BYTES + 2 * RAW_BYTES : (PAIR ? A_BYTES + B_BYTES : 2 * A_BYTES + B_BYTES);  // GEMM1-sized
     static constexpr int A_TMEM_COLS = 64;  // INT4: one stage's bf16 A0 | A1 (128 x 64 K, two K per column)
     // Dequantisation warps, in sets of four (a warp may only touch its TMEM lane quarter,
     // warp % 4, so a set covers the 128 rows of a tile). For decode-sized tiles (the
@@ -146,6 +155,7 @@ struct Cfg {
     static_assert(BN % BOX_ROWS == 0 && BN <= 256, "token tile = whole boxes, at most the MMA's N limit");
     static_assert(STAGES >= 2, "at least two pipeline stages");
     static_assert(!(INT4 && FP8), "INT4 weights take bf16 activations");
+    static_assert(!PAIR || (FP8 && WIDE && BN == 128), "the CTA pair is the token-major FP8 tile");
     static_assert(!INT4 || BN <= 64, "INT4 keeps its A tiles next to the accumulators in TMEM");
     static_assert(!INT4 || (DQG == 4 && DQG * NGRP == DQ), "dequantisation warps: stage groups of 4");
     static_assert(COLS % 8 == 0, "split-K merges columns in chunks of 8");
@@ -207,7 +217,7 @@ struct Tile {
 // All GEMM1 units are claimed before any GEMM2 tile (interleaving the GEMM2 tiles of a
 // block one or two waves after its GEMM1 units measured slower: they hold their SM while
 // waiting for inputs still in flight).
-template <int BN>
+template <int TB>
 __device__ __forceinline__ Tile decode_tile(int L, int T1, const int32_t* blk_start, const int32_t* s_off,
                                             const DevArgs& p) {
     Tile t;
@@ -233,8 +243,8 @@ __device__ __forceinline__ Tile decode_tile(int L, int T1, const int32_t* blk_st
     t.g = lo;
     const int g0 = s_off[lo];
     const int g1 = max(s_off[lo + 1], g0);
-    t.row0 = g0 + (t.blk - blk_start[lo]) * BN;
-    t.nrows = min(BN, g1 - t.row0);
+    t.row0 = g0 + (t.blk - blk_start[lo]) * TB;
+    t.nrows = min(TB, g1 - t.row0);
     if (t.phase == 1) {
         t.dual = true;
         t.a0row = t.g * 2 * p.I + t.c * 128;
@@ -248,6 +258,14 @@ __device__ __forceinline__ Tile decode_tile(int L, int T1, const int32_t* blk_st
         t.col1 = t.col0 + 128;
     }
     return t;
+}
+
+// The rows of a CTA-pair tile that CTA `rank` holds: 128 from row0 + 128 * rank (none
+// when the block's group ends before them).
+__device__ __forceinline__ void pair_rows(Tile& t, uint32_t rank) {
+    const int skip = 128 * (int)rank;
+    t.row0 += skip;
+    t.nrows = max(0, min(128, t.nrows - skip));
 }
 
 // g * sigmoid(alpha*g) * (u + beta) written as g*(u+beta) / (1 + exp(-alpha*g)): one
@@ -441,10 +459,12 @@ __device__ __forceinline__ void dequant_store(bool fp4, const uint8_t* raw, uint
     tmem_st32(at, w);
 }
 
-// Warp-collective bounded wait: lane 0 waits, the verdict is broadcast.
+// Warp-collective bounded wait: lane 0 waits, the verdict is broadcast. CL: the barrier
+// has arrivals from the other CTA of a pair (acquire at cluster scope).
+template <bool CL = false>
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, PipeAbort* ab, int* status) {
     bool ok = true;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, ab, status);
+    if ((threadIdx.x & 31) == 0) ok = CL ? mbar_wait_cl(bar, parity, ab, status) : mbar_wait(bar, parity, ab, status);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     __syncwarp();
     return ok;
@@ -478,20 +498,30 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.G;
+    // CTA pair: rank 1 mirrors rank 0's barriers but only rank 0's full, tempty and
+    // ring_empty count anything: the MMA (issued by rank 0) waits for both CTAs' copies
+    // (each CTA arrives once with its own byte count) and both CTAs' epilogues, and rank
+    // 0's producer, which claims the tiles and writes them into both CTAs' rings, waits
+    // for both CTAs' readers. `lead` maps a barrier to its copy in rank 0.
+    const uint32_t rank = C::PAIR ? cluster_ctarank() : 0u;
+    auto lead = [&](uint64_t* b) -> uint32_t { return mapa_shared(smem_u32(b), 0); };
+    auto peer = [&](const void* v) -> uint32_t { return mapa_shared(smem_u32(v), 1); };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&full[s], C::INT4 ? C::DQG : 1);  // INT4: the dequantisation warps complete it
+            // INT4: the dequantisation warps complete it; pair: one arrival per CTA
+            mbar_init(&full[s], C::INT4 ? C::DQG : (C::PAIR ? 2 : 1));
             if (C::INT4) mbar_init(&raw_full[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < C::NBUF; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], C::EPI);
+            mbar_init(&tempty[b], (C::PAIR ? 2 : 1) * C::EPI);
         }
         for (int r = 0; r < kRing; ++r) {
             mbar_init(&ring_full[r], 1);
-            mbar_init(&ring_empty[r], 1 + C::EPI + C::DQ + (C::WIDE ? 1 : 0));
+            // readers per CTA: MMA (rank 0) or producer (rank 1), the epilogue, the publisher
+            mbar_init(&ring_empty[r], C::PAIR ? 2 * (1 + C::EPI + 1) : 1 + C::EPI + C::DQ + (C::WIDE ? 1 : 0));
         }
         mbar_init(drain, 1);
         mbar_init(epibar, C::EPI);
@@ -500,20 +530,25 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (C::PAIR) {  // the same warp in both CTAs: one allocation at one address in both
+            tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, C::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     // Everything above is private to the SM; the offsets (and all other global data) come
     // from the previous kernels on the stream.
     pdl_wait();
-    // Token blocks per group and their running start: blk_start[g] = sum_{g'<g} ceil(n_g'/BN).
+    // Token blocks per group and their running start: blk_start[g] = sum_{g'<g} ceil(n_g'/TB).
     // The offsets may come from the caller: group bounds are clamped into [0, A] (and a
     // bad array is flagged), so no tile ever reads or writes a row outside the matrices.
     for (int g = threadIdx.x; g < G; g += blockDim.x) {
         const int o0 = __ldg(p.offsets + g), o1 = __ldg(p.offsets + g + 1);
         const int lo = min(max(o0, 0), p.A), hi = min(max(o1, lo), p.A);
         if (o0 != lo || o1 != hi) set_status(p.status, MOE_ERR_EXPERT_ID);
-        blk_start[g + 1] = (hi - lo + C::BN - 1) / C::BN;
+        blk_start[g + 1] = (hi - lo + C::TB - 1) / C::TB;
         s_off[g] = lo;
         if (g == G - 1) s_off[G] = min(max(o1, 0), p.A);
     }
@@ -536,6 +571,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     tc_fence_before();
     __syncthreads();
+    // pair: neither CTA signals the other's barriers before both have initialised them
+    if constexpr (C::PAIR) cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int nblk = blk_start[G];
@@ -558,46 +595,78 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 uint32_t stage = 0, phase = 0, pend_mask = 0, pend_phase = 0;
                 bool ok = true;
                 // Tiles are claimed one ahead, so the atomic's latency overlaps the current tile.
+                // In a CTA pair rank 0 claims and hands every tile number to rank 1 as well.
+                const bool claims = !C::PAIR || rank == 0;
                 auto claim = [&](int i) -> int {
-                    return p.tile_ctr ? (int)atomicAdd(p.tile_ctr, 1u) : (int)blockIdx.x + i * (int)gridDim.x;
+                    return p.tile_ctr ? (int)atomicAdd(p.tile_ctr, 1u) : (int)(blockIdx.x / (C::PAIR ? 2 : 1)) +
+                                                                          i * (int)(gridDim.x / (C::PAIR ? 2 : 1));
                 };
-                int next_L = claim(0);
+                int next_L = claims ? claim(0) : 0;
+                // Completion of a stage's copies: this CTA's full barrier, or rank 0's for a pair.
+                auto land = [&](uint32_t st) -> uint64_t* { return C::INT4 ? &raw_full[st] : &full[st]; };
+                auto load = [&](uint8_t* dst, const CUtensorMap* map, uint32_t st, int x, int y) {
+                    if constexpr (C::PAIR) tma_load_2d_pair(dst, map, lead(&full[st]), x, y);
+                    else tma_load_2d(dst, map, land(st), x, y);
+                };
                 for (int i = 0; ok; ++i) {
                     const int slot = i % kRing;
-                    int L = next_L;
-                    if (L >= total) L = -1;
-                    else next_L = claim(i + 1);
-                    if (!mbar_wait(&ring_empty[slot], ((i / kRing) & 1) ^ 1, ab, p.status)) break;
-                    ring[slot] = L;
-                    mbar_arrive(&ring_full[slot]);
+                    int L;
+                    if (claims) {
+                        L = next_L;
+                        if (L >= total) L = -1;
+                        else next_L = claim(i + 1);
+                        const bool free_slot = C::PAIR ? mbar_wait_cl(&ring_empty[slot], ((i / kRing) & 1) ^ 1, ab, p.status)
+                                                       : mbar_wait(&ring_empty[slot], ((i / kRing) & 1) ^ 1, ab, p.status);
+                        if (!free_slot) break;
+                        ring[slot] = L;
+                        if constexpr (C::PAIR) {  // rank 1's copy of the slot, then its ring_full
+                            st_cluster_u32(peer(&ring[slot]), (uint32_t)L);
+                            mbar_arrive_cluster(peer(&ring_full[slot]));
+                        }
+                        mbar_arrive(&ring_full[slot]);
+                    } else {  // pair rank 1: the tile number comes from rank 0
+                        if (!mbar_wait_cl(&ring_full[slot], (i / kRing) & 1, ab, p.status)) break;
+                        L = *reinterpret_cast<volatile int*>(&ring[slot]);
+                        mbar_arrive_cluster(lead(&ring_empty[slot]));
+                    }
                     if (L < 0) break;
-                    const Tile tl = decode_tile<C::BN>(L, T1, blk_start, s_off, p);
+                    Tile tl = decode_tile<C::TB>(L, T1, blk_start, s_off, p);
+                    if constexpr (C::PAIR) pair_rows(tl, rank);
                     const bool g1 = tl.phase == 1;
                     const CUtensorMap* tw = g1 ? &tmW1 : &tmW2;
                     const CUtensorMap* ta = g1 ? &tmX : &tmH;
                     const int all_kb = (g1 ? p.H : p.I) / C::BK;
                     const int kbase = g1 ? tl.ks * all_kb / p.s1 : 0;  // this tile's K blocks
                     const int num_kb = g1 ? (tl.ks + 1) * all_kb / p.s1 - kbase : all_kb;
-                    const int n_box = (max(16, (tl.nrows + 15) & ~15) + C::BOX_ROWS - 1) / C::BOX_ROWS;
-                    const uint32_t tx = (tl.dual ? 2 : 1) * (C::INT4 ? C::RAW_BYTES : C::A_BYTES) + n_box * C::BOX_BYTES;
-                    auto load_act = [&](uint8_t* st, uint64_t* bar, int kx) {
+                    // pair: a CTA with no rows of the block loads no token box (the MMA's rows
+                    // from it are never stored)
+                    const int n_box = (C::PAIR && tl.nrows <= 0)
+                                          ? 0
+                                          : (max(16, (tl.nrows + 15) & ~15) + C::BOX_ROWS - 1) / C::BOX_ROWS;
+                    // pair: one 128-row weight block per CTA (rank 1 takes A1; without A1 it
+                    // loads A0 again, and those accumulator columns are not stored)
+                    const int wrow = (C::PAIR && rank == 1 && tl.dual) ? tl.a1row : tl.a0row;
+                    const uint32_t tx = (C::PAIR ? 1 : (tl.dual ? 2 : 1)) * (C::INT4 ? C::RAW_BYTES : C::A_BYTES) +
+                                        n_box * C::BOX_BYTES;
+                    auto load_act = [&](uint8_t* st, uint32_t s_idx, int kx) {
                         for (int r = 0; r < n_box; ++r)
-                            tma_load_2d(st + C::B_OFF + r * C::BOX_BYTES, ta, bar, kx, tl.row0 + r * C::BOX_ROWS);
+                            load(st + C::B_OFF + r * C::BOX_BYTES, ta, s_idx, kx, tl.row0 + r * C::BOX_ROWS);
                     };
                     // GEMM2 after GEMM1 in the same launch: weights of the first stages go out
                     // before waiting for the block's h rows.
                     const bool dep = chained && !g1;
                     const int pre = dep ? min(num_kb, C::STAGES) : 0;
                     const uint32_t st0 = stage;
-                    // Wait for the block's h rows, then load the activation rows of the
-                    // prefetched stages. They are loaded even when the wait gave up (the rows
-                    // are in bounds; the results are discarded), so every armed stage completes.
+                    // Wait for the block's h rows (pair: this CTA's half of the block), then
+                    // load the activation rows of the prefetched stages. They are loaded even
+                    // when the wait gave up (the rows are in bounds; the results are
+                    // discarded), so every armed stage completes.
                     auto release_prefetched = [&]() -> bool {
-                        const bool dep_ok = wait_counter_geq(p.done1 + tl.blk, p.c1, ab, p.status);
+                        const int ctr = C::PAIR ? 2 * tl.blk + (int)rank : tl.blk;
+                        const bool dep_ok = wait_counter_geq(p.done1 + ctr, p.c1, ab, p.status);
                         uint32_t s2 = st0;
                         for (int k2 = 0; k2 < pre; ++k2) {
-                            load_act(smem + (size_t)s2 * C::STAGE_BYTES, C::INT4 ? &raw_full[s2] : &full[s2],
-                                     (kbase + k2) * C::BK);
+                            load_act(smem + (size_t)s2 * C::STAGE_BYTES, s2, (kbase + k2) * C::BK);
                             if (++s2 == (uint32_t)C::STAGES) s2 = 0;
                         }
                         return dep_ok;
@@ -607,22 +676,26 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                             ok = false;
                             break;
                         }
-                        if (!mbar_wait(&empty[stage], phase ^ 1, ab, p.status)) {
+                        const bool free_stage = C::PAIR ? mbar_wait_cl(&empty[stage], phase ^ 1, ab, p.status)
+                                                        : mbar_wait(&empty[stage], phase ^ 1, ab, p.status);
+                        if (!free_stage) {
                             ok = false;
                             break;
                         }
                         uint8_t* st = smem + (size_t)stage * C::STAGE_BYTES;
-                        uint64_t* bar = C::INT4 ? &raw_full[stage] : &full[stage];
-                        mbar_arrive_expect_tx(bar, tx);
+                        if constexpr (C::PAIR) mbar_arrive_expect_tx_cluster(lead(&full[stage]), tx);
+                        else mbar_arrive_expect_tx(land(stage), tx);
                         const int kx = (kbase + kb) * C::BK;
                         if constexpr (C::INT4) {  // packed weight bytes: x is a byte offset (2 K per byte)
-                            tma_load_2d(st + C::RAW_OFF, tw, bar, kx / 2, tl.a0row);
-                            if (tl.dual) tma_load_2d(st + C::RAW_OFF + C::RAW_BYTES, tw, bar, kx / 2, tl.a1row);
+                            load(st + C::RAW_OFF, tw, stage, kx / 2, tl.a0row);
+                            if (tl.dual) load(st + C::RAW_OFF + C::RAW_BYTES, tw, stage, kx / 2, tl.a1row);
+                        } else if constexpr (C::PAIR) {
+                            load(st, tw, stage, kx, wrow);
                         } else {
-                            tma_load_2d(st, tw, bar, kx, tl.a0row);
-                            if (tl.dual) tma_load_2d(st + C::A_BYTES, tw, bar, kx, tl.a1row);
+                            load(st, tw, stage, kx, tl.a0row);
+                            if (tl.dual) load(st + C::A_BYTES, tw, stage, kx, tl.a1row);
                         }
-                        if (kb >= pre) load_act(st, bar, kx);
+                        if (kb >= pre) load_act(st, stage, kx);
                         pend_mask |= 1u << stage;
                         pend_phase = (pend_phase & ~(1u << stage)) | (phase << stage);
                         if (++stage == (uint32_t)C::STAGES) {
@@ -633,14 +706,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     if (ok && dep && pre == num_kb && !release_prefetched()) ok = false;  // whole K prefetched
                 }
                 // Never leave with a copy in flight: wait for the last fill of every stage.
-                for (int s = 0; s < C::STAGES; ++s)
-                    if ((pend_mask >> s) & 1u)
-                        mbar_wait_drain(C::INT4 ? &raw_full[s] : &full[s], (pend_phase >> s) & 1u);
+                // (pair: rank 0's full barrier counts both CTAs' copies; rank 1 is held at
+                // the kernel's final cluster barrier until rank 0 has drained)
+                if (!C::PAIR || rank == 0)
+                    for (int s = 0; s < C::STAGES; ++s)
+                        if ((pend_mask >> s) & 1u) {
+                            if constexpr (C::PAIR) mbar_wait_drain_cl(&full[s], (pend_phase >> s) & 1u);
+                            else mbar_wait_drain(land(s), (pend_phase >> s) & 1u);
+                        }
             }
             __syncwarp();
         } else if (warp == 1) {
             // ------------------------------------------------------------ MMA issuer
-            if (lane == 0) {
+            // (pair: rank 0 issues for both CTAs; rank 1's warp only owns its TMEM share)
+            if (lane == 0 && (!C::PAIR || rank == 0)) {
                 uint32_t stage = 0, phase = 0, it = 0;
                 bool ok = true;
                 for (int i = 0; ok; ++i) {
@@ -649,28 +728,35 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     const int L = ring[slot];
                     mbar_arrive(&ring_empty[slot]);
                     if (L < 0) break;
-                    const Tile tl = decode_tile<C::BN>(L, T1, blk_start, s_off, p);
+                    const Tile tl = decode_tile<C::TB>(L, T1, blk_start, s_off, p);
                     const bool g1 = tl.phase == 1;
                     const int all_kb = (g1 ? p.H : p.I) / C::BK;
                     const int kbase = g1 ? tl.ks * all_kb / p.s1 : 0;
                     const int num_kb = g1 ? (tl.ks + 1) * all_kb / p.s1 - kbase : all_kb;
                     const int n_mma = max(16, (tl.nrows + 15) & ~15);
                     // wide FP8: M = the 128 token rows, N = the 256 (or 128) weight rows
-                    const uint32_t idesc = C::WIDE ? idesc_m128(tl.dual ? 256 : 128, true) : idesc_m128(n_mma, C::FP8);
+                    // pair: M = 2 x 128 token rows, N = 2 x 128 weight rows (one block from each CTA)
+                    const uint32_t idesc = C::PAIR ? idesc_m256_fp8(256)
+                                                   : (C::WIDE ? idesc_m128(tl.dual ? 256 : 128, true)
+                                                              : idesc_m128(n_mma, C::FP8));
                     // bf16: one TMEM buffer per tile; FP8: one per 128-deep K block
                     const int units = C::FP8 ? num_kb : 1;
                     const int kb_per_unit = C::FP8 ? 1 : num_kb;
                     int kb = 0;
                     for (int u = 0; u < units && ok; ++u) {
                         const uint32_t buf = it % C::NBUF, bph = (it / C::NBUF) & 1;
-                        if (!mbar_wait(&tempty[buf], bph ^ 1, ab, p.status)) {
+                        const bool drained = C::PAIR ? mbar_wait_cl(&tempty[buf], bph ^ 1, ab, p.status)
+                                                     : mbar_wait(&tempty[buf], bph ^ 1, ab, p.status);
+                        if (!drained) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                         const uint32_t d0 = tmem_base + buf * C::ACC_COLS;
                         for (int j = 0; j < kb_per_unit; ++j, ++kb) {
-                            if (!mbar_wait(&full[stage], phase, ab, p.status)) {
+                            const bool landed = C::PAIR ? mbar_wait_cl(&full[stage], phase, ab, p.status)
+                                                        : mbar_wait(&full[stage], phase, ab, p.status);
+                            if (!landed) {
                                 ok = false;
                                 break;
                             }
@@ -685,6 +771,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                 if constexpr (C::INT4) {
                                     mma_bf16_tmem_a(d0, at + kk * 8, bd, idesc, acc);
                                     if (tl.dual) mma_bf16_tmem_a(d0 + C::BN, at + 32 + kk * 8, bd, idesc, acc);
+                                } else if constexpr (C::PAIR) {
+                                    // token tiles (A, 128 rows per CTA) x weight blocks (B, 128 rows per CTA)
+                                    mma_fp8_pair(d0, bd, smem_desc_sw128(a0 + kk * 32), idesc, acc);
                                 } else if constexpr (C::WIDE) {
                                     // the token tile is the A operand; A0 | A1 (contiguous) the B operand
                                     mma_fp8(d0, bd, smem_desc_sw128(a0 + kk * 32), idesc, acc);
@@ -698,19 +787,23 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                         mma_bf16(d0 + C::BN, smem_desc_sw128(a0 + C::A_BYTES + kk * 32), bd, idesc, acc);
                                 }
                             }
-                            tc_commit(&empty[stage]);
+                            // the stage is free in both CTAs once these MMAs have read it
+                            if constexpr (C::PAIR) tc_commit_pair_both(&empty[stage]);
+                            else tc_commit(&empty[stage]);
                             if (++stage == (uint32_t)C::STAGES) {
                                 stage = 0;
                                 phase ^= 1;
                             }
                         }
                         if (!ok) break;
-                        tc_commit(&tfull[buf]);
+                        if constexpr (C::PAIR) tc_commit_pair_both(&tfull[buf]);
+                        else tc_commit(&tfull[buf]);
                         ++it;
                     }
                 }
                 // All MMAs issued by this thread complete before TMEM is released.
-                tc_commit(drain);
+                if constexpr (C::PAIR) tc_commit_pair(drain);
+                else tc_commit(drain);
                 mbar_wait_drain(drain, 0);
             }
             __syncwarp();
@@ -724,16 +817,21 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 uint32_t pph = 0;
                 for (int i = 0;; ++i) {
                     const int slot = i % kRing;
-                    if (!mbar_wait(&ring_full[slot], (i / kRing) & 1, ab, p.status)) break;
-                    const int L = ring[slot];
-                    mbar_arrive(&ring_empty[slot]);
+                    const bool got = C::PAIR ? mbar_wait_cl(&ring_full[slot], (i / kRing) & 1, ab, p.status)
+                                             : mbar_wait(&ring_full[slot], (i / kRing) & 1, ab, p.status);
+                    if (!got) break;
+                    const int L = *reinterpret_cast<volatile int*>(&ring[slot]);
+                    if constexpr (C::PAIR) mbar_arrive_cluster(lead(&ring_empty[slot]));
+                    else mbar_arrive(&ring_empty[slot]);
                     if (L < 0) break;
                     if (!chained || L >= T1) continue;  // GEMM1 tiles of a two-phase launch only
                     if (!mbar_wait(pubbar, pph, ab, p.status)) break;
                     pph ^= 1;
                     __threadfence();
                     fence_proxy_async_global();
-                    red_release_add_gpu(p.done1 + (L / p.s1) / p.c1, 1);
+                    // pair: one counter per 128-row half of the block, completed by this CTA's tiles
+                    const int blk = (L / p.s1) / p.c1;
+                    red_release_add_gpu(p.done1 + (C::PAIR ? 2 * blk + (int)rank : blk), 1);
                 }
             }
             __syncwarp();
@@ -755,7 +853,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&ring_empty[slot]);
             if (L < 0) break;
-            const Tile tl = decode_tile<C::BN>(L, T1, blk_start, s_off, p);
+            const Tile tl = decode_tile<C::TB>(L, T1, blk_start, s_off, p);
             const bool g1 = tl.phase == 1;
             const int K = g1 ? p.H : p.I;
             const int all_kb = K / C::BK;
@@ -851,12 +949,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         };
         for (int i = 0; ok; ++i) {
             const int slot = i % kRing;
-            if (!warp_wait(&ring_full[slot], (i / kRing) & 1, ab, p.status)) break;
-            const int L = ring[slot];
+            if (!warp_wait<C::PAIR>(&ring_full[slot], (i / kRing) & 1, ab, p.status)) break;
+            const int L = *reinterpret_cast<volatile int*>(&ring[slot]);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ring_empty[slot]);
+            if (lane == 0) {
+                if constexpr (C::PAIR) mbar_arrive_cluster(lead(&ring_empty[slot]));
+                else mbar_arrive(&ring_empty[slot]);
+            }
             if (L < 0) break;
-            const Tile tl = decode_tile<C::BN>(L, T1, blk_start, s_off, p);
+            Tile tl = decode_tile<C::TB>(L, T1, blk_start, s_off, p);
+            if constexpr (C::PAIR) pair_rows(tl, rank);
             const bool g1 = tl.phase == 1;
             const int n_mma = max(16, (tl.nrows + 15) & ~15);
             // output columns of this thread: A0's and A1's row (intermediate or hidden index)
@@ -973,7 +1075,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const float* wsu = wscale + (size_t)(tl.a1row / 128) * num_kb;
                 if (!g1 && chained) {  // h_scale comes from GEMM1 tiles of this block (see below)
                     bool dep_ok = true;
-                    if (lane == 0) dep_ok = wait_counter_geq(p.done1 + tl.blk, p.c1, ab, p.status);
+                    const int ctr = C::PAIR ? 2 * tl.blk + (int)rank : tl.blk;
+                    if (lane == 0) dep_ok = wait_counter_geq(p.done1 + ctr, p.c1, ab, p.status);
                     dep_ok = __shfl_sync(0xffffffffu, dep_ok ? 1 : 0, 0) != 0;
                     __syncwarp();
                     if (!dep_ok) {
@@ -1010,17 +1113,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         q_s0[kPF - 1] = in ? __ldg(wsg + kn) : 0.f;
                         q_s1[kPF - 1] = (in && tl.dual) ? __ldg(wsu + kn) : 0.f;
                     }
-                    if (!warp_wait(&tfull[buf], bph, ab, p.status)) {
+                    if (!warp_wait<C::PAIR>(&tfull[buf], bph, ab, p.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t tb = tmem_base + lane_off + buf * C::ACC_COLS + cg * CC;
-                    if (!quarter_live) {  // no token of this lane quarter in the tile
+                    // the buffer goes back to the MMA (pair: to rank 0, which issues it)
+                    auto release = [&]() {
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&tempty[buf]);
-                    }
+                        if (lane == 0) {
+                            if constexpr (C::PAIR) mbar_arrive_cluster(lead(&tempty[buf]));
+                            else mbar_arrive(&tempty[buf]);
+                        }
+                    };
+                    if (!quarter_live) release();  // no token of this lane quarter in the tile
                     constexpr int W = C::WCH;
 #pragma unroll
                     for (int ch = 0; ch < CC / W; ++ch) {
@@ -1028,11 +1136,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         float p0[W], p1[W];
                         if (tl.dual) tmem_ld_x2<W>(tb + ch * W, tb + C::BN + ch * W, p0, p1);
                         else tmem_ld_x1<W>(tb + ch * W, p0);
-                        if (ch == CC / W - 1) {  // the buffer goes back to the MMA before the arithmetic
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(&tempty[buf]);
-                        }
+                        if (ch == CC / W - 1) release();  // before the arithmetic
 #pragma unroll
                         for (int j = 0; j < W; j += 2) {
                             ffma2(acc0[ch * W + j], acc0[ch * W + j + 1], p0[j], p0[j + 1], f0, f0);
@@ -1308,9 +1412,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
     pdl_trigger();  // this CTA has no tiles left: the next kernel may launch
     __syncthreads();
+    // pair: rank 0 has drained its MMAs (which write rank 1's TMEM and read rank 1's
+    // shared memory) and its copies before either CTA frees TMEM or exits
+    if constexpr (C::PAIR) cluster_sync_all();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::TMEM_COLS);
+        if constexpr (C::PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+        else tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
     // The CTA that finishes last leaves the tile counter, the exit counter and the block
     // flags at zero for the next launch.
@@ -1326,8 +1434,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     __syncthreads();
     if (*s_last) {
-        if (chained)
-            for (int b = threadIdx.x; b < nblk; b += blockDim.x) p.done1[b] = 0;
+        if (chained)  // pair: two counters per block
+            for (int b = threadIdx.x; b < (C::PAIR ? 2 : 1) * nblk; b += blockDim.x) p.done1[b] = 0;
         if (p.s1 > 1)
             for (int t = threadIdx.x; t < nblk * p.c1; t += blockDim.x) p.split_cnt[t] = 0;
         if (threadIdx.x == 0) {
@@ -1391,6 +1499,55 @@ int num_sms() {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (dev < 64) cache[dev] = n;
     return n;
+}
+
+// Launch as clusters of two CTAs (the CTA-pair tile), with programmatic dependent launch.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pair_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                   Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// CTAs of a persistent pair launch: two per cluster that can be resident at once (one
+// CTA per SM; a GPC with an odd number of free SMs leaves one idle).
+template <class C>
+static int pair_grid(size_t smem) {
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 64 && cache[dev]) return cache[dev];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (num_sms() / 2));
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, moe_gemm_kernel<C>, &cfg) != cudaSuccess) return 0;
+    const int g = std::min(2 * n, 2 * (num_sms() / 2));
+    if (dev < 64) cache[dev] = g;
+    return g;
 }
 
 template <class C>
@@ -1469,14 +1626,28 @@ static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
         }
     }
     if (smem > (size_t)limit) return cudaErrorInvalidValue;
-    return launch_pdl(moe_gemm_kernel<C>, dim3(num_sms()), dim3(C::THREADS), smem, stream, tmW1, tmX, tmW2, tmH, p);
+    if constexpr (C::PAIR) {
+        // the occupancy query is taken at the largest dynamic shared memory the kernel may use
+        const int grid = pair_grid<C>((size_t)limit);
+        if (grid < 2) return cudaErrorInvalidConfiguration;
+        return launch_pair_pdl(moe_gemm_kernel<C>, dim3(grid), dim3(C::THREADS), smem, stream, tmW1, tmX, tmW2, tmH,
+                               p);
+    } else {
+        return launch_pdl(moe_gemm_kernel<C>, dim3(num_sms()), dim3(C::THREADS), smem, stream, tmW1, tmX, tmW2, tmH,
+                          p);
+    }
 }
 
 int gemm_pick_bn(int64_t A, int G, int wdtype) {
     const double avg = G > 0 ? (double)A / (double)G : 0.0;
     int bn = 16;
     while (bn < 256 && bn < avg) bn <<= 1;  // smallest tile holding an average group
-    if (wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128 && bn > 128) bn = 128;  // fp32 promotion registers for gate and up
+    // FP8 at 256 is the CTA pair (2 x 128 token rows); it needs two GEMM1 completion
+    // counters per 256-row block within the workspace's block flags (true whenever
+    // groups average more than 128 rows)
+    if (wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128 && bn > 128 &&
+        2 * gemm_max_blocks(A, G, 256) + 1 > gemm_max_blocks(A, G, 16) + 1)
+        bn = 128;
     if ((wdtype == MOE_WDTYPE_INT4_G32 || wdtype == MOE_WDTYPE_NVFP4) && bn > 64)
         bn = 64;  // 4-bit weights: A tiles share TMEM with the accumulators
     return bn;
@@ -1536,6 +1707,7 @@ cudaError_t launch_moe_gemm(const MoeGemmArgs& a, cudaStream_t stream) {
             case 32: return launch_cfg<Cfg<32, true>>(a, stream);
             case 64: return launch_cfg<Cfg<64, true>>(a, stream);
             case 128: return launch_cfg<Cfg<128, true>>(a, stream);
+            case 256: return launch_cfg<Cfg<128, true, false, true>>(a, stream);  // CTA pair
             default: return cudaErrorInvalidValue;
         }
     }

@@ -389,6 +389,155 @@ __device__ __forceinline__ void tmem_ld_x1(uint32_t ta, float* a) {
     else tmem_ld4(ta, a);
 }
 
+// ------------------------------------------------------------------ CTA pairs
+// Two CTAs of a cluster of two share one tcgen05.mma (cta_group::2): the MMA issued by
+// the even CTA (rank 0) reads half of each operand from each CTA's shared memory at the
+// same offsets and writes each CTA's half of the accumulator into that CTA's TMEM. Every
+// tcgen05 allocation, MMA and commit of such a kernel carries cta_group::2.
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// The shared::cluster address of the variable at `smem_addr` (a shared::cta address of
+// this CTA) in the shared memory of cluster CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t smem_addr, uint32_t rank) {
+    uint32_t d;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(smem_addr), "r"(rank));
+    return d;
+}
+
+// Arrive on an mbarrier anywhere in the cluster (release at cluster scope, so this
+// thread's earlier shared-memory writes, local or remote, are visible to the waiter).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_addr, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_addr),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// Acquire-at-cluster-scope variant of mbar_try_wait, for barriers that other CTAs of the
+// cluster arrive on.
+__device__ __forceinline__ bool mbar_try_wait_cl(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(20000u)
+        : "memory");
+    return ok != 0;
+}
+
+// mbar_wait for a barrier with arrivals from the other CTA of the pair: same bound and
+// abort rule.
+__device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, PipeAbort* ab, int* status) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait_cl(a, parity)) return true;
+    const long long t0 = clock64();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait_cl(a, parity)) return true;
+        if ((n & 15) == 0) {
+            if (ab->flag) return false;
+            if (clock64() - t0 > kWaitLimitCycles) {
+                ab->flag = 1;
+                if (status) atomicCAS(status, 0, MOE_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ bool mbar_wait_drain_cl(uint64_t* bar, uint32_t parity) {
+    const uint32_t a = smem_u32(bar);
+    const long long t0 = clock64();
+    while (!mbar_try_wait_cl(a, parity)) {
+        if (clock64() - t0 > kWaitLimitCycles) return false;
+    }
+    return true;
+}
+
+// Every thread of both CTAs (aligned: whole warps).
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Tile load into this CTA's shared memory whose completion (transaction bytes) is
+// signalled on the mbarrier at `bar_cluster_addr`, which may be the pair's other CTA's
+// (the MMA-issuing CTA waits for both halves on one barrier). No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar_cluster_addr,
+                                                 int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y)
+        : "memory");
+}
+
+// TMEM allocation for a CTA pair: one warp of each CTA (the same warp index) executes it.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Arrive once on `bar` (this CTA's) when the pair MMAs issued so far are done.
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// Arrive once on the mbarrier at `bar`'s offset in every CTA of `cta_mask` (both CTAs
+// of the pair: 0b11) when the pair MMAs issued so far are done. This is the completion
+// signal of the tensor core, not a memory copy.
+__device__ __forceinline__ void tc_commit_pair_both(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"((uint16_t)3)
+        : "memory");
+}
+
+// Pair MMA, E4M3 operands, fp32 accumulate: M = 256 (128 rows of A from each CTA), N
+// from the instruction descriptor (half of B's rows from each CTA).
+__device__ __forceinline__ void mma_fp8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Instruction descriptor of the pair MMA: D fp32, E4M3 A/B K-major, M = 256, N = n.
+__device__ __forceinline__ uint32_t idesc_m256_fp8(int n) {
+    uint32_t d = 0;
+    d |= 1u << 4;                     // D format: f32
+    d |= (uint32_t)(n >> 3) << 17;    // N >> 3
+    d |= (uint32_t)(256 >> 4) << 24;  // M >> 4
+    return d;
+}
+
 // Register reallocation between warpgroups: every warp of a warpgroup executes the same
 // instruction. dec returns registers to the CTA's pool, inc blocks until the pool holds
 // enough; the launch's threads x registers must cover the largest split.

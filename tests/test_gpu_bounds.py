@@ -2,8 +2,8 @@
 moe_forward and of the stage calls, and each workspace, sits inside a larger allocation
 whose head and tail hold a canary byte pattern. After the calls every canary is intact and
 the results match the oracle. Tiny and odd shapes: one expert with k = 1, one token with
-sinks and shared experts, T = 3 and T = 37 with ragged groups, FP8 (both tile layouts) and
-INT4 weights."""
+sinks and shared experts, T = 3 and T = 37 with ragged groups, FP8 (all three tile layouts:
+narrow, token-major, CTA pair) and INT4 weights."""
 import math
 
 import numpy as np
@@ -31,8 +31,12 @@ SHAPES = [
                score=W.SCORE_SIGMOID),
     W.Workload("t37_nvfp4_scales", T=37, H=512, I=256, E=8, k=2, n_shared=1, wdtype=W.WDTYPE_NVFP4,
                score=W.SCORE_SIGMOID, expert_scales=(0.52, 1.22)),
-    # about 150 rows per group: the token-major 128-token FP8 tile, with ragged tails
-    W.Workload("t300_fp8_wide", T=300, H=512, I=384, E=4, k=2, n_shared=1, wdtype=W.WDTYPE_FP8,
+    # about 100 rows per group: the token-major 128-token FP8 tile, with ragged tails
+    W.Workload("t300_fp8_wide", T=300, H=512, I=384, E=8, k=2, n_shared=1, wdtype=W.WDTYPE_FP8,
+               score=W.SCORE_SIGMOID, limit=10.0),
+    # about 180 rows per group: the FP8 CTA pair (256-row blocks, 128 rows per CTA); the
+    # shared group's second block has 44 rows, so one CTA of that pair holds none
+    W.Workload("t300_fp8_pair", T=300, H=512, I=384, E=4, k=2, n_shared=1, wdtype=W.WDTYPE_FP8,
                score=W.SCORE_SIGMOID, limit=10.0),
 ]
 

@@ -47,6 +47,22 @@ def test_forward_matches_oracle(name):
         assert_bf16_close(got, ref, name)
 
 
+# FP8 at a size the oracle covers token by token, in the CTA-pair layout the GLM-shaped
+# prefill uses (groups of about 540 rows: two to three 256-row blocks each, ragged tails),
+# with the GLM parameters (sigmoid routing, L = 10, one shared expert)
+PAIR_FULL = W.Workload("glm_fp8_t1024", T=1024, H=1024, I=512, E=16, k=8, n_shared=1, wdtype=W.WDTYPE_FP8,
+                       score=W.SCORE_SIGMOID, limit=10.0)
+
+
+def test_forward_fp8_pair_every_token():
+    wl = PAIR_FULL
+    inp = W.make_inputs(wl, "cuda")
+    out, ids, tw, sw, layer = run_forward(wl, inp)
+    assert layer.status() == 0
+    ref = oracle_layer(wl, inp).moe_rows(np.arange(wl.T, dtype=np.int32))
+    assert_fp8_close(out.float().cpu().numpy(), ref, wl.name)
+
+
 def test_forward_is_deterministic_and_reusable():
     wl = W.WORKLOADS["oai_swiglu"]
     inp = W.make_inputs(wl, "cuda")

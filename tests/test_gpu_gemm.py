@@ -1,6 +1,7 @@
 """Grouped GEMM1 (+ SwiGLU epilogue) and GEMM2 (+ weighted combine) on the GPU against
 the oracle, on synthetic permuted inputs that span several tiles, every token-tile width
-(16/32/64/128/256 rows), ragged group tails, empty groups and shared groups."""
+(16/32/64/128/256 rows, and FP8's two-CTA 256-row pair), ragged group tails, empty groups
+and shared groups."""
 import math
 
 import numpy as np
@@ -101,6 +102,11 @@ GEMM1_CASES = [
     (1024, 8, 2, 1, 512, 384, True, {"skew": 2.0, "scales": True, "limits": True}),  # FP8 tile 128, ragged, shared
     (40, 32, 4, 1, 512, 256, True, {"glm": True}),              # FP8, tile 16, shared group, L = 10
     (200, 8, 2, 0, 1024, 512, True, {"oai": True, "scales": True}),
+    # FP8 CTA pair (groups above 128 rows on average: 256-row token blocks, 128 per CTA);
+    # heavy skew leaves some groups under 128 rows (the odd CTA holds none of them) and
+    # some over 256 (several blocks); a shared group of T rows
+    (1500, 16, 2, 1, 512, 256, True, {"skew": 4.0, "oai": True}),
+    (700, 4, 2, 0, 1024, 384, True, {"scales": True, "limits": True}),
     (128, 8, 2, 1, 512, 384, False, {"limits": True}),          # a clamp per expert (shared group too)
     (300, 16, 4, 0, 512, 256, True, {"limits": True, "scales": True}),  # FP8, tile 32, clamp per expert
     (8, 64, 4, 0, 256, 256, False, {"int4": True}),            # INT4 group-32 weights: tile 16, split-K
@@ -164,7 +170,9 @@ GEMM2_CASES = [
     (600, 4, 2, 1, 384, 256, False, True),      # tile 256, odd number of 128-row chunks of H
     (512, 8, 2, 0, 512, 256, True, False),      # FP8, tile 128
     (256, 8, 2, 0, 512, 256, True, False),      # FP8, tile 64
-    (600, 4, 2, 1, 384, 256, True, True),       # FP8, tile 128, odd chunk count of H, sink-gated shared
+    (600, 4, 2, 1, 384, 256, True, True),       # FP8 CTA pair, odd chunk count of H, sink-gated shared
+    (1500, 16, 2, 1, 384, 256, True, False),    # FP8 CTA pair, skewless, odd chunk count of H
+    (300, 8, 2, 1, 512, 256, True, False),      # FP8, tile 128 (single CTA), shared group
     (40, 32, 4, 1, 512, 256, True, False),
     (8, 64, 4, 0, 256, 256, "int4", False),     # INT4 weights, tile 16
     (300, 16, 4, 2, 512, 256, "int4", True),    # INT4, sink-gated shared groups
