@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
         P = ctypes.POINTER(MoeDims)
         sig = {
             "moe_abi_version": ([], ctypes.c_int),
+            "moe_set_option": ([ctypes.c_int, ctypes.c_int], ctypes.c_int),
             "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
             "moe_workspace_size": ([P, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
             "moe_read_status": ([_VP, ctypes.POINTER(ctypes.c_int32), _VP], ctypes.c_int),
@@ -134,6 +135,18 @@ def _check(fn: str, rc: int):
 
 def moe_abi_version() -> int:
     return int(lib().moe_abi_version())
+
+
+MOE_OPT_FP8_CTA_PAIR = 1
+
+
+def moe_set_option(option: int, value: int) -> int:
+    """Process-wide kernel-layout option (see moe_set_option in the header); returns the
+    previous value."""
+    rc = int(lib().moe_set_option(int(option), int(value)))
+    if rc < 0:
+        raise MoeError("moe_set_option", rc)
+    return rc
 
 
 def moe_workspace_size(dims: MoeDims, kind: int) -> int:

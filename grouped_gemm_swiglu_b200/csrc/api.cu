@@ -199,6 +199,11 @@ extern "C" {
 
 int moe_abi_version(void) { return MOE_ABI_VERSION; }
 
+int moe_set_option(int option, int value) {
+    if (option == MOE_OPT_FP8_CTA_PAIR && (value == 0 || value == 1)) return gemm_set_fp8_pair(value);
+    return MOE_ERR_INVALID_ARG;
+}
+
 const char* moe_status_string(int status) {
     switch (status) {
         case MOE_OK: return "ok";

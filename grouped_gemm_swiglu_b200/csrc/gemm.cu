@@ -47,6 +47,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "internal.h"
@@ -500,17 +501,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int G = p.G;
     // CTA pair: rank 1 mirrors rank 0's barriers but only rank 0's full, tempty and
     // ring_empty count anything: the MMA (issued by rank 0) waits for both CTAs' copies
-    // (each CTA arrives once with its own byte count) and both CTAs' epilogues, and rank
-    // 0's producer, which claims the tiles and writes them into both CTAs' rings, waits
-    // for both CTAs' readers. `lead` maps a barrier to its copy in rank 0.
+    // (rank 0 arms the stage with both CTAs' byte counts; rank 1's copies complete their
+    // bytes on rank 0's barrier) and both CTAs' epilogues, and rank 0's producer, which
+    // claims the tiles and writes them into both CTAs' rings, waits for both CTAs'
+    // readers. `lead` maps a barrier to its copy in rank 0.
     const uint32_t rank = C::PAIR ? cluster_ctarank() : 0u;
     auto lead = [&](uint64_t* b) -> uint32_t { return mapa_shared(smem_u32(b), 0); };
     auto peer = [&](const void* v) -> uint32_t { return mapa_shared(smem_u32(v), 1); };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            // INT4: the dequantisation warps complete it; pair: one arrival per CTA
-            mbar_init(&full[s], C::INT4 ? C::DQG : (C::PAIR ? 2 : 1));
+            mbar_init(&full[s], C::INT4 ? C::DQG : 1);  // INT4: the dequantisation warps complete it
             if (C::INT4) mbar_init(&raw_full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -631,6 +632,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     }
                     if (L < 0) break;
                     Tile tl = decode_tile<C::TB>(L, T1, blk_start, s_off, p);
+                    const int blk_rows = tl.nrows;  // pair: rows of the whole 256-row block
                     if constexpr (C::PAIR) pair_rows(tl, rank);
                     const bool g1 = tl.phase == 1;
                     const CUtensorMap* tw = g1 ? &tmW1 : &tmW2;
@@ -638,16 +640,21 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     const int all_kb = (g1 ? p.H : p.I) / C::BK;
                     const int kbase = g1 ? tl.ks * all_kb / p.s1 : 0;  // this tile's K blocks
                     const int num_kb = g1 ? (tl.ks + 1) * all_kb / p.s1 - kbase : all_kb;
-                    // pair: a CTA with no rows of the block loads no token box (the MMA's rows
-                    // from it are never stored)
-                    const int n_box = (C::PAIR && tl.nrows <= 0)
-                                          ? 0
-                                          : (max(16, (tl.nrows + 15) & ~15) + C::BOX_ROWS - 1) / C::BOX_ROWS;
+                    // token boxes for `rows` rows (pair: a CTA with no rows of the block loads
+                    // none; the MMA's rows from it are never stored)
+                    auto boxes = [&](int rows) {
+                        return (C::PAIR && rows <= 0) ? 0 : (max(16, (rows + 15) & ~15) + C::BOX_ROWS - 1) / C::BOX_ROWS;
+                    };
+                    const int n_box = boxes(tl.nrows);
                     // pair: one 128-row weight block per CTA (rank 1 takes A1; without A1 it
                     // loads A0 again, and those accumulator columns are not stored)
                     const int wrow = (C::PAIR && rank == 1 && tl.dual) ? tl.a1row : tl.a0row;
-                    const uint32_t tx = (C::PAIR ? 1 : (tl.dual ? 2 : 1)) * (C::INT4 ? C::RAW_BYTES : C::A_BYTES) +
-                                        n_box * C::BOX_BYTES;
+                    // bytes that complete a stage: this CTA's copies, or for a pair both CTAs'
+                    // (rank 0 arms the barrier for the pair)
+                    const uint32_t tx = C::PAIR ? 2 * C::A_BYTES + (boxes(min(128, blk_rows)) +
+                                                                    boxes(min(128, blk_rows - 128))) * C::BOX_BYTES
+                                                : (tl.dual ? 2 : 1) * (C::INT4 ? C::RAW_BYTES : C::A_BYTES) +
+                                                      n_box * C::BOX_BYTES;
                     auto load_act = [&](uint8_t* st, uint32_t s_idx, int kx) {
                         for (int r = 0; r < n_box; ++r)
                             load(st + C::B_OFF + r * C::BOX_BYTES, ta, s_idx, kx, tl.row0 + r * C::BOX_ROWS);
@@ -683,8 +690,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                             break;
                         }
                         uint8_t* st = smem + (size_t)stage * C::STAGE_BYTES;
-                        if constexpr (C::PAIR) mbar_arrive_expect_tx_cluster(lead(&full[stage]), tx);
-                        else mbar_arrive_expect_tx(land(stage), tx);
+                        if constexpr (C::PAIR) {
+                            if (rank == 0) mbar_arrive_expect_tx(&full[stage], tx);
+                        } else {
+                            mbar_arrive_expect_tx(land(stage), tx);
+                        }
                         const int kx = (kbase + kb) * C::BK;
                         if constexpr (C::INT4) {  // packed weight bytes: x is a byte offset (2 K per byte)
                             load(st + C::RAW_OFF, tw, stage, kx / 2, tl.a0row);
@@ -1124,7 +1134,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) {
-                            if constexpr (C::PAIR) mbar_arrive_cluster(lead(&tempty[buf]));
+                            if constexpr (C::PAIR) mbar_arrive_remote(lead(&tempty[buf]));  // per K block: no store wait
                             else mbar_arrive(&tempty[buf]);
                         }
                     };
@@ -1638,15 +1648,19 @@ static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
     }
 }
 
+static std::atomic<int> g_fp8_pair{0};  // MOE_OPT_FP8_CTA_PAIR
+
+int gemm_set_fp8_pair(int enable) { return g_fp8_pair.exchange(enable ? 1 : 0); }
+
 int gemm_pick_bn(int64_t A, int G, int wdtype) {
     const double avg = G > 0 ? (double)A / (double)G : 0.0;
     int bn = 16;
     while (bn < 256 && bn < avg) bn <<= 1;  // smallest tile holding an average group
-    // FP8 at 256 is the CTA pair (2 x 128 token rows); it needs two GEMM1 completion
-    // counters per 256-row block within the workspace's block flags (true whenever
-    // groups average more than 128 rows)
+    // FP8 above 128 rows: the 128-token tile, or (when chosen) the CTA pair at "256" (2 x
+    // 128 token rows), which needs two GEMM1 completion counters per 256-row block within
+    // the workspace's block flags (true whenever groups average more than 128 rows)
     if (wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128 && bn > 128 &&
-        2 * gemm_max_blocks(A, G, 256) + 1 > gemm_max_blocks(A, G, 16) + 1)
+        (!g_fp8_pair.load() || 2 * gemm_max_blocks(A, G, 256) + 1 > gemm_max_blocks(A, G, 16) + 1))
         bn = 128;
     if ((wdtype == MOE_WDTYPE_INT4_G32 || wdtype == MOE_WDTYPE_NVFP4) && bn > 64)
         bn = 64;  // 4-bit weights: A tiles share TMEM with the accumulators

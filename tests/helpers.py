@@ -78,3 +78,21 @@ def sample_tokens(T: int, n: int, seed: int = 0) -> np.ndarray:
     rng = np.random.default_rng(seed)
     pick = set([0, T - 1, T // 2]) | set(rng.choice(T, n - 3, replace=False).tolist())
     return np.array(sorted(pick)[:n], dtype=np.int32)
+
+
+class fp8_layout:
+    """Within the block, FP8 layers with groups above 128 rows run in the given layout:
+    pair=True selects the two-CTA tile (moe_set_option(MOE_OPT_FP8_CTA_PAIR, 1))."""
+
+    def __init__(self, pair: bool):
+        self.pair = pair
+
+    def __enter__(self):
+        import grouped_gemm_swiglu_b200 as moe
+        self.old = moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, 1 if self.pair else 0)
+        return self
+
+    def __exit__(self, *exc):
+        import grouped_gemm_swiglu_b200 as moe
+        moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, self.old)
+        return False

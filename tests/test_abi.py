@@ -26,7 +26,7 @@ def test_every_header_function_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert moe.moe_abi_version() == 5
+    assert moe.moe_abi_version() == 6
     for code in range(-7, 1):
         assert moe.status_string(code)
     assert "unknown" in moe.status_string(-99)
@@ -174,3 +174,17 @@ def test_noalloc_size_limit_is_where_the_header_says(L):
         assert _noalloc(L)(fake, fake, ctypes.byref(d), fake, fake, fake, fake, fake, None, None) == -4
     d = _dims(T=28689, H=512, E=288, k=8, n_shared=1, n_sink=0, wdtype=4)
     assert _noalloc(L)(fake, fake, ctypes.byref(d), fake, fake, fake, fake, fake, None, None) == -1
+
+
+def test_set_option_returns_the_previous_value_and_rejects_unknown_ones(L):
+    """moe_set_option is host-only: it never touches a GPU."""
+    old = moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, 1)
+    try:
+        assert old in (0, 1)
+        assert moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, 0) == 1
+        assert moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, 0) == 0
+        assert L.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, 2) == -1
+        assert L.moe_set_option(99, 0) == -1
+        assert moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, 0) == 0  # the refusals changed nothing
+    finally:
+        moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, old)

@@ -12,7 +12,7 @@ import torch
 
 import grouped_gemm_swiglu_b200 as moe
 from grouped_gemm_swiglu_b200 import workloads as W
-from helpers import assert_bf16_close, assert_fp8_close, oracle_layer
+from helpers import assert_bf16_close, assert_fp8_close, fp8_layout, oracle_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -65,6 +65,11 @@ def guarded_ws(d, kind):
 
 @pytest.mark.parametrize("wl", SHAPES, ids=[w.name for w in SHAPES])
 def test_outputs_stay_in_bounds_and_match_the_oracle(wl):
+    with fp8_layout(pair=wl.name.endswith("_pair")):  # the *_pair shape in the CTA-pair layout
+        _check_bounds(wl)
+
+
+def _check_bounds(wl):
     inp = W.make_inputs(wl, "cuda")
     d = moe.MoeDims.of(wl)
     T, k, S, A, G, H, I = wl.T, wl.k, wl.n_sink, d.A, d.G, wl.H, wl.I

@@ -8,7 +8,7 @@ import torch
 import oracle
 import grouped_gemm_swiglu_b200 as moe
 from grouped_gemm_swiglu_b200 import workloads as W
-from helpers import assert_bf16_close, assert_fp8_close, f32, oracle_layer, sample_tokens
+from helpers import assert_bf16_close, assert_fp8_close, f32, fp8_layout, oracle_layer, sample_tokens
 
 pytestmark = pytest.mark.gpu
 
@@ -47,20 +47,34 @@ def test_forward_matches_oracle(name):
         assert_bf16_close(got, ref, name)
 
 
-# FP8 at a size the oracle covers token by token, in the CTA-pair layout the GLM-shaped
-# prefill uses (groups of about 540 rows: two to three 256-row blocks each, ragged tails),
-# with the GLM parameters (sigmoid routing, L = 10, one shared expert)
-PAIR_FULL = W.Workload("glm_fp8_t1024", T=1024, H=1024, I=512, E=16, k=8, n_shared=1, wdtype=W.WDTYPE_FP8,
+# FP8 at a size the oracle covers token by token, with groups of about 540 rows (several
+# token blocks each, ragged tails) and the GLM parameters (sigmoid routing, L = 10, one
+# shared expert), in both layouts of large-group FP8 tiles
+LARGE_FP8 = W.Workload("glm_fp8_t1024", T=1024, H=1024, I=512, E=16, k=8, n_shared=1, wdtype=W.WDTYPE_FP8,
                        score=W.SCORE_SIGMOID, limit=10.0)
 
 
-def test_forward_fp8_pair_every_token():
-    wl = PAIR_FULL
+@pytest.mark.parametrize("pair", [False, True], ids=["cta128", "cta_pair"])
+def test_forward_fp8_large_groups_every_token(pair):
+    wl = LARGE_FP8
     inp = W.make_inputs(wl, "cuda")
-    out, ids, tw, sw, layer = run_forward(wl, inp)
+    with fp8_layout(pair):
+        out, ids, tw, sw, layer = run_forward(wl, inp)
     assert layer.status() == 0
     ref = oracle_layer(wl, inp).moe_rows(np.arange(wl.T, dtype=np.int32))
     assert_fp8_close(out.float().cpu().numpy(), ref, wl.name)
+
+
+def test_forward_glm_fp8_cta_pair_sampled():
+    """The full GLM-shaped FP8 prefill in the CTA-pair layout (sampled tokens)."""
+    wl = W.WORKLOADS["glm_fp8"]
+    inp = W.make_inputs(wl, "cuda")
+    with fp8_layout(True):
+        out, ids, tw, sw, layer = run_forward(wl, inp)
+    assert layer.status() == 0
+    toks = sample_tokens(wl.T, 24, seed=2)
+    ref = oracle_layer(wl, inp).moe_rows(toks)
+    assert_fp8_close(out.float().cpu().numpy()[toks], ref, "glm_fp8 (CTA pair)")
 
 
 def test_forward_is_deterministic_and_reusable():

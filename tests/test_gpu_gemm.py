@@ -11,7 +11,7 @@ import torch
 import oracle
 import grouped_gemm_swiglu_b200 as moe
 from grouped_gemm_swiglu_b200 import workloads as W
-from helpers import assert_bf16_close, assert_fp8_close, bits16, e4m3_to_np, f32, u8
+from helpers import assert_bf16_close, assert_fp8_close, bits16, e4m3_to_np, f32, fp8_layout, u8
 
 pytestmark = pytest.mark.gpu
 
@@ -102,9 +102,10 @@ GEMM1_CASES = [
     (1024, 8, 2, 1, 512, 384, True, {"skew": 2.0, "scales": True, "limits": True}),  # FP8 tile 128, ragged, shared
     (40, 32, 4, 1, 512, 256, True, {"glm": True}),              # FP8, tile 16, shared group, L = 10
     (200, 8, 2, 0, 1024, 512, True, {"oai": True, "scales": True}),
-    # FP8 CTA pair (groups above 128 rows on average: 256-row token blocks, 128 per CTA);
-    # heavy skew leaves some groups under 128 rows (the odd CTA holds none of them) and
-    # some over 256 (several blocks); a shared group of T rows
+    # FP8 with groups above 128 rows on average (both layouts: 128-token tiles, and the
+    # CTA pair's 256-row token blocks, 128 per CTA); heavy skew leaves some groups under
+    # 128 rows (the pair's odd CTA holds none of them) and some over 256 (several
+    # blocks); a shared group of T rows
     (1500, 16, 2, 1, 512, 256, True, {"skew": 4.0, "oai": True}),
     (700, 4, 2, 0, 1024, 384, True, {"scales": True, "limits": True}),
     (128, 8, 2, 1, 512, 384, False, {"limits": True}),          # a clamp per expert (shared group too)
@@ -125,6 +126,20 @@ GEMM1_CASES = [
     (2, 64, 4, 1, 512, 256, False, {"int4": True}),            # INT4, 10 rows
     (3, 4, 2, 1, 512, 384, False, {"int4": True, "scales": True}),  # INT4, groups of several rows
 ]
+
+
+def _pairable(T, E, k, S, fp8):
+    """FP8 cases whose groups average more than 128 rows (the layouts differ there)."""
+    return fp8 is True and T * (k + S) / (E + S) > 128
+
+
+GEMM1_PAIR = [c for c in GEMM1_CASES if _pairable(*c[:4], c[6])]
+
+
+@pytest.mark.parametrize("T,E,k,S,H,I,fp8,extra", GEMM1_PAIR)
+def test_gemm1_swiglu_fp8_cta_pair(T, E, k, S, H, I, fp8, extra):
+    with fp8_layout(pair=True):
+        test_gemm1_swiglu(T, E, k, S, H, I, fp8, extra)
 
 
 @pytest.mark.parametrize("T,E,k,S,H,I,fp8,extra", GEMM1_CASES)
@@ -170,8 +185,8 @@ GEMM2_CASES = [
     (600, 4, 2, 1, 384, 256, False, True),      # tile 256, odd number of 128-row chunks of H
     (512, 8, 2, 0, 512, 256, True, False),      # FP8, tile 128
     (256, 8, 2, 0, 512, 256, True, False),      # FP8, tile 64
-    (600, 4, 2, 1, 384, 256, True, True),       # FP8 CTA pair, odd chunk count of H, sink-gated shared
-    (1500, 16, 2, 1, 384, 256, True, False),    # FP8 CTA pair, skewless, odd chunk count of H
+    (600, 4, 2, 1, 384, 256, True, True),       # FP8 large groups, odd chunk count of H, sink-gated shared
+    (1500, 16, 2, 1, 384, 256, True, False),    # FP8 large groups, odd chunk count of H
     (300, 8, 2, 1, 512, 256, True, False),      # FP8, tile 128 (single CTA), shared group
     (40, 32, 4, 1, 512, 256, True, False),
     (8, 64, 4, 0, 256, 256, "int4", False),     # INT4 weights, tile 16
@@ -187,6 +202,15 @@ GEMM2_CASES = [
     (4096, 128, 2, 0, 384, 256, False, False),
     (4096, 128, 2, 0, 384, 256, True, False),   # FP8, tile 64
 ]
+
+
+GEMM2_PAIR = [c for c in GEMM2_CASES if _pairable(*c[:4], c[6])]
+
+
+@pytest.mark.parametrize("T,E,k,S,H,I,fp8,sinks", GEMM2_PAIR)
+def test_gemm2_combine_fp8_cta_pair(T, E, k, S, H, I, fp8, sinks):
+    with fp8_layout(pair=True):
+        test_gemm2_combine(T, E, k, S, H, I, fp8, sinks)
 
 
 @pytest.mark.parametrize("T,E,k,S,H,I,fp8,sinks", GEMM2_CASES)

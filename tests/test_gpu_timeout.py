@@ -17,7 +17,7 @@ import torch
 
 import grouped_gemm_swiglu_b200 as moe
 from grouped_gemm_swiglu_b200 import workloads as W
-from helpers import assert_bf16_close, assert_fp8_close, oracle_layer
+from helpers import assert_bf16_close, assert_fp8_close, fp8_layout, oracle_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -26,7 +26,8 @@ MOE_ERR_TIMEOUT = -6
 
 CASES = [
     W.WORKLOADS["tiny"],
-    # about 180 rows per group: FP8 in the CTA-pair layout (256-row token blocks)
+    # about 180 rows per group: FP8 in the CTA-pair layout (256-row token blocks; the
+    # test selects it with moe_set_option)
     W.Workload("fp8_pair", T=300, H=512, I=256, E=4, k=2, n_shared=1, wdtype=W.WDTYPE_FP8,
                score=W.SCORE_SIGMOID, limit=10.0),
 ]
@@ -34,6 +35,11 @@ CASES = [
 
 @pytest.mark.parametrize("wl", CASES, ids=[w.name for w in CASES])
 def test_a_wait_that_never_completes_reports_timeout_and_the_context_survives(wl):
+    with fp8_layout(pair=wl.name.endswith("_pair")):  # the FP8 case in the CTA-pair layout
+        _check_timeout(wl)
+
+
+def _check_timeout(wl):
     inp = W.make_inputs(wl, "cuda")
     d = moe.MoeDims.of(wl)
     fp8 = wl.wdtype == W.WDTYPE_FP8
