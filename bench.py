@@ -46,6 +46,10 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the oracle sample")
     ap.add_argument("--tokens", type=int, default=None, help="override the workload's T (profiling runs)")
     ap.add_argument("--experts", type=int, default=None, help="override the workload's E (profiling runs)")
+    ap.add_argument("--mode", choices=["dp", "ep", "tp"], default="dp",
+                    help="dp: every rank runs the whole layer on its own tokens (default); ep: the routed "
+                         "experts split over the ranks, rows exchanged with all_to_all; tp: every expert's "
+                         "intermediate size split over the ranks, outputs all-reduced")
     ap.add_argument("--router-sweep", action="store_true",
                     help="time the router alone at fp32 [T, 258] (256 routed + 2 sinks), k = 6, "
                          "T in 1, 8, 64, 512, 4096, 8192, and print one JSON line")
@@ -566,6 +570,95 @@ def run_ours(args):
     return 0
 
 
+# ------------------------------------------------------------------ expert / tensor parallel
+def parallel_bench(mode, wl, ranks, dev, K, Wm, ops=None, inputs=None, exchange=None):
+    """Times the expert-parallel (mode "ep") or tensor-parallel ("tp") layer, one rank per
+    GPU, and returns the JSON line (rank 0 prints it). ep: every rank routes its own T
+    tokens (the workload's tokens rolled by 17 * rank rows, so ranks route differently)
+    and the routed experts are split in contiguous blocks; value = all ranks' tokens / the
+    slowest rank's step (weak scaling). tp: every rank runs all T tokens on an I/R slice
+    of every expert and the outputs are all-reduced; value = T / the slowest rank's step
+    (strong scaling). A step is one eager forward (the expert-parallel pass reads its row
+    counts on the host, so it is not graph-captured), between CUDA events on its stream
+    and barriers. `ops`, `inputs` and `exchange` let the plumbing run with stand-ins."""
+    import torch
+    from grouped_gemm_swiglu_b200 import ep as EP
+    from grouped_gemm_swiglu_b200 import tp as TP
+    from grouped_gemm_swiglu_b200 import workloads as W
+    from grouped_gemm_swiglu_b200._lib import MoeDims
+    import grouped_gemm_swiglu_b200 as moe
+    ops = ops if ops is not None else moe._lib
+    world, rank = ranks.world, ranks.rank
+    inp = inputs if inputs is not None else W.make_inputs(wl, dev)
+    d = inp["dims"] if "dims" in inp else MoeDims.of(wl)
+    if exchange is None:
+        exchange = EP.TorchExchange() if world > 1 else EP.LocalExchange(1).for_rank(0)
+    T = wl.T
+    if mode == "ep":
+        if d.E % world:
+            raise SystemExit(f"--mode ep: E = {d.E} does not split over {world} ranks")
+        sh = lambda t: EP.shard(t, rank, world, d.E, d.n_shared)  # noqa: E731
+        layer = EP.ExpertParallelMoE(d, rank, world, sh(inp["w1"]), sh(inp["w2"]), sh(inp.get("w1_scale")),
+                                     sh(inp.get("w2_scale")), sh(inp.get("gate_scale")), sh(inp.get("up_scale")),
+                                     exchange=exchange, ops=ops, max_tokens=T)
+        x = torch.roll(inp["x"], 17 * rank, 0).contiguous()
+        logits = torch.roll(inp["logits"], 17 * rank, 0).contiguous()
+    else:
+        if d.I % (128 * world):
+            raise SystemExit(f"--mode tp: I = {d.I} does not split into multiples of 128 over {world} ranks")
+        layer = TP.TensorParallelMoE(d, rank, world, TP.shard_w1(inp["w1"], rank, world),
+                                     TP.shard_w2(inp["w2"], rank, world), TP.shard_w1(inp.get("w1_scale"), rank, world),
+                                     TP.shard_w2(inp.get("w2_scale"), rank, world), inp.get("gate_scale"),
+                                     inp.get("up_scale"), exchange=exchange, ops=ops)
+        x, logits = inp["x"], inp["logits"]
+    out = torch.empty((T, d.H), dtype=torch.bfloat16, device=dev)
+    cuda = torch.device(dev).type == "cuda"
+    for _ in range(Wm):
+        layer.forward(logits, x, out=out)
+    if cuda:
+        torch.cuda.synchronize(dev)
+    times = []
+    for _ in range(K):
+        ranks.barrier()
+        if cuda:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            layer.forward(logits, x, out=out)
+            b.record()
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        else:
+            t0 = time.perf_counter()
+            layer.forward(logits, x, out=out)
+            times.append((time.perf_counter() - t0) * 1e3)
+    ranks.barrier()
+    st = layer.status()
+    ms = ranks.max_over_ranks(sum(times) / len(times))
+    tokens = world * T if mode == "ep" else T
+    return {"metric": METRIC, "value": tokens / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": Wm, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak" if mode == "ep" else "strong", "vs_baseline": None,
+            "dtype": {1: "fp8_e4m3", 2: "int4_w4a16", 3: "nvfp4_w4a16"}.get(wl.wdtype, "bf16"),
+            "data": "synthetic", "config": dict(config_of(wl), mode=mode, parallelism=f"{mode}{world}"),
+            "status": st, "roofline": None, "cpu_baseline": None,
+            "timing": "eager forward between CUDA events on its stream, barrier before each step, mean over "
+                      "the steps, max over ranks",
+            "ms_stats": stats(times)}
+
+
+def run_parallel(args):
+    import torch
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks("nccl", dev)
+    line = parallel_bench(args.mode, workload_of(args), ranks, dev, args.steps, args.warmup)
+    if ranks.rank == 0:
+        print(json.dumps(line), flush=True)
+    ranks.close()
+    return 0
+
+
 # ------------------------------------------------------------------ router sweep
 ROUTER_SWEEP_T = (1, 8, 64, 512, 4096, 8192)
 
@@ -631,6 +724,8 @@ def main():
         return run_router_sweep(args)
     if args.impl == "reference":
         return run_reference(args)
+    if args.mode != "dp":
+        return run_parallel(args)
     return run_ours(args)
 
 

@@ -22,12 +22,14 @@ own tokens. One layer pass on every rank:
 
 The exchange is a caller-supplied object (`TorchExchange` wraps torch.distributed's
 all_to_all_single; NCCL between GPUs); the compute steps are this library's kernels.
-The per-rank row counts are read on the host to size the exchange.
+Every buffer and workspace is allocated once, for a token capacity (`max_tokens`, grown
+if a call brings more), and reused by every pass. The per-rank row counts are computed
+on the device from the offsets, exchanged on the device, and read on the host once per
+pass (send and receive counts together) to size the exchange.
 """
 from __future__ import annotations
 
 import threading
-from dataclasses import dataclass
 
 import torch
 
@@ -50,8 +52,15 @@ class TorchExchange:
         self.dist.all_to_all_single(out, inp, out_splits, in_splits, group=self.group)
 
     def all_reduce(self, t: torch.Tensor) -> None:
-        """In-place sum over the ranks."""
-        self.dist.all_reduce(t, op=self.dist.ReduceOp.SUM, group=self.group)
+        """In-place sum over the ranks, accumulated in fp32 (a bf16 tensor is widened, summed
+        and rounded once, as LocalExchange does; NCCL gives every rank the same bits, and
+        the fp32 sum equals the rank-order sum up to fp32 reassociation)."""
+        if t.dtype == torch.float32:
+            self.dist.all_reduce(t, op=self.dist.ReduceOp.SUM, group=self.group)
+            return
+        acc = t.float()
+        self.dist.all_reduce(acc, op=self.dist.ReduceOp.SUM, group=self.group)
+        t.copy_(acc)
 
 
 class LocalExchange:
@@ -116,29 +125,80 @@ def shard(t: torch.Tensor | None, rank: int, world: int, E: int, n_shared: int):
     return torch.cat([t[rank * n_local:(rank + 1) * n_local], t[E:E + n_shared]]).contiguous()
 
 
-@dataclass
-class _Sent:
-    """What a rank keeps from its dispatch to finish the layer for its own tokens."""
-    T: int
-    dims: MoeDims
-    tw: torch.Tensor
-    sw: torch.Tensor | None
-    offsets: torch.Tensor
-    inv: torch.Tensor
-    x_perm: torch.Tensor
-    row_ids: torch.Tensor
-    a_routed: int
-    send_splits: list[int]
+class _Buffers:
+    """The source side of a pass (this rank's tokens), sized for a token capacity."""
+
+    def __init__(self, layer: "ExpertParallelMoE", T_cap: int, dev):
+        ops, d, R = layer.ops, layer.dims, layer.world
+        self.T_cap = T_cap
+        k, S, E, H, I = d.k, d.n_shared, d.E, d.H, d.I
+        A = T_cap * (k + S)
+        fp8 = d.wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128
+        cap = MoeDims.from_buffer_copy(d)
+        cap.T = T_cap
+        sd = MoeDims.from_buffer_copy(cap)  # the rows travel in bf16
+        sd.wdtype = MOE_WDTYPE_BF16
+        # source side: routing and the permutation of this rank's tokens
+        self.ids = torch.empty((T_cap, k), dtype=torch.int32, device=dev)
+        self.tw = torch.empty((T_cap, k), dtype=torch.float32, device=dev)
+        self.sw = torch.empty((T_cap, d.n_sink), dtype=torch.float32, device=dev) if d.n_sink else None
+        self.offsets = torch.empty((d.G + 1,), dtype=torch.int32, device=dev)
+        self.perm = torch.empty((A,), dtype=torch.int32, device=dev)
+        self.inv = torch.empty((T_cap, k), dtype=torch.int32, device=dev)
+        self.x_perm = torch.empty((A, H), dtype=torch.bfloat16, device=dev)
+        self.row_ids = torch.empty((A,), dtype=torch.int32, device=dev)
+        self.ws_p = ops.alloc_workspace(sd, MOE_WS_PERMUTE, device=dev)
+        self.ws_c = ops.alloc_workspace(cap, MOE_WS_COMBINE, device=dev)
+        self.y_home = torch.empty((A, H), dtype=torch.bfloat16, device=dev)
+        # counts: [send R | recv R | routed rows 1], device and host
+        self.counts = torch.empty((2 * R + 1,), dtype=torch.int64, device=dev)
+        self.bounds = torch.arange(0, E + 1, layer.n_local, dtype=torch.long, device=dev)  # group bounds per rank
+        self.status_words = [self.ws_p, self.ws_c]
+
+
+class _OwnerBuffers:
+    """The owner side of a pass: the rows this rank's experts serve (every rank's routed
+    rows for them, and its own tokens' shared-expert rows), sized for n_cap rows."""
+
+    def __init__(self, layer: "ExpertParallelMoE", n_cap: int, dev):
+        ops, d = layer.ops, layer.dims
+        S, H, I = d.n_shared, d.H, d.I
+        fp8 = d.wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128
+        self.n_cap = n_cap
+        G = layer.n_local + S
+        ld = MoeDims.from_buffer_copy(d)
+        ld.T, ld.k, ld.E, ld.n_sink, ld.n_shared = n_cap, 1, G, 0, 0
+        ld.score, ld.route_scale = MOE_SCORE_SOFTMAX, 1.0
+        self.rows = torch.empty((n_cap, H), dtype=torch.bfloat16, device=dev)
+        self.recv_ids = torch.empty((n_cap,), dtype=torch.int32, device=dev)
+        self.local_ids = torch.empty((n_cap, 1), dtype=torch.int32, device=dev)
+        self.l_offsets = torch.empty((G + 1,), dtype=torch.int32, device=dev)
+        self.l_perm = torch.empty((n_cap,), dtype=torch.int32, device=dev)
+        self.l_inv = torch.empty((n_cap, 1), dtype=torch.int32, device=dev)
+        self.x_loc = torch.empty((n_cap, H), dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev)
+        self.xs = torch.empty((H // 128, n_cap), dtype=torch.float32, device=dev) if fp8 else None
+        self.h = torch.empty((n_cap, I), dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev)
+        self.hs = torch.empty((I // 128, n_cap), dtype=torch.float32, device=dev) if fp8 else None
+        self.y = torch.empty((n_cap, H), dtype=torch.bfloat16, device=dev)
+        self.y_back = torch.empty((n_cap, H), dtype=torch.bfloat16, device=dev)
+        self.ones = torch.ones((n_cap, 1), dtype=torch.float32, device=dev)
+        self.ws_lp = ops.alloc_workspace(ld, MOE_WS_PERMUTE, device=dev)
+        self.ws_le = ops.alloc_workspace(ld, MOE_WS_EXPERTS, device=dev)
+        self.ws_lc = ops.alloc_workspace(ld, MOE_WS_COMBINE, device=dev)
+        self.status_words = [self.ws_lp, self.ws_le, self.ws_lc]
 
 
 class ExpertParallelMoE:
     """One rank of the expert-parallel layer. Weights are this rank's groups only:
     w1 [E/R + n_shared, 2I, H], w2 [E/R + n_shared, H, I] and the matching scales,
     gate/up scales and clamps (see `shard`). `dims` describes the whole layer (global E);
-    dims.T is ignored (each call takes its own token count)."""
+    dims.T is ignored (each call takes its own token count). Buffers are allocated for
+    `max_tokens` tokens per rank on the first call (more if a call brings more) and
+    reused; the receive side holds every other rank's routed rows in the worst case."""
 
     def __init__(self, dims: MoeDims, rank: int, world: int, w1, w2, w1_scale=None, w2_scale=None,
-                 gate_scale=None, up_scale=None, limits=None, router_bias=None, exchange=None, ops=None):
+                 gate_scale=None, up_scale=None, limits=None, router_bias=None, exchange=None, ops=None,
+                 max_tokens: int = 0):
         if world < 1 or not 0 <= rank < world or dims.E % world:
             raise ValueError(f"E = {dims.E} routed experts do not split evenly over {world} ranks")
         self.dims = MoeDims.from_buffer_copy(dims)
@@ -149,105 +209,91 @@ class ExpertParallelMoE:
         self.gate_scale, self.up_scale, self.limits, self.router_bias = gate_scale, up_scale, limits, router_bias
         self.exchange = exchange if exchange is not None else TorchExchange()
         self.ops = ops if ops is not None else _default_ops
+        self.max_tokens = max_tokens
+        self.buf: _Buffers | None = None
+        self.own: _OwnerBuffers | None = None
         self.status_words: list[torch.Tensor] = []
 
-    # ---------------------------------------------------------------- phase 1 (local)
-    def _dispatch(self, logits: torch.Tensor, x: torch.Tensor) -> _Sent:
-        ops, dev = self.ops, x.device
-        T = x.shape[0]
-        d = MoeDims.from_buffer_copy(self.dims)
-        d.T = T
-        ids = torch.empty((T, d.k), dtype=torch.int32, device=dev)
-        tw = torch.empty((T, d.k), dtype=torch.float32, device=dev)
-        sw = torch.empty((T, d.n_sink), dtype=torch.float32, device=dev) if d.n_sink else None
-        ops.moe_route_topk(logits, d, self.router_bias, ids, tw, sw)
-        # the rows travel in bf16; an FP8 layer quantises them on the owning rank
-        sd = MoeDims.from_buffer_copy(d)
-        sd.wdtype = MOE_WDTYPE_BF16
-        A, G = d.A, d.G
-        offsets = torch.empty((G + 1,), dtype=torch.int32, device=dev)
-        perm = torch.empty((A,), dtype=torch.int32, device=dev)
-        inv = torch.empty((T, d.k), dtype=torch.int32, device=dev)
-        x_perm = torch.empty((A, d.H), dtype=torch.bfloat16, device=dev)
-        ws_p = ops.alloc_workspace(sd, MOE_WS_PERMUTE, device=dev)
-        ops.moe_permute(ids, x, sd, offsets, perm, inv, x_perm, None, ws_p)
-        row_ids = torch.empty((A,), dtype=torch.int32, device=dev)
-        ops.moe_ep_row_ids(offsets, sd, row_ids)
-        self.status_words.append(ws_p)
-        offs = offsets.cpu().tolist()  # host copy of the group bounds sizes the exchange
-        nl = self.n_local
-        send = [offs[(r + 1) * nl] - offs[r * nl] for r in range(self.world)]
-        return _Sent(T, d, tw, sw, offsets, inv, x_perm, row_ids, offs[d.E], send)
+    def _buffers(self, T: int, dev) -> _Buffers:
+        if self.buf is None or T > self.buf.T_cap:
+            self.buf = _Buffers(self, max(T, self.max_tokens, 1), dev)
+        return self.buf
 
-    # ---------------------------------------------------------------- phase 3 (local)
-    def _local_experts(self, rows: torch.Tensor, row_ids: torch.Tensor) -> torch.Tensor:
-        """The one-rank path over this rank's groups, for rows in arrival order; returns
-        their expert outputs (bf16, unweighted) in the same order."""
-        ops, dev, d = self.ops, rows.device, self.dims
-        n = rows.shape[0]
-        G = self.n_local + d.n_shared
-        ld = MoeDims.from_buffer_copy(d)
-        ld.T, ld.k, ld.E, ld.n_sink, ld.n_shared = n, 1, G, 0, 0
-        ld.score, ld.route_scale = MOE_SCORE_SOFTMAX, 1.0
-        y_back = torch.empty((n, d.H), dtype=torch.bfloat16, device=dev)
-        if n == 0:
-            return y_back
-        fp8 = d.wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128
-        local_ids = torch.empty((n, 1), dtype=torch.int32, device=dev)
-        ops.moe_ep_rebase(row_ids, n, d.E, d.n_shared, self.local_offset, self.n_local, local_ids)
-        offsets = torch.empty((G + 1,), dtype=torch.int32, device=dev)
-        perm = torch.empty((n,), dtype=torch.int32, device=dev)
-        inv = torch.empty((n, 1), dtype=torch.int32, device=dev)
-        x_loc = torch.empty((n, d.H), dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev)
-        xs = torch.empty((d.H // 128, n), dtype=torch.float32, device=dev) if fp8 else None
-        h = torch.empty((n, d.I), dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev)
-        hs = torch.empty((d.I // 128, n), dtype=torch.float32, device=dev) if fp8 else None
-        y = torch.empty((n, d.H), dtype=torch.bfloat16, device=dev)
-        ws_p = ops.alloc_workspace(ld, MOE_WS_PERMUTE, device=dev)
-        ws_e = ops.alloc_workspace(ld, MOE_WS_EXPERTS, device=dev)
-        ws_c = ops.alloc_workspace(ld, MOE_WS_COMBINE, device=dev)
-        ops.moe_permute(local_ids, rows, ld, offsets, perm, inv, x_loc, xs, ws_p)
-        ops.moe_experts(x_loc, xs, offsets, self.w1, self.w1_scale, self.gate_scale, self.up_scale, self.limits,
-                        self.w2, self.w2_scale, ld, h, hs, y, ws_e)
-        ones = torch.ones((n, 1), dtype=torch.float32, device=dev)
-        ops.moe_combine(y, offsets, inv, ones, None, ld, y_back, ws_c)
-        self.status_words += [ws_p, ws_e, ws_c]
-        return y_back
+    def _owner(self, n: int, dev) -> _OwnerBuffers:
+        """Owner-side buffers for n rows: sized for every rank bringing max_tokens tokens of
+        routed rows, and grown (to the rows that arrived) when a pass brings more."""
+        d = self.dims
+        if self.own is None or n > self.own.n_cap:
+            T = max(self.max_tokens, 1)
+            self.own = _OwnerBuffers(self, max(n, self.world * T * d.k + T * d.n_shared), dev)
+        return self.own
 
     # ---------------------------------------------------------------- the whole pass
     def forward(self, logits: torch.Tensor, x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
         """logits [T, E + n_sink] fp32 and x [T, H] bf16 of this rank's tokens -> out [T, H]."""
-        ops, ex, d = self.ops, self.exchange, self.dims
+        ops, ex, R = self.ops, self.exchange, self.world
         dev = x.device
-        self.status_words = []
-        s = self._dispatch(logits, x)
-        R = self.world
-        # per-rank row counts
-        cnt_out = torch.empty((R,), dtype=torch.int64, device=dev)
-        ex.all_to_all(cnt_out, torch.tensor(s.send_splits, dtype=torch.int64, device=dev), [1] * R, [1] * R)
-        recv_splits = [int(v) for v in cnt_out.cpu().tolist()]
-        n_recv = sum(recv_splits)
-        n_sh = s.x_perm.shape[0] - s.a_routed  # this rank's own shared-expert rows
-        rows = torch.empty((n_recv + n_sh, d.H), dtype=torch.bfloat16, device=dev)
-        row_ids = torch.empty((n_recv + n_sh,), dtype=torch.int32, device=dev)
-        ex.all_to_all(rows[:n_recv], s.x_perm[:s.a_routed], recv_splits, s.send_splits)
-        ex.all_to_all(row_ids[:n_recv], s.row_ids[:s.a_routed], recv_splits, s.send_splits)
-        rows[n_recv:].copy_(s.x_perm[s.a_routed:])
-        row_ids[n_recv:].copy_(s.row_ids[s.a_routed:])
-        y_back = self._local_experts(rows, row_ids)
-        # the routed rows go home in the order they came; the shared rows never left
-        y = torch.empty((s.x_perm.shape[0], d.H), dtype=torch.bfloat16, device=dev)
-        ex.all_to_all(y[:s.a_routed], y_back[:n_recv], s.send_splits, recv_splits)
-        y[s.a_routed:].copy_(y_back[n_recv:])
+        T = x.shape[0]
+        b = self._buffers(T, dev)
+        d = MoeDims.from_buffer_copy(self.dims)
+        d.T = T
+        k, S, H = d.k, d.n_shared, d.H
+        A = d.A
+        # 1. route and permute this rank's tokens (bf16 rows), tag rows with global group ids
+        ids, tw, inv = b.ids[:T], b.tw[:T], b.inv[:T]
+        sw = b.sw[:T] if b.sw is not None else None
+        ops.moe_route_topk(logits, d, self.router_bias, ids, tw, sw)
+        sd = MoeDims.from_buffer_copy(d)
+        sd.wdtype = MOE_WDTYPE_BF16
+        x_perm, row_ids = b.x_perm[:A], b.row_ids[:A]
+        ops.moe_permute(ids, x, sd, b.offsets, b.perm[:A], inv, x_perm, None, b.ws_p)
+        ops.moe_ep_row_ids(b.offsets, sd, row_ids)
+        # 2. row counts per destination rank on the device, exchanged there, read once
+        off64 = b.offsets.to(torch.int64)
+        b.counts[:R].copy_(off64[b.bounds[1:]] - off64[b.bounds[:-1]])
+        b.counts[2 * R].copy_(off64[d.E])
+        ex.all_to_all(b.counts[R:2 * R], b.counts[:R], [1] * R, [1] * R)
+        host = b.counts.cpu().tolist()  # the pass's one host read of counts
+        send, recv, a_routed = host[:R], host[R:2 * R], host[2 * R]
+        n_recv = sum(recv)
+        n = n_recv + (A - a_routed)  # received rows + this rank's own shared-expert rows
+        o = self._owner(n, dev)
+        self.status_words = b.status_words + o.status_words
+        rows, recv_ids = o.rows[:n], o.recv_ids[:n]
+        ex.all_to_all(rows[:n_recv], x_perm[:a_routed], recv, send)
+        ex.all_to_all(recv_ids[:n_recv], row_ids[:a_routed], recv, send)
+        rows[n_recv:].copy_(x_perm[a_routed:])
+        recv_ids[n_recv:].copy_(row_ids[a_routed:])
+        # 3. this rank's experts over the rows in arrival order
+        y_back = o.y_back[:n]
+        if n:
+            G = self.n_local + S
+            ld = MoeDims.from_buffer_copy(self.dims)
+            ld.T, ld.k, ld.E, ld.n_sink, ld.n_shared = n, 1, G, 0, 0
+            ld.score, ld.route_scale = MOE_SCORE_SOFTMAX, 1.0
+            local_ids = o.local_ids[:n]
+            ops.moe_ep_rebase(recv_ids, n, d.E, S, self.local_offset, self.n_local, local_ids)
+            xs = hs = None
+            if o.xs is not None:  # block-major scales of n rows: contiguous [K/128][n] views
+                xs = o.xs.view(-1)[:(H // 128) * n].view(H // 128, n)
+                hs = o.hs.view(-1)[:(d.I // 128) * n].view(d.I // 128, n)
+            ops.moe_permute(local_ids, rows, ld, o.l_offsets, o.l_perm[:n], o.l_inv[:n], o.x_loc[:n], xs, o.ws_lp)
+            ops.moe_experts(o.x_loc[:n], xs, o.l_offsets, self.w1, self.w1_scale, self.gate_scale, self.up_scale,
+                            self.limits, self.w2, self.w2_scale, ld, o.h[:n], hs, o.y[:n], o.ws_le)
+            # back to arrival order: a unit-weight combine (an exact copy of each row)
+            ops.moe_combine(o.y[:n], o.l_offsets, o.l_inv[:n], o.ones[:n], None, ld, y_back, o.ws_lc)
+        # 4. the routed rows go home in the order they came; the shared rows never left
+        y = b.y_home[:A]
+        ex.all_to_all(y[:a_routed], y_back[:n_recv], send, recv)
+        y[a_routed:].copy_(y_back[n_recv:])
         if out is None:
-            out = torch.empty((s.T, d.H), dtype=torch.bfloat16, device=dev)
-        ws_c = ops.alloc_workspace(s.dims, MOE_WS_COMBINE, device=dev)
-        ops.moe_combine(y, s.offsets, s.inv, s.tw, s.sw, s.dims, out, ws_c)
-        self.status_words.append(ws_c)
+            out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        ops.moe_combine(y, b.offsets, inv, tw, sw, d, out, b.ws_c)
         return out
 
     def status(self) -> int:
-        """The first nonzero device status of the last forward's calls (0 = all fine)."""
+        """The first nonzero device status recorded by this layer's calls since its buffers
+        were allocated (0 = all fine)."""
         for ws in self.status_words:
             st = self.ops.moe_read_status(ws)
             if st:

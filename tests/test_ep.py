@@ -117,9 +117,9 @@ def _weights(E, S, seed=0):
     return torch.rand((E + S,), generator=g) + 0.5, torch.randn((E + S,), generator=g)
 
 
-def _one_rank(d, logits, x, w1, w2):
+def _one_rank(d, logits, x, w1, w2, ops=None):
     """The plain pipeline of the stand-ins with every expert on one rank."""
-    ops = CpuOps
+    ops = ops if ops is not None else CpuOps
     T = x.shape[0]
     dd = MoeDims.from_buffer_copy(d)
     dd.T = T
@@ -225,6 +225,52 @@ def test_thread_ranks_match_the_one_rank_pipeline_bit_for_bit(world):
         got, ref = outs[r]
         assert torch.equal(got, ref), f"rank {r}"
         assert layers[r].status() == 0
+
+
+def test_buffers_are_kept_and_reused_across_passes_of_varying_size():
+    """Several passes per rank with token counts that grow and shrink (including a pass
+    with more tokens than max_tokens, and one where the other rank sends more rows than
+    any earlier pass): every pass matches the one-rank pipeline, and a pass that fits the
+    buffers allocates none."""
+    world, E, k, n_sink, n_shared = 2, 8, 2, 2, 2
+    d = _dims(0, E, k, n_sink, n_shared)
+    w1, w2 = _weights(E, n_shared)
+    hub = ep.LocalExchange(world)
+    sizes = [[4, 6], [2, 1], [9, 3], [3, 12], [1, 1]]  # per pass: tokens of rank 0, rank 1
+    res, errs = {}, []
+
+    def run(r):
+        try:
+            layer = ep.ExpertParallelMoE(d, r, world, ep.shard(w1, r, world, E, n_shared),
+                                         ep.shard(w2, r, world, E, n_shared), exchange=hub.for_rank(r), ops=CpuOps,
+                                         max_tokens=8)
+            got = []
+            for i, Ts in enumerate(sizes):
+                logits, x = _inputs(r, Ts[r], E, n_sink, d.H, seed=i)
+                before = (layer.buf, layer.own)
+                out = layer.forward(logits, x)
+                got.append((torch.equal(out, _one_rank(d, logits, x, w1, w2)), before[0] is layer.buf,
+                            before[1] is layer.own, layer.buf.T_cap, layer.own.n_cap))
+            res[r] = (got, layer.status())
+        except Exception as e:  # noqa: BLE001 (reported below)
+            errs.append(e)
+            hub._barrier.abort()
+
+    ts = [threading.Thread(target=run, args=(r,)) for r in range(world)]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join(timeout=120)
+    assert not errs, errs
+    for r in range(world):
+        got, st = res[r]
+        assert st == 0
+        assert all(g[0] for g in got), [g[0] for g in got]
+        # the first pass allocates (capacity 8 tokens, every rank's routed rows: 2*8*2 + 8*2);
+        # the second reuses; a pass of 9 or 12 own tokens grows the source side
+        assert got[0][3] == 8 and got[0][4] == world * 8 * k + 8 * n_shared
+        assert got[1][1] and got[1][2]
+        assert got[4][1] and got[4][2]
 
 
 def test_uneven_expert_split_is_rejected():
