@@ -133,39 +133,11 @@ __global__ void __launch_bounds__(256) permute_count_kernel(const int32_t* __res
     if (threadIdx.x == 0) *counter = 0u;
 }
 
-// blockIdx.x = token: the destinations of its k routed slots and n_shared shared rows
-// are looked up once, perm / inv_perm written, then the CTA streams the row in 16-byte
-// vectors (kScatterThreads at a time): a copy (bf16) or a quantised copy (E4M3 + scales).
+// Token t's row of x to its nd destination rows s_dst[] (-1: none) of x_perm, by the
+// whole CTA in 16-byte vectors: a copy (bf16) or a quantised copy (E4M3 + scales).
 template <bool FP8>
-__global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
-    const int32_t* __restrict__ ids, const int32_t* __restrict__ rank, const int32_t* __restrict__ base,
-    const int32_t* __restrict__ offsets, const uint16_t* __restrict__ x, int T, int H, int k, int E, int n_shared,
-    int64_t A, int32_t* __restrict__ perm, int32_t* __restrict__ inv, void* __restrict__ x_perm,
-    float* __restrict__ x_scale, int* status) {
-    __shared__ int s_dst[32];
-    pdl_trigger();
-    pdl_wait();
-    const int t = blockIdx.x;
-    const int nd = k + n_shared;
-    if (threadIdx.x < nd) {
-        const int d = threadIdx.x;
-        int64_t dst = -1;
-        if (d < k) {
-            const int e = ids[(size_t)t * k + d];
-            const int r = rank[(size_t)t * k + d];
-            if (e >= 0 && e < E && r >= 0) dst = (int64_t)offsets[e] + base[(size_t)(t / kChunk) * E + e] + r;
-        } else {
-            dst = (int64_t)offsets[E + (d - k)] + t;
-        }
-        if (dst >= A) {
-            set_status(status, MOE_ERR_EXPERT_ID);
-            dst = -1;
-        }
-        s_dst[d] = (int)dst;
-        if (d < k) inv[(size_t)t * k + d] = (int)dst;
-        if (dst >= 0) perm[dst] = t;
-    }
-    __syncthreads();
+__device__ __forceinline__ void scatter_row(const uint16_t* __restrict__ x, int t, int H, int nd, const int* s_dst,
+                                            void* __restrict__ x_perm, float* __restrict__ x_scale, int64_t A) {
     const int nvec = H / 8;
     for (int v0 = 0; v0 < nvec; v0 += blockDim.x) {
         const int v = v0 + threadIdx.x;
@@ -213,6 +185,116 @@ __global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
     }
 }
 
+// blockIdx.x = token: the destinations of its k routed slots and n_shared shared rows
+// are looked up once, perm / inv_perm written, then the CTA streams the row in 16-byte
+// vectors (kScatterThreads at a time): a copy (bf16) or a quantised copy (E4M3 + scales).
+template <bool FP8>
+__global__ void __launch_bounds__(kScatterThreads) permute_scatter_kernel(
+    const int32_t* __restrict__ ids, const int32_t* __restrict__ rank, const int32_t* __restrict__ base,
+    const int32_t* __restrict__ offsets, const uint16_t* __restrict__ x, int T, int H, int k, int E, int n_shared,
+    int64_t A, int32_t* __restrict__ perm, int32_t* __restrict__ inv, void* __restrict__ x_perm,
+    float* __restrict__ x_scale, int* status) {
+    __shared__ int s_dst[32];
+    pdl_trigger();
+    pdl_wait();
+    const int t = blockIdx.x;
+    const int nd = k + n_shared;
+    if (threadIdx.x < nd) {
+        const int d = threadIdx.x;
+        int64_t dst = -1;
+        if (d < k) {
+            const int e = ids[(size_t)t * k + d];
+            const int r = rank[(size_t)t * k + d];
+            if (e >= 0 && e < E && r >= 0) dst = (int64_t)offsets[e] + base[(size_t)(t / kChunk) * E + e] + r;
+        } else {
+            dst = (int64_t)offsets[E + (d - k)] + t;
+        }
+        if (dst >= A) {
+            set_status(status, MOE_ERR_EXPERT_ID);
+            dst = -1;
+        }
+        s_dst[d] = (int)dst;
+        if (d < k) inv[(size_t)t * k + d] = (int)dst;
+        if (dst >= 0) perm[dst] = t;
+    }
+    __syncthreads();
+    scatter_row<FP8>(x, t, H, nd, s_dst, x_perm, x_scale, A);
+}
+
+// Batches of at most one counting chunk (T <= 256) in one launch: CTA t stages all T*k
+// ids in shared memory, counts the rows of every group and scans them (every CTA does the
+// same; CTA 0 writes offsets), ranks its own slots among earlier tokens' rows of the same
+// expert (the stable (expert, token, slot) order), and scatters its row. Ids outside
+// [0, E) or repeated within a token are flagged by the CTA of that token.
+template <bool FP8>
+__global__ void __launch_bounds__(kScatterThreads) permute_small_kernel(
+    const int32_t* __restrict__ ids, const uint16_t* __restrict__ x, int T, int H, int k, int E, int n_shared,
+    int64_t A, int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+    void* __restrict__ x_perm, float* __restrict__ x_scale, int* status, int* zero, size_t zero_words) {
+    extern __shared__ int32_t sm_small[];
+    const int G = E + n_shared;
+    int32_t* s_ids = sm_small;             // [T*k]
+    int32_t* s_cnt = s_ids + T * k;        // [G]
+    int32_t* s_off = s_cnt + G;            // [G+1]
+    int32_t* s_mark = s_off + G + 1;       // [E]: 1 + slot of this token routed to e, else 0
+    __shared__ int s_dst[32];
+    __shared__ int s_rank[32];
+    pdl_trigger();
+    for (int g = threadIdx.x; g < G; g += blockDim.x) s_cnt[g] = g < E ? 0 : T;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_mark[e] = 0;
+    if (threadIdx.x < 32) s_rank[threadIdx.x] = 0;
+    pdl_wait();
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < zero_words; i += (size_t)gridDim.x * blockDim.x)
+        zero[i] = 0;
+    const int t = blockIdx.x;
+    __syncthreads();
+    for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
+        const int e = ids[i];
+        s_ids[i] = e;
+        if (e >= 0 && e < E) atomicAdd(&s_cnt[e], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x < k) {  // this token's slots: valid and distinct
+        const int j = threadIdx.x, e = s_ids[t * k + j];
+        bool good = e >= 0 && e < E;
+        for (int j2 = 0; j2 < j && good; ++j2) good = s_ids[t * k + j2] != e;
+        if (!good) set_status(status, MOE_ERR_EXPERT_ID);
+        else s_mark[e] = j + 1;  // distinct valid ids: one writer per expert
+    }
+    block_exclusive_scan_256(s_cnt, G, s_off);
+    __syncthreads();
+    for (int i = threadIdx.x; i < t * k; i += blockDim.x) {  // earlier tokens' rows of this token's experts
+        const int e = s_ids[i];
+        if (e >= 0 && e < E) {
+            const int m = s_mark[e];
+            if (m) atomicAdd(&s_rank[m - 1], 1);
+        }
+    }
+    if (t == 0)
+        for (int g = threadIdx.x; g <= G; g += blockDim.x) offsets[g] = s_off[g];
+    __syncthreads();
+    const int nd = k + n_shared;
+    if (threadIdx.x < nd) {
+        const int d = threadIdx.x;
+        int64_t dst = -1;
+        if (d < k) {
+            const int e = s_ids[t * k + d];
+            if (e >= 0 && e < E && s_mark[e] == d + 1) dst = (int64_t)s_off[e] + s_rank[d];
+        } else {
+            dst = (int64_t)s_off[E + (d - k)] + t;
+        }
+        if (dst >= A) {
+            set_status(status, MOE_ERR_EXPERT_ID);
+            dst = -1;
+        }
+        s_dst[d] = (int)dst;
+        if (d < k) inv[(size_t)t * k + d] = (int)dst;
+        if (dst >= 0) perm[dst] = t;
+    }
+    __syncthreads();
+    scatter_row<FP8>(x, t, H, nd, s_dst, x_perm, x_scale, A);
+}
+
 cudaError_t launch_permute(const int32_t* ids, const void* x, int T, int H, int k, int E, int n_shared, bool fp8,
                            int32_t* offsets, int32_t* perm, int32_t* inv, void* x_perm, float* x_scale,
                            void* scratch, unsigned int* counter, int* status, cudaStream_t stream, int* zero,
@@ -221,6 +303,18 @@ cudaError_t launch_permute(const int32_t* ids, const void* x, int T, int H, int 
     if (T == 0) return cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (G + 1), stream);
     if (G > kMaxGroups) return cudaErrorInvalidValue;
     const int nchunk = (T + kChunk - 1) / kChunk;
+    const int64_t A = (int64_t)T * (k + n_shared);
+    if (nchunk == 1) {  // one launch: counting, scan and scatter per token
+        const size_t sm = sizeof(int32_t) * ((size_t)T * k + 2 * (size_t)G + 1 + (size_t)E);
+        if (sm > 48 * 1024) {
+            cudaError_t e2 = cudaFuncSetAttribute(fp8 ? permute_small_kernel<true> : permute_small_kernel<false>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+            if (e2 != cudaSuccess) return e2;
+        }
+        return launch_pdl(fp8 ? permute_small_kernel<true> : permute_small_kernel<false>, dim3(T), dim3(kScatterThreads),
+                          sm, stream, ids, static_cast<const uint16_t*>(x), T, H, k, E, n_shared, A, offsets, perm,
+                          inv, x_perm, x_scale, status, zero, zero ? zero_words : (size_t)0);
+    }
     int32_t* cnt = static_cast<int32_t*>(scratch);
     int32_t* rank = reinterpret_cast<int32_t*>(static_cast<char*>(scratch) +
                                                (((size_t)nchunk * E * sizeof(int32_t) + 255) & ~size_t(255)));
@@ -233,7 +327,6 @@ cudaError_t launch_permute(const int32_t* ids, const void* x, int T, int H, int 
     err = launch_pdl(permute_count_kernel, dim3(nchunk), dim3(256), sm1, stream, ids, T, k, E, n_shared, cnt, rank,
                      offsets, counter, status, zero, zero ? zero_words : (size_t)0);
     if (err != cudaSuccess) return err;
-    const int64_t A = (int64_t)T * (k + n_shared);
     return launch_pdl(fp8 ? permute_scatter_kernel<true> : permute_scatter_kernel<false>, dim3(T), dim3(kScatterThreads),
                       0, stream, ids, static_cast<const int32_t*>(rank), static_cast<const int32_t*>(cnt), offsets,
                       static_cast<const uint16_t*>(x), T, H, k, E, n_shared, A, perm, inv, x_perm, x_scale, status);
