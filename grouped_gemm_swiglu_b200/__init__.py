@@ -13,12 +13,12 @@ from ._lib import (MOE_OK, MOE_SCORE_SIGMOID, MOE_SCORE_SOFTMAX, MOE_WDTYPE_BF16
                    MOE_WDTYPE_INT4_G32, MOE_WDTYPE_NVFP4,
                    MOE_WS_COMBINE, MOE_WS_EXPERTS, MOE_WS_FORWARD, MOE_WS_GEMM1, MOE_WS_GEMM2_COMBINE,
                    MOE_WS_GATE_ROUTE, MOE_WS_PERMUTE, MoeDims, MoeError, alloc_workspace, header_functions, lib,
-                   MOE_OPT_FP8_CTA_PAIR, moe_abi_version, moe_clear_status, moe_set_option, moe_combine, moe_ep_rebase, moe_ep_row_ids, moe_experts,
+                   MOE_OPT_FP8_CTA_PAIR, MOE_OPT_BF16_CTA_PAIR, moe_abi_version, moe_clear_status, moe_set_option, moe_combine, moe_ep_rebase, moe_ep_row_ids, moe_experts,
                    moe_forward, moe_gate_route, moe_gemm1_swiglu, moe_gemm2_combine,
                    moe_permute, moe_permute_noalloc, moe_read_status, moe_route_topk, moe_workspace_size,
                    status_string)
 
-__all__ = ["MoeDims", "MoeError", "MoELayer", "moe_abi_version", "moe_set_option", "MOE_OPT_FP8_CTA_PAIR", "moe_workspace_size", "moe_read_status",
+__all__ = ["MoeDims", "MoeError", "MoELayer", "moe_abi_version", "moe_set_option", "MOE_OPT_FP8_CTA_PAIR", "MOE_OPT_BF16_CTA_PAIR", "moe_workspace_size", "moe_read_status",
            "moe_clear_status", "moe_route_topk", "moe_gate_route", "moe_permute", "moe_permute_noalloc", "moe_gemm1_swiglu",
            "moe_gemm2_combine", "moe_experts", "moe_combine", "moe_forward", "moe_ep_row_ids", "moe_ep_rebase",
            "alloc_workspace", "status_string", "lib",

@@ -138,6 +138,7 @@ def moe_abi_version() -> int:
 
 
 MOE_OPT_FP8_CTA_PAIR = 1
+MOE_OPT_BF16_CTA_PAIR = 2
 
 
 def moe_set_option(option: int, value: int) -> int:

@@ -201,6 +201,7 @@ int moe_abi_version(void) { return MOE_ABI_VERSION; }
 
 int moe_set_option(int option, int value) {
     if (option == MOE_OPT_FP8_CTA_PAIR && (value == 0 || value == 1)) return gemm_set_fp8_pair(value);
+    if (option == MOE_OPT_BF16_CTA_PAIR && (value == 0 || value == 1)) return gemm_set_bf16_pair(value);
     return MOE_ERR_INVALID_ARG;
 }
 

@@ -72,8 +72,10 @@ struct Cfg {
     // Two CTAs of a cluster share each MMA (cta_group::2, M = 256 token rows): each CTA
     // loads its own 128 token rows and half of the 256 weight rows (the gate rows in the
     // even CTA, the up rows in the odd one; GEMM2: one 128-row chunk of H each), so a CTA
-    // pulls 32 KB through L2 per 128-deep K block instead of 48 KB. A token block is then
-    // TB = 256 rows of a group.
+    // pulls 32 KB through L2 per 128-byte K step instead of 48 KB. A token block is then
+    // TB = 256 rows of a group. FP8 or bf16 (for bf16 the tile's partial sums stay in
+    // TMEM over the whole K range, so each tile drains one of two TMEM buffers while the
+    // tensor core fills the other).
     static constexpr bool PAIR = PAIR_;
     static constexpr int TB = PAIR ? 2 * BN : BN;  // token rows per block
     // INT4 group-32 weights: TMA brings the packed bytes (RAW_BYTES per 128x64 block) and
@@ -107,7 +109,7 @@ struct Cfg {
     // as many stages as fit next to the control block and the largest group table
     // wide FP8 tile (FP8 at 128 tokens): 2 KB per epilogue warp to turn its token rows into
     // row-contiguous stores (16 rows x 128 bytes at a time)
-    static constexpr int XPOSE_BYTES = (FP8_ && BN_ >= 128) ? 8 * 2048 : 0;
+    static constexpr int XPOSE_BYTES = ((FP8_ && BN_ >= 128) || PAIR_) ? 8 * 2048 : 0;
     static constexpr int STAGE_BUDGET =
         kSmemLimit - 1024 - 8 * (kMaxGroupsGemm + 1) - 1024 - 4 * 16 * 16 * 3 - XPOSE_BYTES;
     static constexpr int ACC_COLS = 2 * BN;  // one TMEM buffer: gate | up (GEMM2 uses the first BN)
@@ -130,12 +132,14 @@ struct Cfg {
     // GEMM1 tiles, an idle warp) one warpgroup, which gives registers back (setmaxnreg) to
     // the epilogue warpgroups: the launch's threads x registers cover 4 warps at REG_LOW
     // and WEPI epilogue warps at REG_HIGH.
-    static constexpr bool WIDE = FP8 && BN >= 128;
+    static constexpr bool WIDE = (FP8 && BN >= 128) || PAIR;  // token-major (FP8 at 128 tokens, or a pair)
     static constexpr int WEPI = 8;  // wide FP8 epilogue warps: 8 (128 sums each) or 16 (64)
     static constexpr int EPI = WIDE ? WEPI : (BN >= 256 ? 16 : ((INT4 && BN <= 32) ? 4 : 8));
     static constexpr int EPI0 = WIDE ? 4 : 2;  // first epilogue warp
     static constexpr int REG_LAUNCH = WIDE ? (65536 / (32 * (4 + WEPI))) / 8 * 8 : 0;
-    static constexpr int REG_LOW = 56, REG_HIGH = WEPI == 8 ? 224 : 104;
+    // (the bf16 pair's epilogue holds no promotion sums: its producer and MMA loops get more)
+    static constexpr int REG_LOW = (PAIR && !FP8) ? 88 : 56;
+    static constexpr int REG_HIGH = WEPI == 8 ? ((PAIR && !FP8) ? 208 : 224) : 104;
     static constexpr int WCH = 16;  // wide FP8: TMEM columns per load of each half
     static constexpr int THREADS = 32 * EPI0 + 32 * EPI + 32 * DQ;
     static constexpr int GROUPS = EPI / 4;
@@ -156,7 +160,7 @@ struct Cfg {
     static_assert(BN % BOX_ROWS == 0 && BN <= 256, "token tile = whole boxes, at most the MMA's N limit");
     static_assert(STAGES >= 2, "at least two pipeline stages");
     static_assert(!(INT4 && FP8), "INT4 weights take bf16 activations");
-    static_assert(!PAIR || (FP8 && WIDE && BN == 128), "the CTA pair is the token-major FP8 tile");
+    static_assert(!PAIR || (WIDE && BN == 128 && !INT4), "the CTA pair is a token-major tile of 2 x 128 rows");
     static_assert(!INT4 || BN <= 64, "INT4 keeps its A tiles next to the accumulators in TMEM");
     static_assert(!INT4 || (DQG == 4 && DQG * NGRP == DQ), "dequantisation warps: stage groups of 4");
     static_assert(COLS % 8 == 0, "split-K merges columns in chunks of 8");
@@ -164,7 +168,7 @@ struct Cfg {
     // every tile width except FP8 from 64 columns, whose promotion registers are full,
     // and 256 columns, whose merge path alone would push the kernel past its register
     // cap (a 256-column tile means large groups, which never need a split).
-    static constexpr bool SPLIT_OK = !(FP8 && BN >= 64) && BN < 256;
+    static constexpr bool SPLIT_OK = !(FP8 && BN >= 64) && BN < 256 && !PAIR;
 
     // full/empty per stage, tfull/tempty per TMEM buffer, ring_full/ring_empty x kRing, drain,
     // epibar, and for INT4 raw_full per stage (packed bytes and token rows landed)
@@ -746,7 +750,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     const int n_mma = max(16, (tl.nrows + 15) & ~15);
                     // wide FP8: M = the 128 token rows, N = the 256 (or 128) weight rows
                     // pair: M = 2 x 128 token rows, N = 2 x 128 weight rows (one block from each CTA)
-                    const uint32_t idesc = C::PAIR ? idesc_m256_fp8(256)
+                    const uint32_t idesc = C::PAIR ? idesc_m256(256, C::FP8)
                                                    : (C::WIDE ? idesc_m128(tl.dual ? 256 : 128, true)
                                                               : idesc_m128(n_mma, C::FP8));
                     // bf16: one TMEM buffer per tile; FP8: one per 128-deep K block
@@ -783,7 +787,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                     if (tl.dual) mma_bf16_tmem_a(d0 + C::BN, at + 32 + kk * 8, bd, idesc, acc);
                                 } else if constexpr (C::PAIR) {
                                     // token tiles (A, 128 rows per CTA) x weight blocks (B, 128 rows per CTA)
-                                    mma_fp8_pair(d0, bd, smem_desc_sw128(a0 + kk * 32), idesc, acc);
+                                    if constexpr (C::FP8) mma_fp8_pair(d0, bd, smem_desc_sw128(a0 + kk * 32), idesc, acc);
+                                    else mma_bf16_pair(d0, bd, smem_desc_sw128(a0 + kk * 32), idesc, acc);
                                 } else if constexpr (C::WIDE) {
                                     // the token tile is the A operand; A0 | A1 (contiguous) the B operand
                                     mma_fp8(d0, bd, smem_desc_sw128(a0 + kk * 32), idesc, acc);
@@ -977,7 +982,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const float sg = (g1 && p.gate_scale) ? __ldg(p.gate_scale + tl.g) : 1.f;
             const float su = (g1 && p.up_scale) ? __ldg(p.up_scale + tl.g) : 1.f;
             const float lim = (g1 && p.limits) ? __ldg(p.limits + tl.g) : p.limit;  // this expert's clamp
-            if constexpr (!C::FP8) {
+            if constexpr (!C::FP8 && !C::WIDE) {
                 const uint32_t buf = it % C::NBUF, bph = (it / C::NBUF) & 1;
                 if (!warp_wait(&tfull[buf], bph, ab, p.status)) {
                     ok = false;
@@ -1066,6 +1071,86 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         }
                     }
                 }
+            } else if constexpr (C::WIDE && !C::FP8) {
+                // Token-major bf16 tile (CTA pair): TMEM lane = token row, columns = this
+                // tile's 256 weight rows (gate | up, or two 128-row chunks of H), summed over
+                // the whole K range in one buffer. This warp takes columns cg*CC .. +CC of
+                // each half and writes its token's row piece of h (SwiGLU of the per-group
+                // scaled gate and up) or of y, 16 bytes at a time, row-contiguously.
+                constexpr int CC = C::COLS;
+                constexpr int W = 16;
+                const bool quarter_live = q * 32 < tl.nrows;  // warp-uniform
+                const uint32_t buf = it % C::NBUF, bph = (it / C::NBUF) & 1;
+                if (!warp_wait<C::PAIR>(&tfull[buf], bph, ab, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t tb = tmem_base + lane_off + buf * C::ACC_COLS + cg * CC;
+                auto release = [&]() {  // the buffer goes back to the MMA (pair: to rank 0)
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if constexpr (C::PAIR) mbar_arrive_remote(lead(&tempty[buf]));
+                        else mbar_arrive(&tempty[buf]);
+                    }
+                };
+                if (!quarter_live) {
+                    release();  // no token of this lane quarter in the tile
+                } else if (g1) {
+                    uint4 hv[CC / 8];  // this token's CC values of h, 8 bf16 per piece
+#pragma unroll
+                    for (int ch = 0; ch < CC / W; ++ch) {
+                        float gv[W], uv[W];
+                        tmem_ld_x2<W>(tb + ch * W, tb + C::BN + ch * W, gv, uv);
+                        if (ch == CC / W - 1) release();  // before the arithmetic
+#pragma unroll
+                        for (int v = 0; v < W / 8; ++v) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                const int j = v * 8 + 2 * t;
+                                const float h0 = swiglu_dev(sg * gv[j], su * uv[j], p.alpha, p.beta, lim);
+                                const float h1 = swiglu_dev(sg * gv[j + 1], su * uv[j + 1], p.alpha, p.beta, lim);
+                                const __nv_bfloat162 b = __floats2bfloat162_rn(h0, h1);
+                                w[t] = *reinterpret_cast<const uint32_t*>(&b);
+                            }
+                            hv[ch * (W / 8) + v] = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                    store_rows<CC / 8>(xpose + ew * 2048, hv,
+                                       static_cast<uint8_t*>(p.h) + 2 * (size_t)(tl.col0 + cg * CC), 2 * (size_t)p.I,
+                                       tl.row0 + q * 32, tl.nrows - q * 32, lane);
+                } else {
+                    // y rows (H % 128 == 0, y 16-byte aligned): this token's CC bf16 of each half
+                    uint8_t* ybase = static_cast<uint8_t*>(p.y);
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        if (half == 1 && !tl.dual) break;  // the second block's columns are not stored
+                        uint4 yv[CC / 8];
+#pragma unroll
+                        for (int ch = 0; ch < CC / W; ++ch) {
+                            float v[W];
+                            tmem_ld_x1<W>(tb + half * C::BN + ch * W, v);
+#pragma unroll
+                            for (int u = 0; u < W / 8; ++u) {
+                                uint32_t w[4];
+#pragma unroll
+                                for (int t = 0; t < 4; ++t) {
+                                    const __nv_bfloat162 b =
+                                        __floats2bfloat162_rn(v[u * 8 + 2 * t], v[u * 8 + 2 * t + 1]);
+                                    w[t] = *reinterpret_cast<const uint32_t*>(&b);
+                                }
+                                yv[ch * (W / 8) + u] = make_uint4(w[0], w[1], w[2], w[3]);
+                            }
+                        }
+                        if (half == 1 || !tl.dual) release();  // after the tile's last TMEM load
+                        const int colb = (half ? tl.col1 : tl.col0) + cg * CC;  // first bf16 column
+                        store_rows<CC / 8>(xpose + ew * 2048, yv, ybase + 2 * (size_t)colb, 2 * (size_t)p.H,
+                                           tl.row0 + q * 32, tl.nrows - q * 32, lane);
+                    }
+                }
+                ++it;
             } else if constexpr (C::WIDE) {
                 // Token-major FP8 tile: TMEM lane = token row of the block, columns = weight
                 // rows (gate | up, or two 128-row chunks of H). This warp takes columns
@@ -1648,19 +1733,25 @@ static cudaError_t launch_cfg(const MoeGemmArgs& a, cudaStream_t stream) {
     }
 }
 
-static std::atomic<int> g_fp8_pair{0};  // MOE_OPT_FP8_CTA_PAIR
+static std::atomic<int> g_fp8_pair{0};   // MOE_OPT_FP8_CTA_PAIR
+static std::atomic<int> g_bf16_pair{0};  // MOE_OPT_BF16_CTA_PAIR
 
 int gemm_set_fp8_pair(int enable) { return g_fp8_pair.exchange(enable ? 1 : 0); }
+int gemm_set_bf16_pair(int enable) { return g_bf16_pair.exchange(enable ? 1 : 0); }
+
+// A pair needs two GEMM1 completion counters per 256-row block within the workspace's
+// block flags (true whenever groups average more than 128 rows).
+static bool pair_flags_fit(int64_t A, int G) {
+    return 2 * gemm_max_blocks(A, G, 256) + 1 <= gemm_max_blocks(A, G, 16) + 1;
+}
 
 int gemm_pick_bn(int64_t A, int G, int wdtype) {
     const double avg = G > 0 ? (double)A / (double)G : 0.0;
     int bn = 16;
     while (bn < 256 && bn < avg) bn <<= 1;  // smallest tile holding an average group
     // FP8 above 128 rows: the 128-token tile, or (when chosen) the CTA pair at "256" (2 x
-    // 128 token rows), which needs two GEMM1 completion counters per 256-row block within
-    // the workspace's block flags (true whenever groups average more than 128 rows)
-    if (wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128 && bn > 128 &&
-        (!g_fp8_pair.load() || 2 * gemm_max_blocks(A, G, 256) + 1 > gemm_max_blocks(A, G, 16) + 1))
+    // 128 token rows)
+    if (wdtype == MOE_WDTYPE_FP8_E4M3_BLOCK128 && bn > 128 && (!g_fp8_pair.load() || !pair_flags_fit(A, G)))
         bn = 128;
     if ((wdtype == MOE_WDTYPE_INT4_G32 || wdtype == MOE_WDTYPE_NVFP4) && bn > 64)
         bn = 64;  // 4-bit weights: A tiles share TMEM with the accumulators
@@ -1730,7 +1821,9 @@ cudaError_t launch_moe_gemm(const MoeGemmArgs& a, cudaStream_t stream) {
         case 32: return launch_cfg<Cfg<32, false>>(a, stream);
         case 64: return launch_cfg<Cfg<64, false>>(a, stream);
         case 128: return launch_cfg<Cfg<128, false>>(a, stream);
-        case 256: return launch_cfg<Cfg<256, false>>(a, stream);
+        case 256:  // 256-row token blocks: one CTA, or (when chosen) the token-major CTA pair
+            if (g_bf16_pair.load() && pair_flags_fit(a.A, a.G)) return launch_cfg<Cfg<128, false, false, true>>(a, stream);
+            return launch_cfg<Cfg<256, false>>(a, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -104,6 +104,8 @@ struct MoeGemmArgs {
 int gemm_pick_bn(int64_t A, int G, int wdtype);
 // Process-wide choice of the FP8 CTA-pair layout (moe_set_option): returns the old value.
 int gemm_set_fp8_pair(int enable);
+// The same for bf16 layers with 256-row token blocks (MOE_OPT_BF16_CTA_PAIR).
+int gemm_set_bf16_pair(int enable);
 // Upper bound on token blocks: every non-empty group adds at most one partial block.
 int64_t gemm_max_blocks(int64_t A, int G, int bn);
 size_t gemm_block_flags_bytes(int64_t A, int G);

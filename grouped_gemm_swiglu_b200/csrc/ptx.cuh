@@ -531,12 +531,25 @@ __device__ __forceinline__ void mma_fp8_pair(uint32_t d_tmem, uint64_t a_desc, u
         : "memory");
 }
 
-// Instruction descriptor of the pair MMA: D fp32, E4M3 A/B K-major, M = 256, N = n.
-__device__ __forceinline__ uint32_t idesc_m256_fp8(int n) {
+// Pair MMA, bf16 operands, fp32 accumulate (K = 16 per instruction), same operand split.
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Instruction descriptor of the pair MMA: D fp32, A/B K-major (E4M3, or bf16 for
+// kind::f16), M = 256, N = n.
+__device__ __forceinline__ uint32_t idesc_m256(int n, bool fp8) {
     uint32_t d = 0;
-    d |= 1u << 4;                     // D format: f32
-    d |= (uint32_t)(n >> 3) << 17;    // N >> 3
-    d |= (uint32_t)(256 >> 4) << 24;  // M >> 4
+    d |= 1u << 4;                           // D format: f32
+    if (!fp8) d |= (1u << 7) | (1u << 10);  // A, B: bf16
+    d |= (uint32_t)(n >> 3) << 17;          // N >> 3
+    d |= (uint32_t)(256 >> 4) << 24;        // M >> 4
     return d;
 }
 

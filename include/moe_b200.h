@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 6
+#define MOE_ABI_VERSION 7
 
 typedef enum moe_status {
     MOE_OK = 0,
@@ -140,9 +140,19 @@ int moe_abi_version(void);
  *        blocks, so each SM moves a third fewer bytes from L2. Measured on the GLM-shaped
  *        FP8 prefill it runs at the same speed as the default (2.67 against 2.61 ms).
  *     Results agree to the FP8 tolerance, not necessarily bit for bit (the tensor core's
- *     summation order within a K block may differ between the two layouts). */
+ *     summation order within a K block may differ between the two layouts).
+ *   MOE_OPT_BF16_CTA_PAIR: bf16 layers whose groups average more than 128 rows (256-row
+ *     token blocks).
+ *     0 (default): one CTA per 256-token tile with the weight rows as the MMA's M side;
+ *        the tile's gate and up sums fill all of tensor memory, so the tensor core waits
+ *        while the epilogue drains them.
+ *     1: a CTA pair per 256-token tile with the token rows as M (128 per CTA) and each CTA
+ *        loading one of the two 128-row weight blocks: the same bytes per SM from L2, and
+ *        two accumulator buffers, so one tile's drain overlaps the next tile's MMAs.
+ *     Results agree to the bf16 tolerance (the summation order may differ). */
 typedef enum moe_option {
-    MOE_OPT_FP8_CTA_PAIR = 1
+    MOE_OPT_FP8_CTA_PAIR = 1,
+    MOE_OPT_BF16_CTA_PAIR = 2
 } moe_option;
 
 /* Sets a process-wide option for calls made after it returns (a CUDA graph keeps the

@@ -96,3 +96,24 @@ class fp8_layout:
         import grouped_gemm_swiglu_b200 as moe
         moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, self.old)
         return False
+
+
+class pair_layout:
+    """Within the block, layers whose groups average more than 128 rows run in the given
+    layout, FP8 and bf16 alike: pair=True selects the two-CTA tiles
+    (MOE_OPT_FP8_CTA_PAIR and MOE_OPT_BF16_CTA_PAIR)."""
+
+    def __init__(self, pair: bool):
+        self.pair = pair
+
+    def __enter__(self):
+        import grouped_gemm_swiglu_b200 as moe
+        v = 1 if self.pair else 0
+        self.old = (moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, v), moe.moe_set_option(moe.MOE_OPT_BF16_CTA_PAIR, v))
+        return self
+
+    def __exit__(self, *exc):
+        import grouped_gemm_swiglu_b200 as moe
+        moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, self.old[0])
+        moe.moe_set_option(moe.MOE_OPT_BF16_CTA_PAIR, self.old[1])
+        return False

@@ -26,7 +26,7 @@ def test_every_header_function_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert moe.moe_abi_version() == 6
+    assert moe.moe_abi_version() == 7
     for code in range(-7, 1):
         assert moe.status_string(code)
     assert "unknown" in moe.status_string(-99)
@@ -188,3 +188,12 @@ def test_set_option_returns_the_previous_value_and_rejects_unknown_ones(L):
         assert moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, 0) == 0  # the refusals changed nothing
     finally:
         moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, old)
+    old_b = moe.moe_set_option(moe.MOE_OPT_BF16_CTA_PAIR, 1)
+    try:  # the two options are independent
+        assert old_b in (0, 1)
+        assert moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, old) == old
+        assert moe.moe_set_option(moe.MOE_OPT_BF16_CTA_PAIR, 0) == 1
+        assert L.moe_set_option(moe.MOE_OPT_BF16_CTA_PAIR, -1) == -1
+        assert moe.moe_set_option(moe.MOE_OPT_BF16_CTA_PAIR, 0) == 0
+    finally:
+        moe.moe_set_option(moe.MOE_OPT_BF16_CTA_PAIR, old_b)

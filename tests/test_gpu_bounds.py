@@ -12,7 +12,7 @@ import torch
 
 import grouped_gemm_swiglu_b200 as moe
 from grouped_gemm_swiglu_b200 import workloads as W
-from helpers import assert_bf16_close, assert_fp8_close, fp8_layout, oracle_layer
+from helpers import assert_bf16_close, assert_fp8_close, oracle_layer, pair_layout
 
 pytestmark = pytest.mark.gpu
 
@@ -38,6 +38,10 @@ SHAPES = [
     # shared group's second block has 44 rows, so one CTA of that pair holds none
     W.Workload("t300_fp8_pair", T=300, H=512, I=384, E=4, k=2, n_shared=1, wdtype=W.WDTYPE_FP8,
                score=W.SCORE_SIGMOID, limit=10.0),
+    # the same groups in bf16 (256-row token blocks): the token-major bf16 CTA pair, with
+    # the OAI SwiGLU parameters
+    W.Workload("t300_bf16_pair", T=300, H=512, I=384, E=4, k=2, n_shared=1, score=W.SCORE_SOFTMAX,
+               alpha=1.702, beta=1.0, limit=7.0),
 ]
 
 
@@ -65,7 +69,7 @@ def guarded_ws(d, kind):
 
 @pytest.mark.parametrize("wl", SHAPES, ids=[w.name for w in SHAPES])
 def test_outputs_stay_in_bounds_and_match_the_oracle(wl):
-    with fp8_layout(pair=wl.name.endswith("_pair")):  # the *_pair shape in the CTA-pair layout
+    with pair_layout(pair=wl.name.endswith("_pair")):  # the *_pair shapes in the CTA-pair layouts
         _check_bounds(wl)
 
 

@@ -8,7 +8,7 @@ import torch
 import oracle
 import grouped_gemm_swiglu_b200 as moe
 from grouped_gemm_swiglu_b200 import workloads as W
-from helpers import assert_bf16_close, assert_fp8_close, f32, fp8_layout, oracle_layer, sample_tokens
+from helpers import assert_bf16_close, assert_fp8_close, f32, fp8_layout, oracle_layer, pair_layout, sample_tokens
 
 pytestmark = pytest.mark.gpu
 
@@ -63,6 +63,35 @@ def test_forward_fp8_large_groups_every_token(pair):
     assert layer.status() == 0
     ref = oracle_layer(wl, inp).moe_rows(np.arange(wl.T, dtype=np.int32))
     assert_fp8_close(out.float().cpu().numpy(), ref, wl.name)
+
+
+# bf16 with groups of about 500 rows (256-row token blocks, ragged tails), per-expert
+# gate/up scales and a shared expert, in both layouts of 256-row bf16 tiles
+LARGE_BF16 = W.Workload("bf16_t1024_large_groups", T=1024, H=1024, I=512, E=16, k=8, n_shared=1,
+                        score=W.SCORE_SOFTMAX, expert_scales=(0.52, 1.22))
+
+
+@pytest.mark.parametrize("pair", [False, True], ids=["cta256", "cta_pair"])
+def test_forward_bf16_large_groups_every_token(pair):
+    wl = LARGE_BF16
+    inp = W.make_inputs(wl, "cuda")
+    with pair_layout(pair):
+        out, ids, tw, sw, layer = run_forward(wl, inp)
+    assert layer.status() == 0
+    ref = oracle_layer(wl, inp).moe_rows(np.arange(wl.T, dtype=np.int32))
+    assert_bf16_close(out.float().cpu().numpy(), ref, wl.name)
+
+
+def test_forward_qwen3_bf16_cta_pair_sampled():
+    """The full Qwen3-shaped bf16 prefill in the token-major CTA-pair layout (sampled tokens)."""
+    wl = W.WORKLOADS["qwen3_30b_a3b"]
+    inp = W.make_inputs(wl, "cuda")
+    with pair_layout(True):
+        out, ids, tw, sw, layer = run_forward(wl, inp)
+    assert layer.status() == 0
+    toks = sample_tokens(wl.T, 32, seed=3)
+    ref = oracle_layer(wl, inp).moe_rows(toks)
+    assert_bf16_close(out.float().cpu().numpy()[toks], ref, "qwen3_30b_a3b (CTA pair)")
 
 
 def test_forward_glm_fp8_cta_pair_sampled():

@@ -1,7 +1,7 @@
 """Grouped GEMM1 (+ SwiGLU epilogue) and GEMM2 (+ weighted combine) on the GPU against
 the oracle, on synthetic permuted inputs that span several tiles, every token-tile width
-(16/32/64/128/256 rows, and FP8's two-CTA 256-row pair), ragged group tails, empty groups
-and shared groups."""
+(16/32/64/128/256 rows, and the FP8 and bf16 two-CTA 256-row pairs), ragged group tails,
+empty groups and shared groups."""
 import math
 
 import numpy as np
@@ -11,7 +11,7 @@ import torch
 import oracle
 import grouped_gemm_swiglu_b200 as moe
 from grouped_gemm_swiglu_b200 import workloads as W
-from helpers import assert_bf16_close, assert_fp8_close, bits16, e4m3_to_np, f32, fp8_layout, u8
+from helpers import assert_bf16_close, assert_fp8_close, bits16, e4m3_to_np, f32, fp8_layout, pair_layout, u8
 
 pytestmark = pytest.mark.gpu
 
@@ -108,6 +108,10 @@ GEMM1_CASES = [
     # blocks); a shared group of T rows
     (1500, 16, 2, 1, 512, 256, True, {"skew": 4.0, "oai": True}),
     (700, 4, 2, 0, 1024, 384, True, {"scales": True, "limits": True}),
+    # bf16 with groups above 128 rows on average (256-row token blocks: one CTA, or the
+    # token-major CTA pair), heavy skew, a shared group of T rows, OAI parameters
+    (1500, 16, 2, 1, 512, 256, False, {"skew": 4.0, "oai": True}),
+    (700, 4, 2, 0, 1024, 384, False, {"scales": True, "limits": True}),
     (128, 8, 2, 1, 512, 384, False, {"limits": True}),          # a clamp per expert (shared group too)
     (300, 16, 4, 0, 512, 256, True, {"limits": True, "scales": True}),  # FP8, tile 32, clamp per expert
     (8, 64, 4, 0, 256, 256, False, {"int4": True}),            # INT4 group-32 weights: tile 16, split-K
@@ -134,6 +138,21 @@ def _pairable(T, E, k, S, fp8):
 
 
 GEMM1_PAIR = [c for c in GEMM1_CASES if _pairable(*c[:4], c[6])]
+
+
+def _bf16_pairable(T, E, k, S, fp8, extra=None):
+    """bf16 cases whose groups average more than 128 rows (256-row token blocks)."""
+    extra = extra or {}
+    return fp8 is False and not extra.get("int4") and not extra.get("fp4") and T * (k + S) / (E + S) > 128
+
+
+GEMM1_BF16_PAIR = [c for c in GEMM1_CASES if _bf16_pairable(*c[:4], c[6], c[7])]
+
+
+@pytest.mark.parametrize("T,E,k,S,H,I,fp8,extra", GEMM1_BF16_PAIR)
+def test_gemm1_swiglu_bf16_cta_pair(T, E, k, S, H, I, fp8, extra):
+    with pair_layout(True):
+        test_gemm1_swiglu(T, E, k, S, H, I, fp8, extra)
 
 
 @pytest.mark.parametrize("T,E,k,S,H,I,fp8,extra", GEMM1_PAIR)
@@ -183,6 +202,7 @@ GEMM2_CASES = [
     (300, 16, 4, 1, 512, 256, False, False),    # one shared group with weight 1
     (1024, 8, 2, 0, 512, 256, False, False),    # tile 256
     (600, 4, 2, 1, 384, 256, False, True),      # tile 256, odd number of 128-row chunks of H
+    (1500, 16, 2, 1, 384, 256, False, False),   # tile 256, skewless large groups, odd chunk count of H
     (512, 8, 2, 0, 512, 256, True, False),      # FP8, tile 128
     (256, 8, 2, 0, 512, 256, True, False),      # FP8, tile 64
     (600, 4, 2, 1, 384, 256, True, True),       # FP8 large groups, odd chunk count of H, sink-gated shared
@@ -205,6 +225,13 @@ GEMM2_CASES = [
 
 
 GEMM2_PAIR = [c for c in GEMM2_CASES if _pairable(*c[:4], c[6])]
+GEMM2_BF16_PAIR = [c for c in GEMM2_CASES if _bf16_pairable(*c[:4], c[6])]
+
+
+@pytest.mark.parametrize("T,E,k,S,H,I,fp8,sinks", GEMM2_BF16_PAIR)
+def test_gemm2_combine_bf16_cta_pair(T, E, k, S, H, I, fp8, sinks):
+    with pair_layout(True):
+        test_gemm2_combine(T, E, k, S, H, I, fp8, sinks)
 
 
 @pytest.mark.parametrize("T,E,k,S,H,I,fp8,sinks", GEMM2_PAIR)

@@ -7,8 +7,9 @@ completion counters (the first words after the 256-byte header) start a million 
 zero, so the GEMM1 tiles' release-adds never bring them to the count the GEMM2 tiles wait
 for. Each GEMM2 tile's bounded wait (about a second) gives up, its CTA drains its copies
 and MMAs, frees tensor memory and leaves. No trap, no invalid address: the same workspace
-then runs the layer normally. Two kernel layouts: the single-CTA bf16 tile, and the FP8
-CTA pair (two CTAs of a cluster sharing each MMA), whose CTAs also wait on each other."""
+then runs the layer normally. Three kernel layouts: the single-CTA bf16 tile, and the FP8
+and bf16 CTA pairs (two CTAs of a cluster sharing each MMA), whose CTAs also wait on each
+other."""
 import time
 
 import numpy as np
@@ -17,7 +18,7 @@ import torch
 
 import grouped_gemm_swiglu_b200 as moe
 from grouped_gemm_swiglu_b200 import workloads as W
-from helpers import assert_bf16_close, assert_fp8_close, fp8_layout, oracle_layer
+from helpers import assert_bf16_close, assert_fp8_close, oracle_layer, pair_layout
 
 pytestmark = pytest.mark.gpu
 
@@ -30,12 +31,14 @@ CASES = [
     # test selects it with moe_set_option)
     W.Workload("fp8_pair", T=300, H=512, I=256, E=4, k=2, n_shared=1, wdtype=W.WDTYPE_FP8,
                score=W.SCORE_SIGMOID, limit=10.0),
+    # the same groups in bf16: the token-major bf16 CTA pair
+    W.Workload("bf16_pair", T=300, H=512, I=256, E=4, k=2, n_shared=1, score=W.SCORE_SIGMOID),
 ]
 
 
 @pytest.mark.parametrize("wl", CASES, ids=[w.name for w in CASES])
 def test_a_wait_that_never_completes_reports_timeout_and_the_context_survives(wl):
-    with fp8_layout(pair=wl.name.endswith("_pair")):  # the FP8 case in the CTA-pair layout
+    with pair_layout(pair=wl.name.endswith("_pair")):  # the *_pair cases in the CTA-pair layouts
         _check_timeout(wl)
 
 
