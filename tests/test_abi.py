@@ -197,3 +197,19 @@ def test_set_option_returns_the_previous_value_and_rejects_unknown_ones(L):
         assert moe.moe_set_option(moe.MOE_OPT_BF16_CTA_PAIR, 0) == 0
     finally:
         moe.moe_set_option(moe.MOE_OPT_BF16_CTA_PAIR, old_b)
+
+
+@pytest.mark.parametrize("name", ["qwen3_30b_a3b", "glm_fp8", "oai_swiglu", "decode_t64"])
+def test_layout_options_need_no_other_workspace(L, name):
+    """The CTA-pair layouts run inside the workspace sized without them (their second
+    GEMM1 completion counter per 256-row block fits the block flags; otherwise the
+    single-CTA tile runs): moe_workspace_size does not depend on the options."""
+    d = moe.MoeDims.of(W.WORKLOADS[name])
+    kinds = [moe.MOE_WS_FORWARD, moe.MOE_WS_EXPERTS, moe.MOE_WS_GEMM1, moe.MOE_WS_GEMM2_COMBINE]
+    base = [moe.moe_workspace_size(d, k) for k in kinds]
+    old = (moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, 1), moe.moe_set_option(moe.MOE_OPT_BF16_CTA_PAIR, 1))
+    try:
+        assert [moe.moe_workspace_size(d, k) for k in kinds] == base
+    finally:
+        moe.moe_set_option(moe.MOE_OPT_FP8_CTA_PAIR, old[0])
+        moe.moe_set_option(moe.MOE_OPT_BF16_CTA_PAIR, old[1])
