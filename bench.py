@@ -125,6 +125,29 @@ def w_bytes_all(wl) -> float:
     return wl.G * 3 * wl.I * wl.H * welt
 
 
+def kernel_work(wl, offsets):
+    """Algorithmic work of one grouped-GEMM launch (both GEMMs) for group offsets [G+1]:
+    FLOPs 2*A*H*2I + 2*A*I*H over the A permuted rows; bytes = the weights (and block or
+    group scales) of every group with at least one row, each read once; and, apart, the
+    implementation's own traffic: x_perm read, h written and read back (+ FP8 scales), y
+    written. Returns (flops, weight_bytes, impl_bytes)."""
+    used = int(((offsets[1:] - offsets[:-1]) > 0).sum())
+    A = int(offsets[-1])
+    fp8 = wl.wdtype == 1
+    H, I = wl.H, wl.I
+    elt = 1 if fp8 else 2  # activations (x_perm, h)
+    # weight bytes per element: INT4 a nibble + a bf16 scale per 32; NVFP4 a nibble + an E4M3 scale per 16
+    welt = {2: 0.5 + 2.0 / 32, 3: 0.5 + 1.0 / 16}.get(wl.wdtype, elt)
+    flops = 2.0 * A * H * 2 * I + 2.0 * A * I * H
+    w_bytes = used * 3 * I * H * welt
+    if fp8:
+        w_bytes += used * ((2 * I // 128) * (H // 128) + (H // 128) * (I // 128)) * 4
+    impl_bytes = A * H * elt + 2 * A * I * elt + A * H * 2
+    if fp8:
+        impl_bytes += A * (H // 128 + 2 * (I // 128)) * 4
+    return flops, w_bytes, impl_bytes
+
+
 def stats(xs):
     """mean / median / min of a list of times (ms)."""
     return {"mean": sum(xs) / len(xs), "median": statistics.median(xs), "min": min(xs), "n": len(xs)}
@@ -537,20 +560,11 @@ def run_ours(args):
     # has at least one row, each read once. Its other traffic -- x_perm read, h written and
     # read back, y written -- is the implementation's choice of materialising the
     # intermediates and is reported apart as impl_bytes.
+    hbm, bf16_tf, bf16_sus, peak_src = peaks()
+    H_ = wl.H
     off = offsets.cpu().numpy()
     used = int(((off[1:] - off[:-1]) > 0).sum())
-    hbm, bf16_tf, bf16_sus, peak_src = peaks()
-    elt = 1 if fp8 else 2  # activations (x_perm, h)
-    # weight bytes per element: INT4 a nibble + a bf16 scale per 32; NVFP4 a nibble + an E4M3 scale per 16
-    welt = {2: 0.5 + 2.0 / 32, 3: 0.5 + 1.0 / 16}.get(wl.wdtype, elt)
-    H_, I_ = wl.H, wl.I
-    flops = 2.0 * A * H_ * 2 * I_ + 2.0 * A * I_ * H_
-    w_bytes = used * 3 * I_ * H_ * welt
-    if fp8:
-        w_bytes += used * ((2 * I_ // 128) * (H_ // 128) + (H_ // 128) * (I_ // 128)) * 4
-    impl_bytes = A * H_ * elt + 2 * A * I_ * elt + A * H_ * 2
-    if fp8:
-        impl_bytes += A * (H_ // 128 + 2 * (I_ // 128)) * 4
+    flops, w_bytes, impl_bytes = kernel_work(wl, off)
     t_k = kern_ms / 1e3
     tensor_peak = bf16_tf * (2.0 if fp8 else 1.0)
     tensor_sus = bf16_sus * (2.0 if fp8 else 1.0)
